@@ -1,0 +1,16 @@
+"""Shared test configuration.
+
+Markers:
+  gpu  -- needs a CUDA device (sm_100a); parity tests of the CUDA library.
+Everything unmarked runs on the CPU in a few minutes.
+"""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) CUDA device")
