@@ -1,0 +1,393 @@
+"""Benchmark of the Gated DeltaNet-2 recurrence on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Headline: chunkwise prefill tokens/s on the
+4K-token workload B=4, T=4096, H=16, d_k=d_v=128 (BF16 q/k/v, FP32 gates, FP32
+state, S0 = 0).  One timed step = one gdn2_chunk_fwd call on that batch (one
+kernel launch).  The decode step (batch 256, H=16, d=128, FP32 state, 64
+consecutive in-place steps) is timed in the same run and reported under
+"decode" as state GB/s.
+
+* value      device time, inputs resident in HBM, CUDA events on the launching
+             stream, max over ranks; inputs (675 MB) exceed the 126 MB L2.
+* e2e        the same call from pinned HOST buffers: H2D of every input and D2H
+             of o and S_T inside the timed region, through the public API.
+* roofline   algorithmic bytes per launch / measured launch time, against the
+             measured HBM copy bandwidth (MEASURED_PEAKS.json).
+* cpu_baseline  the FP64 oracle on this host's cores, on a bounded sample.
+* --impl reference  times the oracle alone (the CPU reference arm).
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+(batch, head) recurrences are independent; no data-path collective), so
+scaling is weak and value = tokens of all ranks / max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gdn2_inputs as gi  # noqa: E402
+
+PREFILL = gi.PREFILL_4K
+DECODE = gi.DECODE_B256
+BYTES_PER_TOKEN_HEAD = 2560        # q,k,v bf16 (768) + alpha,b,w fp32 (1536) + o bf16 (256)
+METRIC = "GDN-2 chunk fwd tokens/s @H16 d128 T4K"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def prefill_bytes(B, T, H, dk, dv):
+    tok = B * T * H
+    return tok * (2 * dk * 2 + dv * 2 + 2 * dk * 4 + dv * 4 + dv * 2) + B * H * dk * dv * 4  # + S_T
+
+
+def decode_bytes(B, H, dk, dv):
+    bh = B * H
+    return bh * (2 * dk * dv * 4 + (2 * dk + dv) * 2 + (2 * dk + dv) * 4 + dv * 2)
+
+
+def state_bytes(B, H, dk, dv):
+    return 2 * B * H * dk * dv * 4
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_tokens_per_s(budget_s=12.0, max_heads=None):
+    """Time the FP64 oracle on a bounded sample of the prefill workload.
+
+    Sample: every (batch, head) chain of the workload (up to ``max_heads``) over
+    the first T_s tokens, T_s chosen from a short calibration so that the timed
+    run takes about ``budget_s`` seconds on all host cores.  Returns
+    (tokens/s in the workload's unit, threads, description)."""
+    import oracle
+    B, T, H, dk, dv = PREFILL["B"], PREFILL["T"], PREFILL["H"], PREFILL["dk"], PREFILL["dv"]
+    threads = oracle.num_threads()
+    heads = B * H if max_heads is None else min(B * H, max_heads)
+    calib = gi.chunk_inputs(1, 64, min(heads, threads), dk, dv, dtype="bf16", seed=1)
+    t0 = time.perf_counter()
+    oracle.gdn2(calib["q"], calib["k"], calib["v"], calib["alpha"], calib["b"], calib["w"])
+    per_tok = (time.perf_counter() - t0) / 64           # seconds per token for min(heads, threads) heads in parallel
+    waves = -(-heads // threads)
+    Ts = int(max(64, min(T, budget_s / max(per_tok * waves, 1e-9))))
+    x = gi.chunk_inputs(1, Ts, heads, dk, dv, dtype="bf16", seed=0)
+    t0 = time.perf_counter()
+    oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"])
+    dt = time.perf_counter() - t0
+    token_heads = heads * Ts
+    value = token_heads / H / dt                       # tokens of H heads each, per second
+    desc = f"oracle FP64 on {heads} heads x {Ts} tokens (d=128) of the prefill workload, {dt:.1f} s"
+    return value, threads, desc, dt
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is None:
+            self.out = ""
+            return
+        self.proc.terminate()
+        try:
+            self.out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(getattr(self, "out", ""))) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+
+        def num(s):
+            try:
+                return float(s.strip().split()[0])
+            except (ValueError, IndexError):
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def device_inputs(torch, x, dev):
+    out = {}
+    for n in ("q", "k", "v", "alpha", "b", "w"):
+        t = torch.from_numpy(np.ascontiguousarray(x[n]))
+        out[n] = t.to(dev).to(torch.bfloat16 if n in ("q", "k", "v") else torch.float32)
+    return out
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import gated_delta_rule_111_b200 as g
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=300))
+    g.load_library(rebuild_if_stale=(world == 1))
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- prefill workload (every rank its own replica; seed differs per rank)
+    B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
+    x = gi.chunk_inputs(**PREFILL, seed=rank)
+    d = device_inputs(torch, x, dev)
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    ST = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+
+    def step():
+        g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], None, o=o, S_T=ST, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # nvidia-smi samples every 100 ms: keep the GPU busy with the same step for
+    # about a second before the timed region so the samples see it under load.
+    t_est = time.perf_counter()
+    step()
+    torch.cuda.synchronize()
+    per = max(time.perf_counter() - t_est, 1e-5)
+    with ClockSampler(local) as clk:
+        for _ in range(int(min(4000, 1.2 / per))):
+            step()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        dist.barrier()
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens_per_step = B * T
+    value = tokens_per_step * world / (ms_step / 1e3)
+
+    # ---- e2e: pinned host buffers, copies inside the timed region
+    host = {n: d[n].cpu().pin_memory() for n in d}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_h = torch.empty(ST.shape, dtype=ST.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
+
+    def e2e_step():
+        for n in d:
+            d[n].copy_(host[n], non_blocking=True)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        S_h.copy_(ST, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(2, min(args.steps, 5))
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    del host, o_h, S_h
+
+    # ---- decode workload: 64 consecutive in-place steps, timed as one region
+    del d, o, ST
+    torch.cuda.empty_cache()
+    xd = gi.decode_inputs(**DECODE, seed=rank)
+    steps_d = DECODE["steps"]
+    Bd, Hd = DECODE["B"], DECODE["H"]
+    dd = device_inputs(torch, xd, dev)
+    S0d = torch.from_numpy(xd["S0"]).to(dev)
+    Sd = S0d.clone()
+    od = torch.empty((Bd, Hd, dv), dtype=torch.bfloat16, device=dev)
+    views = [[dd[n][s] for n in ("q", "k", "v", "alpha", "b", "w")] for s in range(steps_d)]
+
+    def decode_run():
+        for s in range(steps_d):
+            g.gdn2_recurrent_step(*views[s], Sd, o=od, stream=stream)
+
+    for _ in range(max(args.warmup, 1)):
+        decode_run()
+    torch.cuda.synchronize()
+    reps = 3
+    ev0.record(stream)
+    for _ in range(reps):
+        decode_run()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    dec_ms = ev0.elapsed_time(ev1) / (reps * steps_d)
+    if world > 1:
+        t = torch.tensor([dec_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dec_ms = float(t.item())
+
+    hbm, hbm_src = measured_peaks()
+    pre_bytes = prefill_bytes(B, T, H, dk, dv)
+    pre_gbs = pre_bytes / (ms_step / 1e3) / 1e9
+    dec_bytes = decode_bytes(Bd, Hd, dk, dv)
+    dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
+    st_gbs = state_bytes(Bd, Hd, dk, dv) / (dec_ms / 1e3) / 1e9
+    traffic = load_traffic()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc, _ = oracle_tokens_per_s(budget_s=args.cpu_budget)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; recipe in gdn2_inputs.py)",
+            "config": {"workload": "GDN-2 chunkwise prefill B=4 T=4096 H=16 d_k=d_v=128 chunk=64, S0=0",
+                       "global_batch": B * world, "seq_len": T, "heads": H, "d_k": dk, "d_v": dv,
+                       "dtypes": "q/k/v/o bf16, alpha/b/w fp32, state fp32, fp32 accumulation",
+                       "l2": "inputs (675 MB per call) larger than the 126 MB L2; no flush",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "e2e": {"value": B * T * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "roofline": {"bound": "hbm", "achieved": pre_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": pre_gbs / hbm, "traffic": traffic.get("gdn2_chunk"),
+                         "kernel": "gdn2 chunkwise prefill", "algorithmic_bytes_per_launch": pre_bytes,
+                         "peak_source": f"{hbm_src} HBM copy bandwidth", "frac_of_8TBps": pre_gbs / 8000.0},
+            "decode": {"metric": "GDN-2 decode state GB/s @B256 H16 d128", "value": st_gbs, "unit": "GB/s",
+                       "us_per_step": dec_ms * 1e3, "steps": steps_d * reps,
+                       "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
+                                    "frac": dec_gbs / hbm, "traffic": traffic.get("gdn2_decode"),
+                                    "algorithmic_bytes_per_launch": dec_bytes, "frac_of_8TBps": dec_gbs / 8000.0}},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def load_traffic():
+    """Per-launch DRAM traffic from the committed ncu summary, if it matches the current sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    try:
+        with open(path) as f:
+            data = json.load(f)
+        import hashlib
+        out = {}
+        for name, rec in data.items():
+            src = os.path.join(ROOT, rec["source"])
+            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+            out[name] = rec["bytes_per_launch"] if h == rec.get("source_sha256_16") else None
+        return out
+    except (OSError, KeyError, ValueError):
+        return {}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    budget = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(budget_s=budget / 4)
+    vals, descs, secs = [], [], []
+    for _ in range(args.steps):
+        v, cores, desc, dt = oracle_tokens_per_s(budget_s=budget)
+        vals.append(v)
+        descs.append(desc)
+        secs.append(dt)
+    value = statistics.median(vals)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": statistics.median(secs) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": "GDN-2 chunkwise prefill B=4 T=4096 H=16 d_k=d_v=128 chunk=64, S0=0",
+                       "global_batch": PREFILL["B"], "seq_len": PREFILL["T"]},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": descs[-1]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "ours":
+        args.warmup = max(3, args.warmup)       # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+"""Python binding of libgdn2, the B200 (sm_100a) Gated DeltaNet-2 recurrence.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libgdn2.so`` behind the C ABI declared in ``include/gdn2.h``.  There
+is no CPU implementation and no fallback; without the compiled library or a CUDA
+device these functions raise.
+
+Functions (same names as the C ABI):
+  gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, ...)  -> (o, S_T)   chunkwise prefill
+  gdn2_recurrent_step(q, k, v, alpha, b, w, S, ...)   -> o          in-place decode step
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from . import build as _build
+
+__all__ = ["gdn2_chunk_fwd", "gdn2_recurrent_step", "library_path", "load_library", "exported_symbols",
+           "GDN2_OK", "GDN2_ERR_INVALID_ARG", "GDN2_ERR_UNSUPPORTED", "GDN2_ERR_CUDA", "Gdn2Error"]
+
+GDN2_OK, GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_CUDA = 0, 1, 2, 3
+GDN2_BF16, GDN2_FP32 = 0, 1
+HEADER = os.path.join(_build.ROOT, "include", "gdn2.h")
+
+_lib = None
+
+
+class Gdn2Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library(rebuild_if_stale: bool = True) -> ctypes.CDLL:
+    """Load libgdn2.so (compiling it first if it is missing or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.build() if rebuild_if_stale else _build.LIB
+    if not os.path.exists(path):
+        raise ImportError(f"libgdn2.so not found at {path}; run python -m gated_delta_rule_111_b200.build")
+    lib = ctypes.CDLL(path)
+    vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+    lib.gdn2_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp]
+    lib.gdn2_chunk_fwd.restype = i
+    lib.gdn2_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
+    lib.gdn2_recurrent_step.restype = i
+    lib.gdn2_status_string.argtypes = [i]
+    lib.gdn2_status_string.restype = ctypes.c_char_p
+    lib.gdn2_last_error.argtypes = []
+    lib.gdn2_last_error.restype = ctypes.c_char_p
+    lib.gdn2_version.restype = i
+    _lib = lib
+    return lib
+
+
+def exported_symbols() -> list[str]:
+    """Function names declared in include/gdn2.h."""
+    text = open(HEADER).read()
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(gdn2_\w+)\s*\(", text, flags=re.M)
+
+
+def _check(status: int):
+    if status != GDN2_OK:
+        lib = load_library()
+        msg = lib.gdn2_last_error().decode()
+        raise Gdn2Error(status, f"{lib.gdn2_status_string(status).decode()}: {msg}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN2_BF16
+    if t.dtype == torch.float32:
+        return GDN2_FP32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, name, dtype, shape, device):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, *, o=None, S_T=None, output_final_state=True,
+                   stream=None):
+    """Chunkwise prefill.  q,k [B,T,H,dk], v [B,T,H,dv] (bf16 or fp32); alpha,b [B,T,H,dk] and
+    w [B,T,H,dv] fp32; S0 [B,H,dk,dv] fp32 or None.  Returns (o, S_T); S_T is None when
+    ``output_final_state`` is False and no S_T buffer is given.  S_T may be S0 (in place)."""
+    lib = load_library()
+    if q.device.type != "cuda":
+        raise ValueError("gdn2_chunk_fwd needs CUDA tensors (there is no CPU implementation)")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("q", q, dk), ("k", k, dk), ("v", v, dv)):
+        _need(t, name, dt, (B, T, H, d), dev)
+    for name, t, d in (("alpha", alpha, dk), ("b", b, dk), ("w", w, dv)):
+        _need(t, name, torch.float32, (B, T, H, d), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _need(o, "o", dt, (B, T, H, dv), dev)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    elif S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dk, dv), dev)
+    _check(lib.gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                              _ptr(S_T), B, T, H, dk, dv, code, _stream(stream, dev)))
+    return o, S_T
+
+
+def gdn2_recurrent_step(q, k, v, alpha, b, w, S, *, o=None, stream=None):
+    """One decode step, state updated in place.  q,k [B,H,dk], v [B,H,dv] (bf16 or fp32);
+    alpha,b [B,H,dk], w [B,H,dv] fp32; S [B,H,dk,dv] fp32 (overwritten).  Returns o [B,H,dv]."""
+    lib = load_library()
+    if q.device.type != "cuda":
+        raise ValueError("gdn2_recurrent_step needs CUDA tensors (there is no CPU implementation)")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("q", q, dk), ("k", k, dk), ("v", v, dv)):
+        _need(t, name, dt, (B, H, d), dev)
+    for name, t, d in (("alpha", alpha, dk), ("b", b, dk), ("w", w, dv)):
+        _need(t, name, torch.float32, (B, H, d), dev)
+    _need(S, "S", torch.float32, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=dt, device=dev)
+    else:
+        _need(o, "o", dt, (B, H, dv), dev)
+    _check(lib.gdn2_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
+                                   B, H, dk, dv, code, _stream(stream, dev)))
+    return o

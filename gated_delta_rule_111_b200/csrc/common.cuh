@@ -1,0 +1,39 @@
+// Internal helpers shared by the libgdn2 kernels (not part of the public ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn2.h"
+
+namespace gdn2 {
+
+// Element type of q, k, v, o.
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float load(const float *p) { return __ldg(p); }
+    static __device__ __forceinline__ void store(float *p, float x) { *p = x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16 *p) { return __bfloat162float(__ldg(p)); }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+};
+
+// alpha below FLT_MIN is treated as FLT_MIN (documented precondition: alpha > 0).
+__device__ __forceinline__ float clamp_alpha(float a) { return fmaxf(a, 1.17549435e-38f); }
+
+// Streaming (read-once / write-once) 16-byte accesses for the decode state.
+__device__ __forceinline__ float4 ld_stream(const float4 *p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(float4 *p, float4 v) { __stcs(p, v); }
+
+// Host-side launchers (one per kernel family); each returns cudaGetLastError().
+cudaError_t launch_recurrent_step(const void *q, const void *k, const void *v, const float *alpha,
+                                  const float *b, const float *w, float *S, void *o, int B, int H,
+                                  int dk, int dv, gdn2_dtype dt, cudaStream_t stream);
+
+cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *alpha,
+                              const float *b, const float *w, const float *S0, void *o, float *S_T,
+                              int B, int T, int H, int dk, int dv, gdn2_dtype dt, cudaStream_t stream);
+
+}  // namespace gdn2

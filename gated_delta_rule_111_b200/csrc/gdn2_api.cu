@@ -1,0 +1,146 @@
+// C ABI of libgdn2: argument validation on the host, then kernel dispatch on the
+// caller's stream.  Nothing here allocates device memory.
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace gdn2 {
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const float *b,
+                            const float *w, const float *S0, void *o, float *S_T, int B, int T, int H,
+                            cudaStream_t stream);
+bool chunk_tc_supported(int dk, int dv, gdn2_dtype dt);
+}  // namespace gdn2
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+gdn2_status fail(gdn2_status s, const char *fmt, const char *detail) {
+    snprintf(g_last_error, sizeof(g_last_error), fmt, detail);
+    return s;
+}
+
+gdn2_status cuda_status(cudaError_t err, const char *where) {
+    if (err == cudaSuccess) return GDN2_OK;
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(err));
+    return GDN2_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn2_status check_common(int B, int H, int dk, int dv, gdn2_dtype dt) {
+    if (B < 0 || H < 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "negative B or H");
+    if (dt != GDN2_BF16 && dt != GDN2_FP32) return fail(GDN2_ERR_UNSUPPORTED, "%s", "unknown dtype");
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+        return fail(GDN2_ERR_UNSUPPORTED, "%s", "head sizes must be 64 or 128");
+    return GDN2_OK;
+}
+
+gdn2_status check_ptr(const void *p, const char *name) {
+    if (!p) return fail(GDN2_ERR_INVALID_ARG, "null pointer: %s", name);
+    if (!aligned16(p)) return fail(GDN2_ERR_INVALID_ARG, "pointer not 16-byte aligned: %s", name);
+    return GDN2_OK;
+}
+
+// [a, a+na) and [b, b+nb) overlap?
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const char *pa = static_cast<const char *>(a), *pb = static_cast<const char *>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn2_status_string(gdn2_status s) {
+    switch (s) {
+        case GDN2_OK: return "GDN2_OK";
+        case GDN2_ERR_INVALID_ARG: return "GDN2_ERR_INVALID_ARG";
+        case GDN2_ERR_UNSUPPORTED: return "GDN2_ERR_UNSUPPORTED";
+        case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA";
+    }
+    return "GDN2_UNKNOWN_STATUS";
+}
+
+const char *gdn2_last_error(void) { return g_last_error; }
+
+int gdn2_version(void) { return 100; }
+
+gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *b,
+                           const float *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
+                           int d_v, gdn2_dtype dt, void *stream) {
+    g_last_error[0] = 0;
+    gdn2_status st = check_common(B, H, d_k, d_v, dt);
+    if (st != GDN2_OK) return st;
+    if (T < 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "negative T");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (B == 0 || H == 0) return GDN2_OK;
+    const size_t es = dt == GDN2_BF16 ? 2 : 4;
+    const size_t state_bytes = (size_t)B * H * d_k * d_v * sizeof(float);
+    if (S0 && (st = check_ptr(S0, "S0")) != GDN2_OK) return st;
+    if (S_T && (st = check_ptr(S_T, "S_T")) != GDN2_OK) return st;
+    if (S0 && S_T && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes))
+        return fail(GDN2_ERR_INVALID_ARG, "%s", "S_T partially overlaps S0 (only exact aliasing is allowed)");
+    if (T == 0) {
+        if (!S_T || S_T == S0) return GDN2_OK;
+        cudaError_t err = S0 ? cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, s)
+                             : cudaMemsetAsync(S_T, 0, state_bytes, s);
+        return cuda_status(err, "T = 0 state copy");
+    }
+    const void *ins[6] = {q, k, v, alpha, b, w};
+    const char *names[6] = {"q", "k", "v", "alpha", "b", "w"};
+    for (int i = 0; i < 6; ++i)
+        if ((st = check_ptr(ins[i], names[i])) != GDN2_OK) return st;
+    if ((st = check_ptr(o, "o")) != GDN2_OK) return st;
+    const size_t tok = (size_t)B * T * H;
+    const size_t in_bytes[6] = {tok * d_k * es, tok * d_k * es, tok * d_v * es,
+                                tok * d_k * 4,  tok * d_k * 4,  tok * d_v * 4};
+    const size_t o_bytes = tok * d_v * es;
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(o, o_bytes, ins[i], in_bytes[i])) return fail(GDN2_ERR_INVALID_ARG, "o overlaps %s", names[i]);
+    if (overlaps(o, o_bytes, S0, state_bytes) || overlaps(o, o_bytes, S_T, state_bytes))
+        return fail(GDN2_ERR_INVALID_ARG, "%s", "o overlaps a state buffer");
+    if (S_T)
+        for (int i = 0; i < 6; ++i)
+            if (overlaps(S_T, state_bytes, ins[i], in_bytes[i]))
+                return fail(GDN2_ERR_INVALID_ARG, "S_T overlaps %s", names[i]);
+
+    cudaError_t err;
+    if (gdn2::chunk_tc_supported(d_k, d_v, dt))
+        err = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, s);
+    else
+        err = gdn2::launch_chunk_simt(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, dt, s);
+    return cuda_status(err, "gdn2_chunk_fwd launch");
+}
+
+gdn2_status gdn2_recurrent_step(const void *q, const void *k, const void *v, const float *alpha,
+                                const float *b, const float *w, float *S, void *o, int B, int H, int d_k,
+                                int d_v, gdn2_dtype dt, void *stream) {
+    g_last_error[0] = 0;
+    gdn2_status st = check_common(B, H, d_k, d_v, dt);
+    if (st != GDN2_OK) return st;
+    if (B == 0 || H == 0) return GDN2_OK;
+    const void *ins[6] = {q, k, v, alpha, b, w};
+    const char *names[6] = {"q", "k", "v", "alpha", "b", "w"};
+    for (int i = 0; i < 6; ++i)
+        if ((st = check_ptr(ins[i], names[i])) != GDN2_OK) return st;
+    if ((st = check_ptr(S, "S")) != GDN2_OK) return st;
+    if ((st = check_ptr(o, "o")) != GDN2_OK) return st;
+    const size_t es = dt == GDN2_BF16 ? 2 : 4;
+    const size_t bh = (size_t)B * H;
+    const size_t state_bytes = bh * d_k * d_v * sizeof(float);
+    const size_t in_bytes[6] = {bh * d_k * es, bh * d_k * es, bh * d_v * es, bh * d_k * 4, bh * d_k * 4, bh * d_v * 4};
+    const size_t o_bytes = bh * d_v * es;
+    for (int i = 0; i < 6; ++i) {
+        if (overlaps(o, o_bytes, ins[i], in_bytes[i])) return fail(GDN2_ERR_INVALID_ARG, "o overlaps %s", names[i]);
+        if (overlaps(S, state_bytes, ins[i], in_bytes[i])) return fail(GDN2_ERR_INVALID_ARG, "S overlaps %s", names[i]);
+    }
+    if (overlaps(o, o_bytes, S, state_bytes)) return fail(GDN2_ERR_INVALID_ARG, "%s", "o overlaps S");
+    cudaError_t err = gdn2::launch_recurrent_step(q, k, v, alpha, b, w, S, o, B, H, d_k, d_v, dt,
+                                                  static_cast<cudaStream_t>(stream));
+    return cuda_status(err, "gdn2_recurrent_step launch");
+}
+
+}  // extern "C"

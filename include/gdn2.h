@@ -1,0 +1,124 @@
+/*
+ * libgdn2 -- Gated DeltaNet-2 recurrence on NVIDIA B200 (sm_100a).
+ *
+ * The recurrence ("Gated DeltaNet-2: Decoupling Erase and Write in Linear
+ * Attention", iplexlaw.co.kr analysis, section "Independent decisions on two
+ * axes"), per batch item b, head h and token t, with state S in R^{d_k x d_v}:
+ *
+ *     Sbar = diag(alpha_t) S_{t-1}        channel-wise decay of the key rows
+ *     e    = b_t (.) k_t                  erase vector (key channels)
+ *     z    = w_t (.) v_t                  write vector (value channels)
+ *     r    = Sbar^T e                     old read at the erase address
+ *     S_t  = Sbar + k_t (z - r)^T         delta write
+ *     o_t  = S_t^T q_t                    the query reads the updated state
+ *
+ * Two entry points compute exactly this, in the two execution modes the pages
+ * describe ("Token processing and parallel training": chunkwise WY with 64-token
+ * chunks for training/prefill; the mindpattern.ai DeltaNet trail: a fused
+ * recurrent mode for decode, with identical mathematics).
+ *
+ * Conventions shared by every call
+ *   - All pointers are DEVICE pointers, 16-byte aligned, to dense row-major
+ *     tensors.  The library allocates nothing and keeps no pointer after return.
+ *   - Per-token tensors have layout [B][T][H][d] (decode: [B][H][d]).  q, k are
+ *     d_k wide, v and o are d_v wide; alpha and b are d_k wide; w is d_v wide.
+ *   - States are FP32 [B][H][d_k][d_v]: row i is key channel i.
+ *   - q, k, v and o share the element type `dt` (BF16 or FP32).  Gates (alpha,
+ *     b, w) and states are always FP32.  Accumulation is FP32.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream and never synchronise the device.
+ *   - Supported head sizes: d_k, d_v in {64, 128}.  Other sizes return
+ *     GDN2_ERR_UNSUPPORTED.
+ *   - Preconditions (documented, not checked on the device): 0 < alpha <= 1
+ *     (values below FLT_MIN are treated as FLT_MIN); b and w are not clamped
+ *     (the pages ablate an erase gate in [0, 2]).  For the BF16 tensor-core
+ *     prefill, the decay accumulated over one 64-token chunk must satisfy
+ *     prod(alpha) >= 1e-34 per key channel (sum of -ln(alpha) <= 78).
+ *   - Errors: argument problems are detected on the host before any launch and
+ *     return GDN2_ERR_INVALID_ARG / GDN2_ERR_UNSUPPORTED with nothing enqueued.
+ *     A failed launch returns GDN2_ERR_CUDA; gdn2_last_error() describes it.
+ *     Kernels never trap.
+ */
+#ifndef GDN2_H_
+#define GDN2_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN2_OK = 0,
+    GDN2_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative size, aliasing not allowed */
+    GDN2_ERR_UNSUPPORTED = 2,  /* head size or dtype this build does not implement */
+    GDN2_ERR_CUDA = 3          /* a CUDA runtime call or kernel launch failed */
+} gdn2_status;
+
+typedef enum {
+    GDN2_BF16 = 0,  /* q, k, v, o are bfloat16 */
+    GDN2_FP32 = 1   /* q, k, v, o are float32  */
+} gdn2_dtype;
+
+/*
+ * Chunkwise prefill ("Token processing and parallel training": 64-token chunks,
+ * cumulative channel-wise decay absorbed into asymmetric erase factors,
+ * triangular solves and dense products within each chunk, FP32 decay and
+ * state/solve precision).
+ *
+ *   q, k      [B][T][H][d_k]  dt            read
+ *   v         [B][T][H][d_v]  dt            read
+ *   alpha, b  [B][T][H][d_k]  float         read
+ *   w         [B][T][H][d_v]  float         read
+ *   S0        [B][H][d_k][d_v] float        read; NULL means a zero initial state
+ *   o         [B][T][H][d_v]  dt            written (o_t of every token)
+ *   S_T       [B][H][d_k][d_v] float        written (state after token T-1); may be
+ *                                           NULL, and may alias S0 (in-place chaining)
+ *
+ * T may be any value >= 0 (the last chunk may be partial; chunking restarts at
+ * t = 0 in every call, which does not change the result).  T = 0 writes S_T = S0.
+ * B = 0 or H = 0 is a no-op.  o must not overlap any input.
+ * BF16 with d_k = d_v = 128 runs on the tcgen05 tensor-core path; every other
+ * combination runs an FP32 CUDA-core path with the same mathematics.
+ */
+gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v,
+                           const float *alpha, const float *b, const float *w,
+                           const float *S0, void *o, float *S_T,
+                           int B, int T, int H, int d_k, int d_v,
+                           gdn2_dtype dt, void *stream);
+
+/*
+ * Fused single-token decode step (the recurrent mode; the same mathematics with
+ * T = 1, updating the state in place).
+ *
+ *   q, k      [B][H][d_k]  dt     read
+ *   v         [B][H][d_v]  dt     read
+ *   alpha, b  [B][H][d_k]  float  read
+ *   w         [B][H][d_v]  float  read
+ *   S         [B][H][d_k][d_v] float   read and overwritten with S_t
+ *   o         [B][H][d_v]  dt     written
+ *
+ * Memory-bound: each call reads and writes every state once.  B = 0 or H = 0 is
+ * a no-op.  o must not overlap S or any input.
+ */
+gdn2_status gdn2_recurrent_step(const void *q, const void *k, const void *v,
+                                const float *alpha, const float *b, const float *w,
+                                float *S, void *o,
+                                int B, int H, int d_k, int d_v,
+                                gdn2_dtype dt, void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *gdn2_status_string(gdn2_status s);
+
+/* Text of the last GDN2_ERR_CUDA / argument error seen by this thread (static
+ * thread-local buffer, valid until the next call on the same thread). */
+const char *gdn2_last_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int gdn2_version(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* GDN2_H_ */

@@ -1,0 +1,120 @@
+"""The C ABI of libgdn2 without a GPU: the library loads, exports every function
+declared in include/gdn2.h, and rejects bad arguments on the host before any
+CUDA call.  Every call below returns during host-side validation."""
+import ctypes
+import subprocess
+
+import pytest
+import torch
+
+import gated_delta_rule_111_b200 as g
+
+BF16, FP32 = 0, 1
+A16 = 0x10000          # a fake, 16-byte aligned "device" address; never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return g.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = g.exported_symbols()
+    assert set(declared) >= {"gdn2_chunk_fwd", "gdn2_recurrent_step", "gdn2_status_string",
+                             "gdn2_last_error", "gdn2_version"}
+    out = subprocess.check_output(["nm", "-D", "--defined-only", g.library_path()], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [s for s in declared if s not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for s in declared:
+        getattr(lib, s)
+
+
+def test_status_strings(lib):
+    assert lib.gdn2_status_string(0) == b"GDN2_OK"
+    assert lib.gdn2_status_string(1) == b"GDN2_ERR_INVALID_ARG"
+    assert lib.gdn2_status_string(2) == b"GDN2_ERR_UNSUPPORTED"
+    assert lib.gdn2_status_string(3) == b"GDN2_ERR_CUDA"
+    assert lib.gdn2_version() >= 100
+
+
+def _chunk(lib, q=A16, k=A16, v=A16, a=A16, b=A16, w=A16, S0=None, o=A16 * 64, ST=None,
+           B=1, T=4, H=1, dk=128, dv=128, dt=BF16):
+    P = ctypes.c_void_p
+    return lib.gdn2_chunk_fwd(P(q), P(k), P(v), P(a), P(b), P(w), P(S0), P(o), P(ST), B, T, H, dk, dv, dt, None)
+
+
+def _step(lib, q=A16, k=A16, v=A16, a=A16, b=A16, w=A16, S=A16 * 128, o=A16 * 512, B=1, H=1, dk=128, dv=128,
+          dt=BF16):
+    P = ctypes.c_void_p
+    return lib.gdn2_recurrent_step(P(q), P(k), P(v), P(a), P(b), P(w), P(S), P(o), B, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 128), (128, 96), (256, 256), (0, 128)])
+def test_unsupported_head_sizes(lib, dk, dv):
+    assert _chunk(lib, dk=dk, dv=dv) == g.GDN2_ERR_UNSUPPORTED
+    assert _step(lib, dk=dk, dv=dv) == g.GDN2_ERR_UNSUPPORTED
+
+
+def test_unknown_dtype(lib):
+    assert _chunk(lib, dt=7) == g.GDN2_ERR_UNSUPPORTED
+    assert _step(lib, dt=-1) == g.GDN2_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "a", "b", "w", "o"])
+def test_null_pointer_rejected(lib, field):
+    assert _chunk(lib, **{field: None}) == g.GDN2_ERR_INVALID_ARG
+    assert b"null pointer" in lib.gdn2_last_error()
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "a", "b", "w", "o", "S0", "ST"])
+def test_misaligned_pointer_rejected(lib, field):
+    assert _chunk(lib, **{field: A16 * 1024 + 4}) == g.GDN2_ERR_INVALID_ARG
+    assert b"aligned" in lib.gdn2_last_error()
+
+
+def test_step_null_state_rejected(lib):
+    assert _step(lib, S=None) == g.GDN2_ERR_INVALID_ARG
+
+
+def test_negative_sizes(lib):
+    assert _chunk(lib, T=-1) == g.GDN2_ERR_INVALID_ARG
+    assert _chunk(lib, B=-2) == g.GDN2_ERR_INVALID_ARG
+    assert _step(lib, H=-1) == g.GDN2_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_noop(lib):
+    # B = 0 or H = 0 returns before any CUDA call, even with null pointers.
+    assert _chunk(lib, q=None, o=None, B=0) == g.GDN2_OK
+    assert _chunk(lib, q=None, o=None, H=0) == g.GDN2_OK
+    assert _step(lib, q=None, S=None, B=0) == g.GDN2_OK
+
+
+def test_t0_inplace_state_is_noop(lib):
+    # T = 0 with S_T aliasing S0 leaves the state as it is; nothing to enqueue.
+    assert _chunk(lib, q=None, o=None, T=0, S0=A16 * 4096, ST=A16 * 4096) == g.GDN2_OK
+
+
+def test_overlapping_output_rejected(lib):
+    # o overlapping an input, and a state that partially overlaps S0.
+    assert _chunk(lib, q=A16 * 64, o=A16 * 64) == g.GDN2_ERR_INVALID_ARG
+    assert b"overlaps" in lib.gdn2_last_error()
+    assert _chunk(lib, S0=A16 * 4096, ST=A16 * 4096 + 16) == g.GDN2_ERR_INVALID_ARG
+    assert _step(lib, o=A16 * 128, S=A16 * 128) == g.GDN2_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    x = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdn2_chunk_fwd(x, x, x, x, x, x)
+    y = torch.zeros(1, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdn2_recurrent_step(y, y, y, y, y, y, torch.zeros(1, 1, 64, 64))
+
+
+def test_product_package_does_not_import_oracle():
+    import pathlib
+    pkg = pathlib.Path(g.__file__).parent
+    for p in list(pkg.rglob("*.py")) + list(pkg.rglob("*.cu")) + list(pkg.rglob("*.cuh")):
+        text = p.read_text()
+        assert "oracle" not in text.replace("oracle-free", ""), f"{p} mentions the oracle"

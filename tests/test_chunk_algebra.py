@@ -1,0 +1,81 @@
+"""The chunkwise algebra the CUDA kernels implement, checked in FP64 against the
+token-by-token oracle (CPU only).
+
+"Token processing and parallel training" (Gated DeltaNet-2 analysis) sketches
+the parallel form: 64-token chunks, cumulative channel-wise decay absorbed into
+asymmetric erase factors, a triangular solve and dense products per chunk.  Our
+re-derivation, per chunk of n tokens starting from state S:
+
+  gamma_t = prod_{j<=t} alpha_j  (per key channel),   rho_t = 1 / gamma_t
+  Etil = e * gamma,  Qtil = q * gamma,  Ktil = k * rho        (e = b*k, z = w*v)
+  A = strict_tril(Etil Ktil^T),  P = tril(Qtil Ktil^T)
+  U = (I + A)^{-1} (Z - Etil S)      -- the per-token corrections z_t - r_t
+  O = Qtil S + P U
+  S <- diag(gamma_n) (S + Ktil^T U)
+
+Chunking is an exact re-association of the token recurrence ("identical
+mathematics" of the two modes), so this must match the oracle to rounding.
+"""
+import numpy as np
+import pytest
+
+import gdn2_inputs as gi
+import oracle
+
+
+def chunk_model(q, k, v, alpha, b, w, S0, C=64, form="factored"):
+    """FP64 chunkwise forward for one (batch, head): inputs [T, d], S0 [dk, dv]."""
+    T, dk = q.shape
+    dv = v.shape[1]
+    S = np.zeros((dk, dv)) if S0 is None else S0.astype(np.float64).copy()
+    o = np.zeros((T, dv))
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(T, c0 + C))
+        qc, kc, vc, ac, bc, wc = (x[sl].astype(np.float64) for x in (q, k, v, alpha, b, w))
+        n = qc.shape[0]
+        e, z = bc * kc, wc * vc
+        if form == "factored":
+            gamma = np.cumprod(ac, axis=0)
+            rho = np.cumprod(1.0 / ac, axis=0)
+            Et, Qt, Kt = e * gamma, qc * gamma, kc * rho
+            A = np.tril(Et @ Kt.T, -1)
+            P = np.tril(Qt @ Kt.T)
+            U = np.linalg.solve(np.eye(n) + A, z - Et @ S)
+            o[sl] = Qt @ S + P @ U
+            S = gamma[-1][:, None] * (S + Kt.T @ U)
+        else:  # difference-of-logs form used by the FP32 CUDA-core kernel
+            g = np.cumsum(np.log(ac), axis=0)
+            D = np.exp(g[:, None, :] - g[None, :, :])           # [t, s, i] decay ratio, used for s <= t
+            mask = np.tril(np.ones((n, n)), -1)
+            A = np.einsum("ti,si,tsi->ts", e, kc, D) * mask
+            P = np.einsum("ti,si,tsi->ts", qc, kc, D) * (mask + np.eye(n))
+            Et, Qt = e * np.exp(g), qc * np.exp(g)
+            Kh = kc * np.exp(g[-1][None, :] - g)
+            U = np.linalg.solve(np.eye(n) + A, z - Et @ S)
+            o[sl] = Qt @ S + P @ U
+            S = np.exp(g[-1])[:, None] * S + Kh.T @ U
+    return o, S
+
+
+@pytest.mark.parametrize("form", ["factored", "logdiff"])
+@pytest.mark.parametrize("T,C", [(150, 64), (64, 64), (1, 64), (65, 64), (37, 16)])
+def test_chunk_algebra_matches_token_recurrence(form, T, C):
+    x = gi.chunk_inputs(1, T, 2, 16, 12, dtype="fp32", seed=11, s0_std=0.3)
+    o_ref, S_ref = oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], x["S0"])
+    for h in range(2):
+        args = [x[n][0, :, h] for n in ("q", "k", "v", "alpha", "b", "w")]
+        o, S = chunk_model(*args, x["S0"][0, h], C=C, form=form)
+        scale = np.sqrt(np.mean(o_ref[0, :, h] ** 2))
+        assert np.max(np.abs(o - o_ref[0, :, h])) <= 1e-12 * scale
+        assert np.max(np.abs(S - S_ref[0, h])) <= 1e-12 * np.sqrt(np.mean(S_ref[0, h] ** 2))
+
+
+def test_chunk_algebra_gdn2_specific_gates():
+    """Erase gate above 1 (the pages ablate b in [0, 2]) and a write gate that differs from it."""
+    x = gi.chunk_inputs(1, 100, 1, 8, 8, dtype="fp32", seed=5, s0_std=0.5)
+    b2 = 2.0 * x["b"]
+    o_ref, S_ref = oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], b2, x["w"], x["S0"])
+    args = [x["q"][0, :, 0], x["k"][0, :, 0], x["v"][0, :, 0], x["alpha"][0, :, 0], b2[0, :, 0], x["w"][0, :, 0]]
+    o, S = chunk_model(*args, x["S0"][0, 0])
+    assert np.max(np.abs(o - o_ref[0, :, 0])) <= 1e-11 * np.sqrt(np.mean(o_ref ** 2))
+    assert np.max(np.abs(S - S_ref[0, 0])) <= 1e-11 * np.sqrt(np.mean(S_ref ** 2))

@@ -1,0 +1,268 @@
+"""Parity of the CUDA library (through its C ABI) with the FP64 oracle.
+
+Error metric: max |x_gpu - x_ref| / RMS(x_ref) over the compared tensor.
+Tolerances: FP32 inputs 1e-4 (o and S_T); BF16 q/k/v with FP32 gates and
+accumulation: o 2e-2, S_T 1e-2.  At full workload sizes the oracle recomputes a
+sample of (batch, head) pairs -- every head is an independent recurrence, so a
+sampled head is compared element by element over all tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gdn2_inputs as gi
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+TOL_FP32 = 1e-4
+TOL_BF16_O = 2e-2
+TOL_BF16_S = 1e-2
+
+
+def rel(x, ref):
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.max(np.abs(x - ref)) / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
+
+
+@pytest.fixture(scope="module")
+def g():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gated_delta_rule_111_b200 as mod
+    mod.load_library()
+    return mod
+
+
+def to_dev(x, keys=("q", "k", "v", "alpha", "b", "w")):
+    dt = torch.bfloat16 if x["dtype"] == "bf16" else torch.float32
+    out = {}
+    for n in keys:
+        t = torch.from_numpy(np.ascontiguousarray(x[n]))
+        out[n] = t.to("cuda").to(dt if n in ("q", "k", "v") else torch.float32)
+    out["S0"] = None if x.get("S0") is None else torch.from_numpy(x["S0"]).cuda()
+    return out
+
+
+def run_chunk(g, x, **kw):
+    d = to_dev(x)
+    o, ST = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], d["S0"], **kw)
+    torch.cuda.synchronize()
+    return o.float().cpu().numpy(), (None if ST is None else ST.cpu().numpy())
+
+
+def sel_heads(x, pairs):
+    """Inputs restricted to the (b, h) pairs, as a batch of len(pairs) single-head sequences."""
+    out = {}
+    for n in ("q", "k", "v", "alpha", "b", "w"):
+        out[n] = np.stack([x[n][b, :, h] for b, h in pairs])[:, :, None, :]
+    out["S0"] = None if x["S0"] is None else np.stack([x["S0"][b, h] for b, h in pairs])[:, None]
+    return out
+
+
+def check_sampled(x, o, ST, pairs, tol_o, tol_s, ref="gdn2"):
+    s = sel_heads(x, pairs)
+    if ref == "gdn2":
+        o_ref, S_ref = oracle.gdn2(s["q"], s["k"], s["v"], s["alpha"], s["b"], s["w"], s["S0"])
+    elif ref == "kda":
+        beta = np.stack([x["beta"][b, :, h] for b, h in pairs])[:, :, None]
+        o_ref, S_ref = oracle.kda(s["q"], s["k"], s["v"], s["alpha"], beta, s["S0"])
+    else:
+        beta = np.stack([x["beta"][b, :, h] for b, h in pairs])[:, :, None]
+        a1 = np.stack([x["alpha_scalar"][b, :, h] for b, h in pairs])[:, :, None]
+        o_ref, S_ref = oracle.gdn(s["q"], s["k"], s["v"], a1, beta, s["S0"])
+    og = np.stack([o[b, :, h] for b, h in pairs])[:, :, None]
+    eo = rel(og, o_ref)
+    assert eo <= tol_o, f"o error {eo:.3e} > {tol_o}"
+    if ST is not None:
+        Sg = np.stack([ST[b, h] for b, h in pairs])[:, None]
+        es = rel(Sg, S_ref)
+        assert es <= tol_s, f"S_T error {es:.3e} > {tol_s}"
+    return eo
+
+
+# ---------------------------------------------------------------- small, full comparison
+
+def test_tiny_fp32_full(g):
+    """B=1, T=256, H=2, d=64, FP32 throughout, S0 = 0: every output checked."""
+    x = gi.chunk_inputs(**gi.TINY_FP32, seed=0)
+    o, ST = run_chunk(g, x)
+    o_ref, S_ref = oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], None)
+    assert rel(o, o_ref) <= TOL_FP32
+    assert rel(ST, S_ref) <= TOL_FP32
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 129, 200])
+@pytest.mark.parametrize("d", [64, 128])
+def test_small_full(g, dtype, T, d):
+    """Several chunks and a ragged tail, nonzero S0; every output checked."""
+    x = gi.chunk_inputs(2, T, 3, d, d, dtype=dtype, seed=T + d, s0_std=0.05)
+    o, ST = run_chunk(g, x)
+    o_ref, S_ref = oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], x["S0"])
+    if dtype == "fp32":
+        assert rel(o, o_ref) <= TOL_FP32 and rel(ST, S_ref) <= TOL_FP32
+    else:
+        assert rel(o, o_ref) <= TOL_BF16_O and rel(ST, S_ref) <= TOL_BF16_S
+
+
+def test_delta_identity_fp32(g):
+    """b = 1, w = 1, unit keys, q = k: every output equals v (the delta rule writes the error)."""
+    x = gi.chunk_inputs(1, 130, 2, 128, 128, dtype="fp32", seed=9, s0_std=0.1)
+    kk = x["k"]
+    d = to_dev(x)
+    kd = torch.from_numpy(kk).cuda()
+    ones = torch.ones_like(d["b"])
+    o, _ = g.gdn2_chunk_fwd(kd, kd, d["v"], d["alpha"], ones, torch.ones_like(d["w"]), d["S0"])
+    torch.cuda.synchronize()
+    assert rel(o.cpu().numpy(), x["v"]) <= TOL_FP32
+
+
+def test_no_erase_matches_closed_form(g):
+    """b = 0: the output is the decayed causal linear-attention sum (explicit O(T^2) oracle)."""
+    x = gi.chunk_inputs(1, 96, 2, 64, 64, dtype="fp32", seed=4, s0_std=0.1)
+    x["b"] = np.zeros_like(x["b"])
+    o, _ = run_chunk(g, x)
+    o_ref = oracle.b0_sum(x["q"], x["k"], x["v"], x["alpha"], x["w"], x["S0"])
+    assert rel(o, o_ref) <= TOL_FP32
+
+
+def test_state_inplace_and_optional_outputs(g):
+    x = gi.chunk_inputs(1, 100, 2, 128, 128, dtype="bf16", seed=3, s0_std=0.05)
+    d = to_dev(x)
+    ref_o, ref_S = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], d["S0"])
+    S = d["S0"].clone()
+    o2, S2 = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], S, S_T=S)
+    assert S2.data_ptr() == S.data_ptr()
+    o3, S3 = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], d["S0"], output_final_state=False)
+    torch.cuda.synchronize()
+    assert S3 is None
+    assert torch.equal(o2, ref_o) and torch.equal(S, ref_S) and torch.equal(o3, ref_o)
+
+
+def test_zero_length_and_empty(g):
+    x = gi.chunk_inputs(2, 1, 2, 64, 64, dtype="bf16", seed=1, s0_std=0.1)
+    d = to_dev(x)
+    z = {n: t[:, :0].contiguous() for n, t in d.items() if n != "S0"}
+    o, ST = g.gdn2_chunk_fwd(z["q"], z["k"], z["v"], z["alpha"], z["b"], z["w"], d["S0"])
+    o0, ST0 = g.gdn2_chunk_fwd(z["q"], z["k"], z["v"], z["alpha"], z["b"], z["w"], None)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and torch.equal(ST, d["S0"]) and torch.count_nonzero(ST0) == 0
+    e = {n: t[:0].contiguous() for n, t in d.items() if n != "S0"}
+    o, ST = g.gdn2_chunk_fwd(e["q"], e["k"], e["v"], e["alpha"], e["b"], e["w"], None)
+    assert o.numel() == 0 and ST.numel() == 0
+
+
+def test_deterministic(g):
+    x = gi.chunk_inputs(2, 300, 4, 128, 128, dtype="bf16", seed=8, s0_std=0.05)
+    a = run_chunk(g, x)
+    b = run_chunk(g, x)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------- full workload sizes
+
+@pytest.fixture(scope="module")
+def prefill_4k():
+    return gi.chunk_inputs(**gi.PREFILL_4K, seed=0)
+
+
+def test_prefill_4k_sampled(g, prefill_4k):
+    """B=4, T=4096, H=16, d=128, BF16 q/k/v, FP32 gates, S0 = 0 (the prefill workload)."""
+    o, ST = run_chunk(g, prefill_4k)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(ST))
+    check_sampled(prefill_4k, o, ST, [(0, 0), (1, 7), (2, 11), (3, 15)], TOL_BF16_O, TOL_BF16_S)
+
+
+@pytest.mark.parametrize("variant", ["kda", "gdn"])
+def test_reductions_at_prefill_shape(g, variant):
+    """b = w = beta per (token, head): matches the separately coded KDA recurrence; with scalar
+    alpha as well, the Gated DeltaNet recurrence ("Independent decisions on two axes")."""
+    x = gi.chunk_inputs(**gi.PREFILL_4K, seed=0, gates=variant)
+    o, ST = run_chunk(g, x)
+    check_sampled(x, o, ST, [(1, 3), (3, 12)], TOL_BF16_O, TOL_BF16_S, ref=variant)
+
+
+@pytest.fixture(scope="module")
+def long_ragged():
+    return gi.chunk_inputs(**gi.LONG_RAGGED, seed=0)
+
+
+def test_long_ragged_sampled(g, long_ragged):
+    """B=1, T=65573 (not a multiple of 64), H=16, d=128, S0 ~ N(0, 0.02^2)."""
+    o, ST = run_chunk(g, long_ragged)
+    check_sampled(long_ragged, o, ST, [(0, 2), (0, 9)], TOL_BF16_O, TOL_BF16_S)
+
+
+def test_long_ragged_split_chaining(g, long_ragged):
+    """Splitting at T1 = floor(T/2) and chaining S_T into the second call equals one call."""
+    x = long_ragged
+    T = x["T"]
+    T1 = T // 2
+    d = to_dev(x)
+    o_full, S_full = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], d["S0"])
+    parts = [{n: d[n][:, sl].contiguous() for n in ("q", "k", "v", "alpha", "b", "w")}
+             for sl in (slice(0, T1), slice(T1, T))]
+    oa, Sa = g.gdn2_chunk_fwd(*(parts[0][n] for n in ("q", "k", "v", "alpha", "b", "w")), d["S0"])
+    ob, Sb = g.gdn2_chunk_fwd(*(parts[1][n] for n in ("q", "k", "v", "alpha", "b", "w")), Sa)
+    torch.cuda.synchronize()
+    o_split = torch.cat([oa, ob], 1).float().cpu().numpy()
+    assert rel(o_split, o_full.float().cpu().numpy()) <= TOL_BF16_O
+    assert rel(Sb.cpu().numpy(), S_full.cpu().numpy()) <= TOL_BF16_S
+    check_sampled(x, o_split, Sb.cpu().numpy(), [(0, 5)], TOL_BF16_O, TOL_BF16_S)
+
+
+# ---------------------------------------------------------------- decode step
+
+def run_decode(g, x, steps):
+    dt = torch.bfloat16 if x["dtype"] == "bf16" else torch.float32
+    dev = {n: torch.from_numpy(x[n]).cuda().to(dt if n in ("q", "k", "v") else torch.float32)
+           for n in ("q", "k", "v", "alpha", "b", "w")}
+    S = torch.from_numpy(x["S0"]).cuda()
+    outs = []
+    for s in range(steps):
+        outs.append(g.gdn2_recurrent_step(*(dev[n][s] for n in ("q", "k", "v", "alpha", "b", "w")), S))
+    torch.cuda.synchronize()
+    return torch.stack(outs).float().cpu().numpy(), S.cpu().numpy()
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64), (64, 128)])
+def test_decode_small(g, dtype, dk, dv):
+    x = gi.decode_inputs(5, 3, 4, dk, dv, dtype=dtype, seed=dk + dv, s0_std=0.1)
+    o, S = run_decode(g, x, 5)
+    S_ref = x["S0"].astype(np.float64)
+    tol_o, tol_s = (TOL_FP32, TOL_FP32) if dtype == "fp32" else (TOL_BF16_O, TOL_BF16_S)
+    for s in range(5):
+        o_ref, S_ref = oracle.gdn2_step(*(x[n][s] for n in ("q", "k", "v", "alpha", "b", "w")), S_ref)
+        assert rel(o[s], o_ref) <= tol_o
+    assert rel(S, S_ref) <= tol_s
+
+
+def test_decode_b256_64_steps_sampled(g):
+    """Batch 256, H=16, d=128, FP32 state N(0, 0.02^2), 64 consecutive in-place steps."""
+    x = gi.decode_inputs(**gi.DECODE_B256, seed=0)
+    o, S = run_decode(g, x, 64)
+    pairs = [(0, 0), (17, 5), (128, 9), (255, 15), (200, 3), (64, 12)]
+    Sr = np.stack([x["S0"][b, h] for b, h in pairs])[:, None].astype(np.float64)
+    for s in range(64):
+        args = [np.stack([x[n][s, b, h] for b, h in pairs])[:, None] for n in ("q", "k", "v", "alpha", "b", "w")]
+        o_ref, Sr = oracle.gdn2_step(*args, Sr)
+        og = np.stack([o[s, b, h] for b, h in pairs])[:, None]
+        assert rel(og, o_ref) <= TOL_BF16_O, f"step {s}"
+    Sg = np.stack([S[b, h] for b, h in pairs])[:, None]
+    assert rel(Sg, Sr) <= TOL_BF16_S
+    assert np.all(np.isfinite(S))
+
+
+def test_decode_equals_chunk_of_one_token(g):
+    """The two modes compute the same mathematics: T = 1 prefill equals one decode step."""
+    x = gi.chunk_inputs(4, 1, 3, 128, 128, dtype="fp32", seed=21, s0_std=0.1)
+    d = to_dev(x)
+    o_c, S_c = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], d["S0"])
+    S = d["S0"].clone()
+    o_d = g.gdn2_recurrent_step(*(d[n][:, 0].contiguous() for n in ("q", "k", "v", "alpha", "b", "w")), S)
+    torch.cuda.synchronize()
+    assert rel(o_d.cpu().numpy(), o_c[:, 0].cpu().numpy()) <= TOL_FP32
+    assert rel(S.cpu().numpy(), S_c.cpu().numpy()) <= TOL_FP32
