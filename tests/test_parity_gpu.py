@@ -2,9 +2,19 @@
 
 Error metric: max |x_gpu - x_ref| / RMS(x_ref) over the compared tensor.
 Tolerances: FP32 inputs 1e-4 (o and S_T); BF16 q/k/v with FP32 gates and
-accumulation: o 2e-2, S_T 1e-2.  At full workload sizes the oracle recomputes a
-sample of (batch, head) pairs -- every head is an independent recurrence, so a
-sampled head is compared element by element over all tokens.
+accumulation: o 2e-2, S_T 1e-2.
+
+A BF16 output o cannot be closer to the exact value than its own rounding:
+half a BF16 ulp is up to 2^-8 of |o|, and on these workloads max|o| reaches
+15-20 x RMS(o), so rounding the exact FP64 result to BF16 alone gives
+max|delta|/RMS of 0.035-0.048.  For BF16 outputs the 2e-2 bound therefore
+applies to the error beyond that rounding: each element's |delta| is reduced by
+half a BF16 ulp at its magnitude before the max is taken (``rel_bf16``).  The
+normwise error RMS(delta)/RMS(ref) is checked as well (<= 1e-2).
+
+At full workload sizes the oracle recomputes a sample of (batch, head) pairs --
+every head is an independent recurrence, so a sampled head is compared element
+by element over all tokens.
 """
 import numpy as np
 import pytest
@@ -24,6 +34,42 @@ def rel(x, ref):
     x = np.asarray(x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     return float(np.max(np.abs(x - ref)) / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
+
+
+def half_ulp_bf16(a):
+    """Half a BF16 ulp at magnitude |a| (8-bit significand): 2^(floor(log2|a|) - 8)."""
+    a = np.abs(a)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8.0), 0.0)
+
+
+def rel_bf16(x, ref):
+    """max(|x - ref| - half BF16 ulp, 0) / RMS(ref): error beyond the output's own rounding."""
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    slack = half_ulp_bf16(np.maximum(np.abs(ref), np.abs(x)))
+    excess = np.maximum(np.abs(x - ref) - slack, 0.0)
+    return float(np.max(excess) / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
+
+
+def rel_rms(x, ref):
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.sqrt(np.mean((x - ref) ** 2)) / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
+
+
+TOL_BF16_O_RMS = 1e-2
+
+
+def check_o(x, ref, dtype):
+    if dtype == "fp32":
+        e = rel(x, ref)
+        assert e <= TOL_FP32, f"o error {e:.3e} > {TOL_FP32}"
+    else:
+        e, en = rel_bf16(x, ref), rel_rms(x, ref)
+        assert e <= TOL_BF16_O, f"o error beyond BF16 rounding {e:.3e} > {TOL_BF16_O}"
+        assert en <= TOL_BF16_O_RMS, f"o normwise error {en:.3e} > {TOL_BF16_O_RMS}"
+    return e
 
 
 @pytest.fixture(scope="module")
@@ -61,7 +107,7 @@ def sel_heads(x, pairs):
     return out
 
 
-def check_sampled(x, o, ST, pairs, tol_o, tol_s, ref="gdn2"):
+def check_sampled(x, o, ST, pairs, tol_s, ref="gdn2"):
     s = sel_heads(x, pairs)
     if ref == "gdn2":
         o_ref, S_ref = oracle.gdn2(s["q"], s["k"], s["v"], s["alpha"], s["b"], s["w"], s["S0"])
@@ -73,8 +119,7 @@ def check_sampled(x, o, ST, pairs, tol_o, tol_s, ref="gdn2"):
         a1 = np.stack([x["alpha_scalar"][b, :, h] for b, h in pairs])[:, :, None]
         o_ref, S_ref = oracle.gdn(s["q"], s["k"], s["v"], a1, beta, s["S0"])
     og = np.stack([o[b, :, h] for b, h in pairs])[:, :, None]
-    eo = rel(og, o_ref)
-    assert eo <= tol_o, f"o error {eo:.3e} > {tol_o}"
+    eo = check_o(og, o_ref, x["dtype"])
     if ST is not None:
         Sg = np.stack([ST[b, h] for b, h in pairs])[:, None]
         es = rel(Sg, S_ref)
@@ -101,10 +146,8 @@ def test_small_full(g, dtype, T, d):
     x = gi.chunk_inputs(2, T, 3, d, d, dtype=dtype, seed=T + d, s0_std=0.05)
     o, ST = run_chunk(g, x)
     o_ref, S_ref = oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], x["S0"])
-    if dtype == "fp32":
-        assert rel(o, o_ref) <= TOL_FP32 and rel(ST, S_ref) <= TOL_FP32
-    else:
-        assert rel(o, o_ref) <= TOL_BF16_O and rel(ST, S_ref) <= TOL_BF16_S
+    check_o(o, o_ref, dtype)
+    assert rel(ST, S_ref) <= (TOL_FP32 if dtype == "fp32" else TOL_BF16_S)
 
 
 def test_delta_identity_fp32(g):
@@ -172,7 +215,7 @@ def test_prefill_4k_sampled(g, prefill_4k):
     """B=4, T=4096, H=16, d=128, BF16 q/k/v, FP32 gates, S0 = 0 (the prefill workload)."""
     o, ST = run_chunk(g, prefill_4k)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(ST))
-    check_sampled(prefill_4k, o, ST, [(0, 0), (1, 7), (2, 11), (3, 15)], TOL_BF16_O, TOL_BF16_S)
+    check_sampled(prefill_4k, o, ST, [(0, 0), (1, 7), (2, 11), (3, 15)], TOL_BF16_S)
 
 
 @pytest.mark.parametrize("variant", ["kda", "gdn"])
@@ -181,7 +224,7 @@ def test_reductions_at_prefill_shape(g, variant):
     alpha as well, the Gated DeltaNet recurrence ("Independent decisions on two axes")."""
     x = gi.chunk_inputs(**gi.PREFILL_4K, seed=0, gates=variant)
     o, ST = run_chunk(g, x)
-    check_sampled(x, o, ST, [(1, 3), (3, 12)], TOL_BF16_O, TOL_BF16_S, ref=variant)
+    check_sampled(x, o, ST, [(1, 3), (3, 12)], TOL_BF16_S, ref=variant)
 
 
 @pytest.fixture(scope="module")
@@ -192,7 +235,7 @@ def long_ragged():
 def test_long_ragged_sampled(g, long_ragged):
     """B=1, T=65573 (not a multiple of 64), H=16, d=128, S0 ~ N(0, 0.02^2)."""
     o, ST = run_chunk(g, long_ragged)
-    check_sampled(long_ragged, o, ST, [(0, 2), (0, 9)], TOL_BF16_O, TOL_BF16_S)
+    check_sampled(long_ragged, o, ST, [(0, 2), (0, 9)], TOL_BF16_S)
 
 
 def test_long_ragged_split_chaining(g, long_ragged):
@@ -208,9 +251,9 @@ def test_long_ragged_split_chaining(g, long_ragged):
     ob, Sb = g.gdn2_chunk_fwd(*(parts[1][n] for n in ("q", "k", "v", "alpha", "b", "w")), Sa)
     torch.cuda.synchronize()
     o_split = torch.cat([oa, ob], 1).float().cpu().numpy()
-    assert rel(o_split, o_full.float().cpu().numpy()) <= TOL_BF16_O
+    assert rel_bf16(o_split, o_full.float().cpu().numpy()) <= TOL_BF16_O
     assert rel(Sb.cpu().numpy(), S_full.cpu().numpy()) <= TOL_BF16_S
-    check_sampled(x, o_split, Sb.cpu().numpy(), [(0, 5)], TOL_BF16_O, TOL_BF16_S)
+    check_sampled(x, o_split, Sb.cpu().numpy(), [(0, 5)], TOL_BF16_S)
 
 
 # ---------------------------------------------------------------- decode step
@@ -233,10 +276,10 @@ def test_decode_small(g, dtype, dk, dv):
     x = gi.decode_inputs(5, 3, 4, dk, dv, dtype=dtype, seed=dk + dv, s0_std=0.1)
     o, S = run_decode(g, x, 5)
     S_ref = x["S0"].astype(np.float64)
-    tol_o, tol_s = (TOL_FP32, TOL_FP32) if dtype == "fp32" else (TOL_BF16_O, TOL_BF16_S)
+    tol_s = TOL_FP32 if dtype == "fp32" else TOL_BF16_S
     for s in range(5):
         o_ref, S_ref = oracle.gdn2_step(*(x[n][s] for n in ("q", "k", "v", "alpha", "b", "w")), S_ref)
-        assert rel(o[s], o_ref) <= tol_o
+        check_o(o[s], o_ref, dtype)
     assert rel(S, S_ref) <= tol_s
 
 
@@ -250,7 +293,7 @@ def test_decode_b256_64_steps_sampled(g):
         args = [np.stack([x[n][s, b, h] for b, h in pairs])[:, None] for n in ("q", "k", "v", "alpha", "b", "w")]
         o_ref, Sr = oracle.gdn2_step(*args, Sr)
         og = np.stack([o[s, b, h] for b, h in pairs])[:, None]
-        assert rel(og, o_ref) <= TOL_BF16_O, f"step {s}"
+        check_o(og, o_ref, "bf16")
     Sg = np.stack([S[b, h] for b, h in pairs])[:, None]
     assert rel(Sg, Sr) <= TOL_BF16_S
     assert np.all(np.isfinite(S))
