@@ -19,7 +19,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_recurrent_step", "library_path", "load_library", "exported_symbols",
+__all__ = ["gdn2_chunk_fwd", "gdn2_recurrent_step", "gdn2_device_error", "library_path", "load_library", "exported_symbols",
            "GDN2_OK", "GDN2_ERR_INVALID_ARG", "GDN2_ERR_UNSUPPORTED", "GDN2_ERR_CUDA", "Gdn2Error"]
 
 GDN2_OK, GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_CUDA = 0, 1, 2, 3
@@ -58,6 +58,8 @@ def load_library(rebuild_if_stale: bool = True) -> ctypes.CDLL:
     lib.gdn2_last_error.argtypes = []
     lib.gdn2_last_error.restype = ctypes.c_char_p
     lib.gdn2_version.restype = i
+    lib.gdn2_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
+    lib.gdn2_device_error.restype = i
     _lib = lib
     return lib
 
@@ -102,6 +104,14 @@ def _stream(stream, device):
     if stream is None:
         stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def gdn2_device_error(clear: bool = True) -> int:
+    """Synchronously read (and by default clear) the kernels' device-side failure flag."""
+    lib = load_library()
+    code = ctypes.c_uint(0)
+    _check(lib.gdn2_device_error(ctypes.byref(code), int(clear)))
+    return int(code.value)
 
 
 def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, *, o=None, S_T=None, output_final_state=True,

@@ -10,6 +10,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                             const float *w, const float *S0, void *o, float *S_T, int B, int T, int H,
                             cudaStream_t stream);
 bool chunk_tc_supported(int dk, int dv, gdn2_dtype dt);
+cudaError_t read_device_error(unsigned int *value, bool clear);
 }  // namespace gdn2
 
 namespace {
@@ -67,6 +68,11 @@ const char *gdn2_status_string(gdn2_status s) {
 const char *gdn2_last_error(void) { return g_last_error; }
 
 int gdn2_version(void) { return 100; }
+
+gdn2_status gdn2_device_error(unsigned int *code, int clear) {
+    if (!code) return fail(GDN2_ERR_INVALID_ARG, "%s", "null pointer: code");
+    return cuda_status(gdn2::read_device_error(code, clear != 0), "gdn2_device_error");
+}
 
 gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *b,
                            const float *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,

@@ -114,6 +114,13 @@ const char *gdn2_status_string(gdn2_status s);
  * thread-local buffer, valid until the next call on the same thread). */
 const char *gdn2_last_error(void);
 
+/* Device-side failure flag of the current device (synchronous; call between
+ * launches).  *code = 0 when every kernel finished normally; nonzero when a
+ * bounded wait inside a kernel gave up (the kernel then skipped its remaining
+ * work, released its resources and returned; outputs of that call are
+ * undefined).  clear != 0 resets the flag. */
+gdn2_status gdn2_device_error(unsigned int *code, int clear);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int gdn2_version(void);
 

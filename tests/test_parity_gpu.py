@@ -309,3 +309,8 @@ def test_decode_equals_chunk_of_one_token(g):
     torch.cuda.synchronize()
     assert rel(o_d.cpu().numpy(), o_c[:, 0].cpu().numpy()) <= TOL_FP32
     assert rel(S.cpu().numpy(), S_c.cpu().numpy()) <= TOL_FP32
+
+
+def test_zz_no_device_error_flag(g):
+    """No bounded wait inside any kernel gave up during the parity runs above."""
+    assert g.gdn2_device_error(clear=True) == 0
