@@ -9,26 +9,31 @@
 //
 //   gamma_t = prod_{j<=t} alpha_j,  rho_t = 1/gamma_t          (per key channel, FP32)
 //   Etil = b*k*gamma,  Qtil = q*gamma,  Ktil = k*rho,  Z = w*v   (gate prep)
-//   A = strict_tril(Etil Ktil^T),  P = tril(Qtil Ktil^T)         (Gram, tensor core)
-//   T = (I + A)^{-1}                                            (FP32 blocked solve)
-//   W = T Etil,  Y = T Z                                        (tensor core)
-//   U = Y - W S                                                 (tensor core + epilogue)
-//   O = Qtil S + P U                                            (tensor core)
-//   S <- diag(gamma_n) (S + Ktil^T U)                           (tensor core + FP32 epilogue)
+//   [A | Etil S] and [P | Qtil S] = [Etil; Qtil] [Ktil; S^T]^T  (one tensor-core product)
+//   A <- strict_tril(A),  P <- tril(P),  T = (I + A)^{-1}        (FP32 blocked solve)
+//   R = Z - Etil S                                               (FP32 epilogue)
+//   U = T R                                                      (tensor core)
+//   O = Qtil S + P U                                             (tensor core, accumulated)
+//   S <- diag(gamma_n) (S + Ktil^T U)                            (tensor core + FP32 epilogue)
 //
-// Precision: every operand is rounded to TF32 (10-bit mantissa); accumulation,
-// decay, solve and the carried state are FP32.  With BF16 operands the products
-// of decay-scaled factors lose too much (the read r = Sbar^T e nearly cancels
-// the write z in the delta rule), so TF32 is used throughout.  The key factor
-// Ktil = k / gamma grows within a chunk as exp(-sum ln alpha); the kernel
-// requires that growth to stay below ~1e34 (sum of -ln alpha over one chunk
-// <= 78 per key channel), documented in gdn2.h.
+// U holds the per-token corrections z_t - r_t of the token recurrence, so this
+// is the same arithmetic as the token loop, re-associated.
+//
+// Precision: tensor-core operands are rounded to TF32 (10-bit mantissa);
+// accumulation, decay, solve, R and the carried state are FP32.  BF16 operands
+// lose too much here: the read r = Sbar^T e nearly cancels the write z in the
+// delta rule, and products of decay-scaled factors carry that error into o and
+// S.  The key factor Ktil = k / gamma grows within a chunk as
+// exp(-sum ln alpha); it must stay below ~1e34 (sum of -ln alpha over one chunk
+// <= 78 per key channel), as documented in gdn2.h.
 //
 // Layout: one CTA per (batch, head, 64-column half of d_v); 256 threads (8
 // warps) run the phases of a chunk in turn; thread 0 issues TMA loads and MMAs.
-// alpha, b and w are TMA-loaded (128-byte swizzle) straight into the operand
-// tiles they become (Ktil, Etil, Z) and transformed in place, so a chunk needs
-// ~220 KB of shared memory.  Tensor Memory: 512 columns.
+// Every shared-memory operand is K-major with the 128-byte swizzle.  Operands
+// needed transposed (Ktil^T, [T; P]) are written to Tensor Memory and read from
+// there as the A operand.  alpha, b and w are TMA-loaded straight into the
+// tiles they become and transformed in place; the next chunk's loads are
+// issued as soon as each tile is consumed.
 #include <cudaTypedefs.h>
 #include <stdio.h>
 
@@ -49,55 +54,53 @@ constexpr int kDVS = 64;          // value columns per CTA
 constexpr int kThreads = 256;
 constexpr long long kWaitLimit = 4000000000ll;   // ~2 s of SM cycles per wait
 
-// Shared-memory map (bytes from a 1024-aligned base).  128-byte-swizzled tiles
-// of FP32/TF32 elements, 32 elements per 128-byte row:
-//   X1  [Etil -> W ; Qtil]  K-major, 128 rows x 128 channels, 4 atoms of 16 KB
-//   KT  Ktil                 64 tokens x 128 channels, 4 atoms of 8 KB
-//   ZU  Z, later U           64 tokens x 64 columns, 2 atoms of 8 KB
-//   TP  [T ; P]              K-major, 128 rows x 64 tokens, 2 atoms of 16 KB
-//   ST  S (operand copy)     128 channels x 64 columns, 2 atoms of 16 KB
-// Raw (unswizzled) BF16 staging for q, k (64 x 128) and v (64 x 64).
+// Shared-memory map (bytes from a 1024-aligned base).  Tiles hold FP32/TF32,
+// 32 elements per 128-byte swizzled row, K-major:
+//   X1  rows 0-63 Etil[t][i], rows 64-127 Qtil[t][i]     4 atoms x 16 KB (i = key channel)
+//   KS  rows 0-63 Ktil[s][i], rows 64-127 S[i][j] as [j][i]   4 atoms x 16 KB
+//   RU  R, later U, as [j][t]                             2 atoms x 8 KB (t = token)
+//   ZW  w, then Z = w*v, as [t][j] (FP32, epilogue only)   2 atoms x 8 KB
+// and unswizzled BF16 staging of q, k (64 x 128) and v (64 x 64).
 constexpr uint32_t OFF_X1 = 0;
-constexpr uint32_t OFF_KT = OFF_X1 + 65536;
-constexpr uint32_t OFF_ZU = OFF_KT + 32768;
-constexpr uint32_t OFF_TP = OFF_ZU + 16384;
-constexpr uint32_t OFF_ST = OFF_TP + 32768;
-constexpr uint32_t OFF_RQ = OFF_ST + 32768;
+constexpr uint32_t OFF_KS = OFF_X1 + 65536;
+constexpr uint32_t OFF_RU = OFF_KS + 65536;
+constexpr uint32_t OFF_ZW = OFF_RU + 16384;
+constexpr uint32_t OFF_RQ = OFF_ZW + 16384;
 constexpr uint32_t OFF_RK = OFF_RQ + 16384;
 constexpr uint32_t OFF_RV = OFF_RK + 16384;
 constexpr uint32_t OFF_GN = OFF_RV + 8192;      // float[128]   decay over the chunk
-constexpr uint32_t OFF_PART = OFF_GN + 512;     // float[4][128] partial decay products
-constexpr uint32_t OFF_BAR = OFF_PART + 2048;   // 6 mbarriers
+constexpr uint32_t OFF_PART = OFF_GN + 512;     // float[2][128] half-chunk decay products
+constexpr uint32_t OFF_BAR = OFF_PART + 1024;   // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 64;     // tmem base, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // + alignment slack
-// Solve scratch, inside the q/k staging (free between prep and the next load).
-constexpr uint32_t OFF_AS = OFF_RQ;             // float[64][65]  A (strictly lower)
-constexpr uint32_t OFF_XS = OFF_RQ + 16896;     // float[32][33]  block-product scratch
+// Solve scratch inside the q/k/v staging (free between prep and the next load).
 constexpr int LDA = 65, LDX = 33;
+constexpr uint32_t OFF_AS = OFF_RQ;                     // float[64][65] A, strictly lower
+constexpr uint32_t OFF_TS = OFF_AS + 16896;             // float[64][65] T
+constexpr uint32_t OFF_XS = OFF_TS + 16896;             // float[32][33] block products
+static_assert(OFF_XS + 32 * LDX * 4 <= OFF_GN, "solve scratch overflows the staging area");
 
-// Tensor Memory columns.
-constexpr uint32_t TM_G = 0;      // Gram: lanes 0-63 A, lanes 64-127 P          (64 cols)
-constexpr uint32_t TM_W = 64;     // W = T Etil (lanes 0-63)                      (128 cols)
-constexpr uint32_t TM_Y = 192;    // Y = T Z   (lanes 0-63)                       (64 cols)
-constexpr uint32_t TM_X = 256;    // lanes 0-63 W S, lanes 64-127 Qtil S + P U    (64 cols)
-constexpr uint32_t TM_D = 320;    // Ktil^T U                                     (64 cols)
+// Tensor Memory columns (512 allocated).
+constexpr uint32_t TM_G = 0;      // [Etil;Qtil] Ktil^T : lanes 0-63 A, lanes 64-127 P   (64 cols)
+constexpr uint32_t TM_X = 64;     // [Etil;Qtil] S, then + [T;P] U : lanes 64-127 -> O    (64 cols)
+constexpr uint32_t TM_U = 128;    // [T;P] R : lanes 0-63 U                               (64 cols)
+constexpr uint32_t TM_D = 192;    // Ktil^T U                                             (64 cols)
+constexpr uint32_t TM_KT = 256;   // A operand Ktil^T: lane i, column s                   (64 cols)
+constexpr uint32_t TM_TP = 320;   // A operand [T;P]: lane t (P at 64+t), column s        (64 cols)
 constexpr uint32_t TM_COLS = 512;
 
 enum { BAR_QKV = 0, BAR_A, BAR_B, BAR_W, BAR_MMA, NBARS };
 
-// TMA byte counts per chunk.
 constexpr uint32_t TX_QKV = 16384 + 16384 + 8192;
 constexpr uint32_t TX_A = 4 * 8192;
 constexpr uint32_t TX_B = 4 * 8192;
 constexpr uint32_t TX_W = 2 * 8192;
 
 // Element byte offsets inside the tiles.
-__device__ __forceinline__ uint32_t x1_off(uint32_t r, uint32_t i) { return (i >> 5) * 16384u + swz128(r, (i & 31u) * 4u); }
-__device__ __forceinline__ uint32_t kt_off(uint32_t t, uint32_t i) { return (i >> 5) * 8192u + swz128(t, (i & 31u) * 4u); }
-__device__ __forceinline__ uint32_t zu_off(uint32_t t, uint32_t j) { return (j >> 5) * 8192u + swz128(t, (j & 31u) * 4u); }
-__device__ __forceinline__ uint32_t tp_off(uint32_t r, uint32_t s) { return (s >> 5) * 16384u + swz128(r, (s & 31u) * 4u); }
-__device__ __forceinline__ uint32_t st_off(uint32_t i, uint32_t j) { return (j >> 5) * 16384u + swz128(i, (j & 31u) * 4u); }
+__device__ __forceinline__ uint32_t x_off(uint32_t r, uint32_t i) { return (i >> 5) * 16384u + swz128(r, (i & 31u) * 4u); }
+__device__ __forceinline__ uint32_t ru_off(uint32_t j, uint32_t t) { return (t >> 5) * 8192u + swz128(j, (t & 31u) * 4u); }
+__device__ __forceinline__ uint32_t zw_off(uint32_t t, uint32_t j) { return (j >> 5) * 8192u + swz128(t, (j & 31u) * 4u); }
 
 struct Maps {
     CUtensorMap q, k, v, alpha, b, w;
@@ -110,8 +113,9 @@ struct Ctx {
 };
 
 __device__ __forceinline__ float *fptr(const Ctx &c, uint32_t off) { return reinterpret_cast<float *>(c.sm + off); }
+__device__ __forceinline__ float &at(const Ctx &c, uint32_t off) { return *reinterpret_cast<float *>(c.sm + off); }
 
-// Issue the TMA loads of one chunk's inputs (thread 0 only).
+// TMA loads of one chunk's inputs (thread 0 only).
 __device__ __forceinline__ void load_qkv(const Ctx &c, const Maps &m, int h, int t0, int bidx, int col0) {
     mbar_expect_tx(c.bar[BAR_QKV], TX_QKV);
     tma_load_4d(c.sa + OFF_RQ, &m.q, 0, h, t0, bidx, c.bar[BAR_QKV]);
@@ -119,106 +123,74 @@ __device__ __forceinline__ void load_qkv(const Ctx &c, const Maps &m, int h, int
     tma_load_4d(c.sa + OFF_RV, &m.v, col0, h, t0, bidx, c.bar[BAR_QKV]);
 }
 __device__ __forceinline__ void load_alpha(const Ctx &c, const Maps &m, int h, int t0, int bidx) {
-    mbar_expect_tx(c.bar[BAR_A], TX_A);
-    for (int a = 0; a < 4; ++a) tma_load_4d(c.sa + OFF_KT + a * 8192, &m.alpha, 32 * a, h, t0, bidx, c.bar[BAR_A]);
+    mbar_expect_tx(c.bar[BAR_A], TX_A);   // rows 0-63 of each KS atom
+    for (int a = 0; a < 4; ++a) tma_load_4d(c.sa + OFF_KS + a * 16384, &m.alpha, 32 * a, h, t0, bidx, c.bar[BAR_A]);
 }
 __device__ __forceinline__ void load_b(const Ctx &c, const Maps &m, int h, int t0, int bidx) {
-    mbar_expect_tx(c.bar[BAR_B], TX_B);
+    mbar_expect_tx(c.bar[BAR_B], TX_B);   // rows 0-63 of each X1 atom
     for (int a = 0; a < 4; ++a) tma_load_4d(c.sa + OFF_X1 + a * 16384, &m.b, 32 * a, h, t0, bidx, c.bar[BAR_B]);
 }
 __device__ __forceinline__ void load_w(const Ctx &c, const Maps &m, int h, int t0, int bidx, int col0) {
     mbar_expect_tx(c.bar[BAR_W], TX_W);
-    for (int a = 0; a < 2; ++a) tma_load_4d(c.sa + OFF_ZU + a * 8192, &m.w, col0 + 32 * a, h, t0, bidx, c.bar[BAR_W]);
+    for (int a = 0; a < 2; ++a) tma_load_4d(c.sa + OFF_ZW + a * 8192, &m.w, col0 + 32 * a, h, t0, bidx, c.bar[BAR_W]);
 }
 
-__device__ __forceinline__ float2 ldbf2(const uint8_t *p) {
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(p);
-    return __bfloat1622float2(x);
-}
-__device__ __forceinline__ void st_tf32x2(uint8_t *p, float a, float b) {
-    *reinterpret_cast<float2 *>(p) = make_float2(to_tf32(a), to_tf32(b));
-}
-__device__ __forceinline__ void st_tf32x4(uint8_t *p, float a, float b, float c, float d) {
-    *reinterpret_cast<float4 *>(p) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
-}
+__device__ __forceinline__ float ldbf(const uint8_t *p) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p)); }
 
 // ---------------------------------------------------------------------------
-// Gate prep: cumulative decay along the chunk (running FP32 products, equal to
-// exp of the cumulative log-decay up to rounding) and the operand factors,
-// written in place over the loaded gates.  Padding tokens (t >= n) have zero
-// q, k, b, w, v from the TMA bounds fill and alpha forced to 1.
-__device__ __forceinline__ void prep(const Ctx &c, int tid, int n) {
-    const int cp = tid & 63, tq = tid >> 6;        // channel pair, token quarter
-    const uint32_t ch = 2u * cp;
+// Gate prep.  Thread (lane quarter qd, half th, lane l) owns key channel
+// i = 32 qd + l for tokens [32 th, 32 th + 32).  Cumulative decay is a running
+// FP32 product (exp of the cumulative log-decay up to rounding).  Padding tokens
+// (t >= n) have zero q, k, b, w, v from the TMA bounds fill and alpha forced to 1.
+__device__ __forceinline__ void prep(const Ctx &c, uint32_t tmem, int tid, int qd, int th, int lane, int n) {
+    const int i = 32 * qd + lane;
     float *part = fptr(c, OFF_PART);
-    float2 pa = make_float2(1.f, 1.f);
-    for (int t = 16 * tq; t < 16 * tq + 16; ++t) {
-        if (t < n) {
-            const float2 a = *reinterpret_cast<const float2 *>(c.sm + OFF_KT + kt_off(t, ch));
-            pa.x *= clamp_alpha(a.x);
-            pa.y *= clamp_alpha(a.y);
-        }
-    }
-    part[tq * 128 + ch] = pa.x;
-    part[tq * 128 + ch + 1] = pa.y;
+    float pa = 1.f;
+    for (int t = 32 * th; t < 32 * th + 32; ++t)
+        if (t < n) pa *= clamp_alpha(at(c, OFF_KS + x_off(t, i)));
+    part[th * 128 + i] = pa;
     __syncthreads();
-    float g0 = 1.f, g1 = 1.f, tot0 = 1.f, tot1 = 1.f;
-    for (int q2 = 0; q2 < 4; ++q2) {
-        const float p0 = part[q2 * 128 + ch], p1 = part[q2 * 128 + ch + 1];
-        if (q2 < tq) { g0 *= p0; g1 *= p1; }
-        tot0 *= p0; tot1 *= p1;
+    const float p0 = part[i], p1 = part[128 + i];
+    if (th == 0) fptr(c, OFF_GN)[i] = p0 * p1;
+    float g = th ? p0 : 1.f;
+    float r = 1.f / g;
+    float kt[32];
+#pragma unroll
+    for (int tt = 0; tt < 32; ++tt) {
+        const int t = 32 * th + tt;
+        const uint32_t o = x_off(t, i);
+        float a = (t < n) ? clamp_alpha(at(c, OFF_KS + o)) : 1.f;
+        g *= a;
+        r *= __fdividef(1.f, a);
+        const float kk = ldbf(c.sm + OFF_RK + t * 256 + i * 2);
+        const float qq = ldbf(c.sm + OFF_RQ + t * 256 + i * 2);
+        const float bb = at(c, OFF_X1 + o);
+        at(c, OFF_X1 + o) = to_tf32(bb * kk * g);
+        at(c, OFF_X1 + x_off(64 + t, i)) = to_tf32(qq * g);
+        kt[tt] = to_tf32(kk * r);
+        at(c, OFF_KS + o) = kt[tt];
     }
-    if (tq == 0) {
-        float *gn = fptr(c, OFF_GN);
-        gn[ch] = tot0;
-        gn[ch + 1] = tot1;
-    }
-    float r0 = 1.f / g0, r1 = 1.f / g1;
-    for (int t = 16 * tq; t < 16 * tq + 16; ++t) {
-        uint8_t *pk = c.sm + OFF_KT + kt_off(t, ch);
-        uint8_t *pe = c.sm + OFF_X1 + x1_off(t, ch);
-        uint8_t *pq = c.sm + OFF_X1 + x1_off(64 + t, ch);
-        float2 a = *reinterpret_cast<const float2 *>(pk);
-        if (t >= n) a = make_float2(1.f, 1.f);
-        a.x = clamp_alpha(a.x);
-        a.y = clamp_alpha(a.y);
-        g0 *= a.x; g1 *= a.y;
-        r0 *= __fdividef(1.f, a.x);
-        r1 *= __fdividef(1.f, a.y);
-        const float2 kk = ldbf2(c.sm + OFF_RK + t * 256 + ch * 2);
-        const float2 qq = ldbf2(c.sm + OFF_RQ + t * 256 + ch * 2);
-        const float2 bb = *reinterpret_cast<const float2 *>(pe);
-        st_tf32x2(pe, bb.x * kk.x * g0, bb.y * kk.y * g1);
-        st_tf32x2(pq, qq.x * g0, qq.y * g1);
-        st_tf32x2(pk, kk.x * r0, kk.y * r1);
-    }
-    // Z = w * v in place over w.
+    tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + TM_KT + 32 * th, kt);
+    // Z = w * v in place over w (FP32; used only by the R epilogue).
     const int j2 = tid & 31, tg = tid >> 5;
     for (int m = 0; m < 8; ++m) {
         const int t = tg + 8 * m;
-        uint8_t *pz = c.sm + OFF_ZU + zu_off(t, 2 * j2);
-        const float2 w = *reinterpret_cast<const float2 *>(pz);
-        const float2 v = ldbf2(c.sm + OFF_RV + t * 128 + j2 * 4);
-        st_tf32x2(pz, w.x * v.x, w.y * v.y);
+        float2 *pz = reinterpret_cast<float2 *>(c.sm + OFF_ZW + zw_off(t, 2 * j2));
+        const float2 w = *pz;
+        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(c.sm + OFF_RV + t * 128 + j2 * 4);
+        const float2 vf = __bfloat1622float2(v);
+        *pz = make_float2(w.x * vf.x, w.y * vf.y);
     }
 }
 
 // ---------------------------------------------------------------------------
-// T = (I + A)^{-1}, A strictly lower 64 x 64 in As (FP32).  Blocked: 16 x 16
-// diagonal blocks by forward substitution, then the 16- and 32-wide
-// off-diagonal blocks by T_ab = -T_aa (sum_c A_ac T_cb).  T (FP32, zero above
-// the diagonal) is written into rows 0-63 of the TP tile.
-__device__ __forceinline__ float tget(const Ctx &c, int r, int s) {
-    return *reinterpret_cast<const float *>(c.sm + OFF_TP + tp_off(r, s));
-}
-__device__ __forceinline__ void tset(const Ctx &c, int r, int s, float x) {
-    *reinterpret_cast<float *>(c.sm + OFF_TP + tp_off(r, s)) = x;
-}
-
+// T = (I + A)^{-1}, A strictly lower 64 x 64 (FP32, As), result in Ts (FP32,
+// zero above the diagonal).  16 x 16 diagonal blocks by forward substitution,
+// then T_ab = -T_aa (sum_c A_ac T_cb) for the 16- and 32-wide off-diagonal blocks.
 __device__ __forceinline__ void solve(const Ctx &c, int tid) {
     const float *As = fptr(c, OFF_AS);
+    float *Ts = fptr(c, OFF_TS);
     float *Xs = fptr(c, OFF_XS);
-    // 1. Diagonal 16 x 16 blocks (64 threads: block a, column j); zero the upper blocks.
     if (tid < 64) {
         const int a = tid >> 4, j = tid & 15, base = 16 * a;
         float x[16];
@@ -230,25 +202,24 @@ __device__ __forceinline__ void solve(const Ctx &c, int tid) {
             x[i] = acc;
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) tset(c, base + i, base + j, x[i]);
+        for (int i = 0; i < 16; ++i) Ts[(base + i) * LDA + base + j] = x[i];
     } else {
-        // upper off-diagonal blocks (a < b): 6 blocks x 256 elements over 192 threads
-        for (int e = tid - 64; e < 6 * 256; e += 192) {
+        // zero the blocks above the diagonal: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+        for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
             const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
-            // blocks (a, b), a < b, in the order (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
             const int a = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
             const int b = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            tset(c, 16 * a + i, 16 * b + j, 0.f);
+            Ts[(16 * a + i) * LDA + 16 * b + j] = 0.f;
         }
     }
     __syncthreads();
-    // 2. T_10 = -T_11 A_10 T_00 and T_32 = -T_33 A_32 T_22.
+    // T_10 = -T_11 A_10 T_00 and T_32 = -T_33 A_32 T_22
     for (int e = tid; e < 512; e += kThreads) {
         const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
         const int a = blk ? 3 : 1, b = a - 1;
         float acc = 0.f;
 #pragma unroll
-        for (int l = 0; l < 16; ++l) acc = fmaf(As[(16 * a + i) * LDA + 16 * b + l], tget(c, 16 * b + l, 16 * b + j), acc);
+        for (int l = 0; l < 16; ++l) acc = fmaf(As[(16 * a + i) * LDA + 16 * b + l], Ts[(16 * b + l) * LDA + 16 * b + j], acc);
         Xs[blk * 16 * LDX + i * LDX + j] = acc;
     }
     __syncthreads();
@@ -257,16 +228,16 @@ __device__ __forceinline__ void solve(const Ctx &c, int tid) {
         const int a = blk ? 3 : 1, b = a - 1;
         float acc = 0.f;
 #pragma unroll
-        for (int l = 0; l < 16; ++l) acc = fmaf(tget(c, 16 * a + i, 16 * a + l), Xs[blk * 16 * LDX + l * LDX + j], acc);
-        tset(c, 16 * a + i, 16 * b + j, -acc);
+        for (int l = 0; l < 16; ++l) acc = fmaf(Ts[(16 * a + i) * LDA + 16 * a + l], Xs[blk * 16 * LDX + l * LDX + j], acc);
+        Ts[(16 * a + i) * LDA + 16 * b + j] = -acc;
     }
     __syncthreads();
-    // 3. Lower-left 32 x 32 block: T_BA = -T_BB A_BA T_AA.
+    // lower-left 32 x 32 block: T_BA = -T_BB A_BA T_AA
     for (int e = tid; e < 1024; e += kThreads) {
         const int i = e >> 5, j = e & 31;
         float acc = 0.f;
 #pragma unroll 8
-        for (int l = 0; l < 32; ++l) acc = fmaf(As[(32 + i) * LDA + l], tget(c, l, j), acc);
+        for (int l = 0; l < 32; ++l) acc = fmaf(As[(32 + i) * LDA + l], Ts[l * LDA + j], acc);
         Xs[i * LDX + j] = acc;
     }
     __syncthreads();
@@ -274,9 +245,10 @@ __device__ __forceinline__ void solve(const Ctx &c, int tid) {
         const int i = e >> 5, j = e & 31;
         float acc = 0.f;
 #pragma unroll 8
-        for (int l = 0; l < 32; ++l) acc = fmaf(tget(c, 32 + i, 32 + l), Xs[l * LDX + j], acc);
-        tset(c, 32 + i, j, -acc);
+        for (int l = 0; l < 32; ++l) acc = fmaf(Ts[(32 + i) * LDA + 32 + l], Xs[l * LDX + j], acc);
+        Ts[(32 + i) * LDA + j] = -acc;
     }
+    __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -297,6 +269,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
     const int bidx = head / H, h = head % H;
     const int col0 = half * kDVS;
     const int nchunks = (T + kC - 1) / kC;
+    const int srow = 32 * qd + lane;                    // the TMEM lane this thread reads
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i) mbar_init(c.bar[i], 1);
@@ -313,6 +286,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);   // this warp's lane quarter
     if (tid == 0) {
         load_qkv(c, maps, h, 0, bidx, col0);
         load_alpha(c, maps, h, 0, bidx);
@@ -320,9 +294,9 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         load_w(c, maps, h, 0, bidx, col0);
     }
 
-    // State slice owned by this thread: key channel i = 32*qd + lane, value
-    // columns col0 + 32*chh + [0, 32).  FP32 in registers across all chunks.
-    const int srow = 32 * qd + lane;
+    // State slice owned by this thread: key channel i = srow, value columns
+    // col0 + 32*chh + [0, 32).  FP32 in registers across all chunks; its TF32
+    // copy is KS rows 64 + j (j = local column), channel i.
     float S[32];
     {
         const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 32 * chh;
@@ -332,14 +306,11 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-            st_tf32x4(c.sm + OFF_ST + st_off(srow, 32 * chh + j), S[j], S[j + 1], S[j + 2], S[j + 3]);
+        for (int j = 0; j < 32; ++j) at(c, OFF_KS + x_off(64 + 32 * chh + j, srow)) = to_tf32(S[j]);
     }
 
-    const uint32_t tq_lane = (uint32_t)(32 * qd) << 16;   // TMEM lane field of this warp
     uint32_t mma_phase = 0;
     bool ok = true;
-
     auto wait_all = [&](int which, uint32_t parity) {
         if (!mbar_wait(c.bar[which], parity, kWaitLimit)) {
             *abort_flag = 1;
@@ -354,6 +325,11 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         tc_fence_after();
         return r;
     };
+    auto sync_for_mma = [&]() {   // make this phase's smem / TMEM writes visible to the tensor core
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    };
 
     for (int ck = 0; ck < nchunks && ok; ++ck) {
         const int t0 = ck * kC;
@@ -362,132 +338,103 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         const bool more = ck + 1 < nchunks;
         // ---- gate prep
         if (!(ok = wait_all(BAR_QKV, ph) && wait_all(BAR_A, ph) && wait_all(BAR_B, ph) && wait_all(BAR_W, ph))) break;
-        prep(c, tid, n);
-        fence_proxy_async_smem();
-        __syncthreads();
-        // ---- Gram: [Etil; Qtil] Ktil^T -> TM_G
+        prep(c, tmem, tid, qd, chh, lane, n);
+        sync_for_mma();
+        // ---- [Etil; Qtil] x [Ktil; S^T]^T -> TM_G (Gram) and TM_X (Etil S, Qtil S)
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t id = idesc_tf32(128, 64, 0, 0);
+            const uint32_t id = idesc_tf32(128, 128, 0, 0);
             for (int kk = 0; kk < 16; ++kk) {
-                const uint64_t a = sdesc_sw128(c.sa + OFF_X1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                const uint64_t b = sdesc_sw128(c.sa + OFF_KT + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                mma_tf32(tmem + TM_G, a, b, id, kk > 0);
+                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_tf32(tmem + TM_G, sdesc_sw128(c.sa + OFF_X1 + koff, 16, 1024),
+                         sdesc_sw128(c.sa + OFF_KS + koff, 16, 1024), id, kk > 0);
             }
             mma_commit(c.bar[BAR_MMA]);
         }
         if (!(ok = mma_wait())) break;
-        {   // A (rows 0-63, strictly lower, FP32 for the solve) and P (rows 64-127, lower, TF32)
-            float v[32];
-            tmem_ld32(tmem + tq_lane + TM_G + 32 * chh, v);
-            const int r = srow;
-            if (r < 64) {
+        if (tid == 0 && more) {     // X1 and the Ktil rows of KS are consumed: next b and alpha
+            load_alpha(c, maps, h, t0 + kC, bidx);
+            load_b(c, maps, h, t0 + kC, bidx);
+        }
+        {
+            float g[32];
+            tmem_ld32(tlane + TM_G + 32 * chh, g);
+            if (srow < 64) {        // A row (strictly lower) and R = Z - Etil S
                 float *As = fptr(c, OFF_AS);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int s = 32 * chh + j;
-                    As[r * LDA + s] = (s < r) ? v[j] : 0.f;
+                    As[srow * LDA + s] = (s < srow) ? g[j] : 0.f;
                 }
-            } else {
-                const int t = r - 64;
+                float x[32];
+                tmem_ld32(tlane + TM_X + 32 * chh, x);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const int s = 32 * chh + j;
-                    st_tf32x4(c.sm + OFF_TP + tp_off(r, s), (s <= t) ? v[j] : 0.f, (s + 1 <= t) ? v[j + 1] : 0.f,
-                              (s + 2 <= t) ? v[j + 2] : 0.f, (s + 3 <= t) ? v[j + 3] : 0.f);
+                for (int j = 0; j < 32; ++j) {
+                    const int col = 32 * chh + j;
+                    const float z = at(c, OFF_ZW + zw_off(srow, col));
+                    at(c, OFF_RU + ru_off(col, srow)) = to_tf32(z - x[j]);
                 }
+            } else {                // P row (lower incl. diagonal) -> A operand in TMEM
+                const int t = srow - 64;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) g[j] = (32 * chh + j <= t) ? to_tf32(g[j]) : 0.f;
+                tmem_st32(tlane + TM_TP + 32 * chh, g);
             }
         }
-        __syncthreads();
+        sync_for_mma();
+        if (tid == 0 && more) load_w(c, maps, h, t0 + kC, bidx, col0);   // Z consumed
         solve(c, tid);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // ---- next chunk's q, k, v may land now; W = T Etil, Y = T Z
+        if (srow < 64) {            // T rows -> A operand in TMEM
+            float tv[32];
+            const float *Ts = fptr(c, OFF_TS);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) tv[j] = to_tf32(Ts[srow * LDA + 32 * chh + j]);
+            tmem_st32(tlane + TM_TP + 32 * chh, tv);
+        }
+        sync_for_mma();
+        // ---- U = [T; P] R (lanes 0-63)
         if (tid == 0) {
-            if (more) load_qkv(c, maps, h, t0 + kC, bidx, col0);
+            if (more) load_qkv(c, maps, h, t0 + kC, bidx, col0);         // staging free again
             tc_fence_after();
-            const uint32_t idw = idesc_tf32(128, 128, 0, 1), idy = idesc_tf32(128, 64, 0, 1);
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t a = sdesc_sw128(c.sa + OFF_TP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                const uint64_t bw = sdesc_sw128(c.sa + OFF_X1 + kk * 1024, 16384, 1024);
-                const uint64_t by = sdesc_sw128(c.sa + OFF_ZU + kk * 1024, 8192, 1024);
-                mma_tf32(tmem + TM_W, a, bw, idw, kk > 0);
-                mma_tf32(tmem + TM_Y, a, by, idy, kk > 0);
-            }
+            const uint32_t id = idesc_tf32(128, 64, 0, 0);
+            for (int kk = 0; kk < 8; ++kk)
+                mma_tf32_ts(tmem + TM_U, tmem + TM_TP + 8 * kk,
+                            sdesc_sw128(c.sa + OFF_RU + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id, kk > 0);
             mma_commit(c.bar[BAR_MMA]);
         }
         if (!(ok = mma_wait())) break;
-        if (qd < 2) {   // W rows (lanes 0-63) -> X1 rows 0-63, channels [64*chh, 64*chh + 64)
-            float v[32];
+        if (srow < 64) {            // U -> RU (transposed)
+            float u[32];
+            tmem_ld32(tlane + TM_U + 32 * chh, u);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int c0 = 64 * chh + 32 * hh;
-                tmem_ld32(tmem + tq_lane + TM_W + c0, v);
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    st_tf32x4(c.sm + OFF_X1 + x1_off(srow, c0 + j), v[j], v[j + 1], v[j + 2], v[j + 3]);
-            }
+            for (int j = 0; j < 32; ++j) at(c, OFF_RU + ru_off(32 * chh + j, srow)) = to_tf32(u[j]);
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // ---- [W; Qtil] S -> TM_X
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_tf32(128, 64, 0, 1);
-            for (int kk = 0; kk < 16; ++kk) {
-                const uint64_t a = sdesc_sw128(c.sa + OFF_X1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                const uint64_t b = sdesc_sw128(c.sa + OFF_ST + kk * 1024, 16384, 1024);
-                mma_tf32(tmem + TM_X, a, b, id, kk > 0);
-            }
-            mma_commit(c.bar[BAR_MMA]);
-        }
-        if (!(ok = mma_wait())) break;
-        if (tid == 0 && more) load_b(c, maps, h, t0 + kC, bidx);   // X1 rows 0-63 are free again
-        if (qd < 2) {   // U = Y - W S (lanes 0-63) -> ZU tile
-            float ws[32], y[32];
-            tmem_ld32(tmem + tq_lane + TM_X + 32 * chh, ws);
-            tmem_ld32(tmem + tq_lane + TM_Y + 32 * chh, y);
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                st_tf32x4(c.sm + OFF_ZU + zu_off(srow, 32 * chh + j), y[j] - ws[j], y[j + 1] - ws[j + 1],
-                          y[j + 2] - ws[j + 2], y[j + 3] - ws[j + 3]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
+        sync_for_mma();
         // ---- Ktil^T U -> TM_D;  [T; P] U accumulated onto TM_X (lanes 64-127 become O)
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t idd = idesc_tf32(128, 64, 1, 1), ido = idesc_tf32(128, 64, 0, 1);
+            const uint32_t id = idesc_tf32(128, 64, 0, 0);
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ak = sdesc_sw128(c.sa + OFF_KT + kk * 1024, 8192, 1024);
-                const uint64_t at = sdesc_sw128(c.sa + OFF_TP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                const uint64_t bu = sdesc_sw128(c.sa + OFF_ZU + kk * 1024, 8192, 1024);
-                mma_tf32(tmem + TM_D, ak, bu, idd, kk > 0);
-                mma_tf32(tmem + TM_X, at, bu, ido, 1);
+                const uint64_t bu = sdesc_sw128(c.sa + OFF_RU + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, bu, id, kk > 0);
+                mma_tf32_ts(tmem + TM_X, tmem + TM_TP + 8 * kk, bu, id, 1);
             }
             mma_commit(c.bar[BAR_MMA]);
         }
         if (!(ok = mma_wait())) break;
-        if (tid == 0 && more) {    // Ktil and Z/U tiles are free: next alpha and w
-            load_alpha(c, maps, h, t0 + kC, bidx);
-            load_w(c, maps, h, t0 + kC, bidx, col0);
-        }
-        {   // state: S <- gamma_n (S + Ktil^T U); operand copy for the next chunk
+        {   // state: S <- gamma_n (S + Ktil^T U); TF32 operand copy for the next chunk
             float d[32];
-            tmem_ld32(tmem + tq_lane + TM_D + 32 * chh, d);
+            tmem_ld32(tlane + TM_D + 32 * chh, d);
             const float gn = fptr(c, OFF_GN)[srow];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) S[j] = gn * (S[j] + d[j]);
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                st_tf32x4(c.sm + OFF_ST + st_off(srow, 32 * chh + j), S[j], S[j + 1], S[j + 2], S[j + 3]);
+            for (int j = 0; j < 32; ++j) {
+                S[j] = gn * (S[j] + d[j]);
+                at(c, OFF_KS + x_off(64 + 32 * chh + j, srow)) = to_tf32(S[j]);
+            }
         }
-        if (qd >= 2) {   // outputs: lanes 64-127 of TM_X
+        if (srow >= 64) {           // outputs from lanes 64-127 of TM_X
             float v[32];
-            tmem_ld32(tmem + tq_lane + TM_X + 32 * chh, v);
+            tmem_ld32(tlane + TM_X + 32 * chh, v);
             const int t = srow - 64;
             if (t < n) {
                 __nv_bfloat16 *dst = o + (((size_t)bidx * T + t0 + t) * H + h) * 128 + col0 + 32 * chh;
@@ -506,9 +453,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                 }
             }
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
+        sync_for_mma();
     }
 
     if (ok && S_T) {
@@ -518,7 +463,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             *reinterpret_cast<float4 *>(S_T + off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
     if (!ok && tid == 0) {
-        // Drain any copies still in flight (bounded) before the CTA releases its shared memory.
+        // Drain copies still in flight (bounded) before the CTA releases its shared memory.
         for (int i = 0; i < NBARS; ++i) (void)mbar_wait(c.bar[i], 0, kWaitLimit / 8);
     }
     tc_fence_before();
