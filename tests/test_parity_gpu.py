@@ -43,11 +43,13 @@ def half_ulp_bf16(a):
     return np.where(a > 0, np.exp2(e - 8.0), 0.0)
 
 
-def rel_bf16(x, ref):
-    """max(|x - ref| - half BF16 ulp, 0) / RMS(ref): error beyond the output's own rounding."""
+def rel_bf16(x, ref, roundings=1):
+    """max(|x - ref| - half BF16 ulp, 0) / RMS(ref): error beyond the output's own rounding.
+
+    ``roundings=2`` when both sides are BF16 results (each carries its own rounding)."""
     x = np.asarray(x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
-    slack = half_ulp_bf16(np.maximum(np.abs(ref), np.abs(x)))
+    slack = roundings * half_ulp_bf16(np.maximum(np.abs(ref), np.abs(x)))
     excess = np.maximum(np.abs(x - ref) - slack, 0.0)
     return float(np.max(excess) / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
 
@@ -251,7 +253,8 @@ def test_long_ragged_split_chaining(g, long_ragged):
     ob, Sb = g.gdn2_chunk_fwd(*(parts[1][n] for n in ("q", "k", "v", "alpha", "b", "w")), Sa)
     torch.cuda.synchronize()
     o_split = torch.cat([oa, ob], 1).float().cpu().numpy()
-    assert rel_bf16(o_split, o_full.float().cpu().numpy()) <= TOL_BF16_O
+    # both are BF16 results with different chunk boundaries: allow each its own rounding
+    assert rel_bf16(o_split, o_full.float().cpu().numpy(), roundings=2) <= TOL_BF16_O
     assert rel(Sb.cpu().numpy(), S_full.cpu().numpy()) <= TOL_BF16_S
     check_sampled(x, o_split, Sb.cpu().numpy(), [(0, 5)], TOL_BF16_S)
 
