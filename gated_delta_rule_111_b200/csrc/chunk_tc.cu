@@ -16,6 +16,12 @@
 //   O = Qtil S + P U                                             (tensor core, accumulated)
 //   S <- diag(gamma_n) (S + Ktil^T U)                            (tensor core + FP32 epilogue)
 //
+// The state path (R, U and Ktil in the state update) is computed with split
+// TF32 operands: x = x_hi + x_lo, both TF32, and
+//   T R = T R_hi + T R_lo,   Ktil^T U = Ktil_hi^T U_hi + Ktil_hi^T U_lo + Ktil_lo^T U_hi,
+// which carries about 21 bits of each operand.  With plain TF32 there the
+// carried state drifts by ~0.7% of its RMS over 16K tokens; split, ~0.03%.
+//
 // U holds the per-token corrections z_t - r_t of the token recurrence, so this
 // is the same arithmetic as the token loop, re-associated.
 //
@@ -58,13 +64,15 @@ constexpr long long kWaitLimit = 4000000000ll;   // ~2 s of SM cycles per wait
 // 32 elements per 128-byte swizzled row, K-major:
 //   X1  rows 0-63 Etil[t][i], rows 64-127 Qtil[t][i]     4 atoms x 16 KB (i = key channel)
 //   KS  rows 0-63 Ktil[s][i], rows 64-127 S[i][j] as [j][i]   4 atoms x 16 KB
-//   RU  R, later U, as [j][t]                             2 atoms x 8 KB (t = token)
+//   RU  R_hi, later U_hi, as [j][t]                       2 atoms x 8 KB (t = token)
+//   RL  R_lo, later U_lo, as [j][t]                       2 atoms x 8 KB
 //   ZW  w, then Z = w*v, as [t][j] (FP32, epilogue only)   2 atoms x 8 KB
 // and unswizzled BF16 staging of q, k (64 x 128) and v (64 x 64).
 constexpr uint32_t OFF_X1 = 0;
 constexpr uint32_t OFF_KS = OFF_X1 + 65536;
 constexpr uint32_t OFF_RU = OFF_KS + 65536;
-constexpr uint32_t OFF_ZW = OFF_RU + 16384;
+constexpr uint32_t OFF_RL = OFF_RU + 16384;
+constexpr uint32_t OFF_ZW = OFF_RL + 16384;
 constexpr uint32_t OFF_RQ = OFF_ZW + 16384;
 constexpr uint32_t OFF_RK = OFF_RQ + 16384;
 constexpr uint32_t OFF_RV = OFF_RK + 16384;
@@ -88,6 +96,7 @@ constexpr uint32_t TM_U = 128;    // [T;P] R : lanes 0-63 U                     
 constexpr uint32_t TM_D = 192;    // Ktil^T U                                             (64 cols)
 constexpr uint32_t TM_KT = 256;   // A operand Ktil^T: lane i, column s                   (64 cols)
 constexpr uint32_t TM_TP = 320;   // A operand [T;P]: lane t (P at 64+t), column s        (64 cols)
+constexpr uint32_t TM_KL = 384;   // A operand Ktil_lo^T (low TF32 part of Ktil^T)        (64 cols)
 constexpr uint32_t TM_COLS = 512;
 
 enum { BAR_QKV = 0, BAR_A, BAR_B, BAR_W, BAR_MMA, NBARS };
@@ -154,7 +163,7 @@ __device__ __forceinline__ void prep(const Ctx &c, uint32_t tmem, int tid, int q
     if (th == 0) fptr(c, OFF_GN)[i] = p0 * p1;
     float g = th ? p0 : 1.f;
     float r = 1.f / g;
-    float kt[32];
+    float kt[32], kl[32];
 #pragma unroll
     for (int tt = 0; tt < 32; ++tt) {
         const int t = 32 * th + tt;
@@ -167,10 +176,13 @@ __device__ __forceinline__ void prep(const Ctx &c, uint32_t tmem, int tid, int q
         const float bb = at(c, OFF_X1 + o);
         at(c, OFF_X1 + o) = to_tf32(bb * kk * g);
         at(c, OFF_X1 + x_off(64 + t, i)) = to_tf32(qq * g);
-        kt[tt] = to_tf32(kk * r);
+        const float kf = kk * r;
+        kt[tt] = to_tf32(kf);
+        kl[tt] = to_tf32(kf - kt[tt]);
         at(c, OFF_KS + o) = kt[tt];
     }
     tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + TM_KT + 32 * th, kt);
+    tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + TM_KL + 32 * th, kl);
     // Z = w * v in place over w (FP32; used only by the R epilogue).
     const int j2 = tid & 31, tg = tid >> 5;
     for (int m = 0; m < 8; ++m) {
@@ -371,8 +383,10 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int col = 32 * chh + j;
-                    const float z = at(c, OFF_ZW + zw_off(srow, col));
-                    at(c, OFF_RU + ru_off(col, srow)) = to_tf32(z - x[j]);
+                    const float rr = at(c, OFF_ZW + zw_off(srow, col)) - x[j];
+                    const float hi = to_tf32(rr);
+                    at(c, OFF_RU + ru_off(col, srow)) = hi;
+                    at(c, OFF_RL + ru_off(col, srow)) = to_tf32(rr - hi);
                 }
             } else {                // P row (lower incl. diagonal) -> A operand in TMEM
                 const int t = srow - 64;
@@ -397,9 +411,11 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             if (more) load_qkv(c, maps, h, t0 + kC, bidx, col0);         // staging free again
             tc_fence_after();
             const uint32_t id = idesc_tf32(128, 64, 0, 0);
-            for (int kk = 0; kk < 8; ++kk)
-                mma_tf32_ts(tmem + TM_U, tmem + TM_TP + 8 * kk,
-                            sdesc_sw128(c.sa + OFF_RU + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
+                mma_tf32_ts(tmem + TM_U, tmem + TM_TP + 8 * kk, sdesc_sw128(c.sa + OFF_RU + koff, 16, 1024), id, kk > 0);
+                mma_tf32_ts(tmem + TM_U, tmem + TM_TP + 8 * kk, sdesc_sw128(c.sa + OFF_RL + koff, 16, 1024), id, 1);
+            }
             mma_commit(c.bar[BAR_MMA]);
         }
         if (!(ok = mma_wait())) break;
@@ -407,7 +423,11 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             float u[32];
             tmem_ld32(tlane + TM_U + 32 * chh, u);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) at(c, OFF_RU + ru_off(32 * chh + j, srow)) = to_tf32(u[j]);
+            for (int j = 0; j < 32; ++j) {
+                const float hi = to_tf32(u[j]);
+                at(c, OFF_RU + ru_off(32 * chh + j, srow)) = hi;
+                at(c, OFF_RL + ru_off(32 * chh + j, srow)) = to_tf32(u[j] - hi);
+            }
         }
         sync_for_mma();
         // ---- Ktil^T U -> TM_D;  [T; P] U accumulated onto TM_X (lanes 64-127 become O)
@@ -415,9 +435,17 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             tc_fence_after();
             const uint32_t id = idesc_tf32(128, 64, 0, 0);
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t bu = sdesc_sw128(c.sa + OFF_RU + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, bu, id, kk > 0);
-                mma_tf32_ts(tmem + TM_X, tmem + TM_TP + 8 * kk, bu, id, 1);
+                const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
+                const uint64_t uh = sdesc_sw128(c.sa + OFF_RU + koff, 16, 1024);
+                const uint64_t ul = sdesc_sw128(c.sa + OFF_RL + koff, 16, 1024);
+                mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, uh, id, kk > 0);
+                mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, ul, id, 1);
+                mma_tf32_ts(tmem + TM_D, tmem + TM_KL + 8 * kk, uh, id, 1);
+            }
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
+                mma_tf32_ts(tmem + TM_X, tmem + TM_TP + 8 * kk, sdesc_sw128(c.sa + OFF_RU + koff, 16, 1024), id, 1);
+                mma_tf32_ts(tmem + TM_X, tmem + TM_TP + 8 * kk, sdesc_sw128(c.sa + OFF_RL + koff, 16, 1024), id, 1);
             }
             mma_commit(c.bar[BAR_MMA]);
         }
