@@ -8,38 +8,34 @@
 // decay and state/solve precision.  Per chunk of n tokens from state S:
 //
 //   gamma_t = prod_{j<=t} alpha_j,  rho_t = 1/gamma_t          (per key channel, FP32)
-//   Etil = b*k*gamma,  Qtil = q*gamma,  Ktil = k*rho,  Z = w*v   (gate prep)
+//   Etil = b*k*gamma,  Qtil = q*gamma,  Ktil = k*rho            (gate prep)
 //   [A | Etil S] and [P | Qtil S] = [Etil; Qtil] [Ktil; S^T]^T  (one tensor-core product)
-//   A <- strict_tril(A),  P <- tril(P),  T = (I + A)^{-1}        (FP32 blocked solve)
-//   R = Z - Etil S                                               (FP32 epilogue)
-//   U = T R                                                      (tensor core)
-//   O = Qtil S + P U                                             (tensor core, accumulated)
+//   R = w*v - Etil S                                             (FP32 epilogue)
+//   (I + strict_tril(A)) U = R                                   (FP32 blocked forward substitution)
+//   O = Qtil S + tril(P) U                                       (tensor core, accumulated)
 //   S <- diag(gamma_n) (S + Ktil^T U)                            (tensor core + FP32 epilogue)
 //
-// The state path (R, U and Ktil in the state update) is computed with split
-// TF32 operands: x = x_hi + x_lo, both TF32, and
-//   T R = T R_hi + T R_lo,   Ktil^T U = Ktil_hi^T U_hi + Ktil_hi^T U_lo + Ktil_lo^T U_hi,
-// which carries about 21 bits of each operand.  With plain TF32 there the
-// carried state drifts by ~0.7% of its RMS over 16K tokens; split, ~0.03%.
-//
 // U holds the per-token corrections z_t - r_t of the token recurrence, so this
-// is the same arithmetic as the token loop, re-associated.
+// is the token loop's arithmetic, re-associated.
 //
-// Precision: tensor-core operands are rounded to TF32 (10-bit mantissa);
-// accumulation, decay, solve, R and the carried state are FP32.  BF16 operands
-// lose too much here: the read r = Sbar^T e nearly cancels the write z in the
-// delta rule, and products of decay-scaled factors carry that error into o and
-// S.  The key factor Ktil = k / gamma grows within a chunk as
-// exp(-sum ln alpha); it must stay below ~1e34 (sum of -ln alpha over one chunk
-// <= 78 per key channel), as documented in gdn2.h.
+// Precision: tensor-core operands are TF32 (10-bit mantissa); accumulation,
+// decay, R, the solve and the carried state are FP32.  The state update uses
+// split operands, x = x_hi + x_lo with both parts TF32:
+//   Ktil^T U = Ktil_hi^T U_hi + Ktil_hi^T U_lo + Ktil_lo^T U_hi,
+// which carries about 21 bits of each operand (plain TF32 there lets the state
+// drift by ~0.7% of its RMS over 16K tokens; split, ~0.03%).  BF16 operands lose
+// too much: the read r = Sbar^T e nearly cancels the write z in the delta rule.
+// The key factor Ktil = k / gamma grows within a chunk as exp(-sum ln alpha); it
+// must stay below ~1e34 (sum of -ln alpha over one chunk <= 78 per key channel),
+// as documented in gdn2.h.
 //
 // Layout: one CTA per (batch, head, 64-column half of d_v); 256 threads (8
 // warps) run the phases of a chunk in turn; thread 0 issues TMA loads and MMAs.
-// Every shared-memory operand is K-major with the 128-byte swizzle.  Operands
-// needed transposed (Ktil^T, [T; P]) are written to Tensor Memory and read from
-// there as the A operand.  alpha, b and w are TMA-loaded straight into the
-// tiles they become and transformed in place; the next chunk's loads are
-// issued as soon as each tile is consumed.
+// Every shared-memory MMA operand is K-major with the 128-byte swizzle.  The
+// operands needed transposed (Ktil^T, P) are written to Tensor Memory and read
+// from there as the A operand.  alpha, b and w are TMA-loaded straight into the
+// tiles they become and transformed in place; each next-chunk load is issued as
+// soon as its tile is consumed.
 #include <cudaTypedefs.h>
 #include <stdio.h>
 
@@ -60,19 +56,19 @@ constexpr int kDVS = 64;          // value columns per CTA
 constexpr int kThreads = 256;
 constexpr long long kWaitLimit = 4000000000ll;   // ~2 s of SM cycles per wait
 
-// Shared-memory map (bytes from a 1024-aligned base).  Tiles hold FP32/TF32,
+// Shared-memory map (bytes from a 1024-aligned base).  MMA tiles hold TF32,
 // 32 elements per 128-byte swizzled row, K-major:
-//   X1  rows 0-63 Etil[t][i], rows 64-127 Qtil[t][i]     4 atoms x 16 KB (i = key channel)
-//   KS  rows 0-63 Ktil[s][i], rows 64-127 S[i][j] as [j][i]   4 atoms x 16 KB
-//   RU  R_hi, later U_hi, as [j][t]                       2 atoms x 8 KB (t = token)
-//   RL  R_lo, later U_lo, as [j][t]                       2 atoms x 8 KB
-//   ZW  w, then Z = w*v, as [t][j] (FP32, epilogue only)   2 atoms x 8 KB
+//   X1  rows 0-63 Etil[t][i], rows 64-127 Qtil[t][i]         4 atoms x 16 KB (i = key channel)
+//   KS  rows 0-63 Ktil_hi[s][i], rows 64-127 S[i][j] as [j][i]  4 atoms x 16 KB
+//   UH  U_hi as [j][t]                                        2 atoms x 8 KB (t = token)
+//   UL  U_lo as [j][t]                                        2 atoms x 8 KB
+//   ZW  w, then R, then U, as [t][j] (FP32, same swizzle)     2 atoms x 8 KB
 // and unswizzled BF16 staging of q, k (64 x 128) and v (64 x 64).
 constexpr uint32_t OFF_X1 = 0;
 constexpr uint32_t OFF_KS = OFF_X1 + 65536;
-constexpr uint32_t OFF_RU = OFF_KS + 65536;
-constexpr uint32_t OFF_RL = OFF_RU + 16384;
-constexpr uint32_t OFF_ZW = OFF_RL + 16384;
+constexpr uint32_t OFF_UH = OFF_KS + 65536;
+constexpr uint32_t OFF_UL = OFF_UH + 16384;
+constexpr uint32_t OFF_ZW = OFF_UL + 16384;
 constexpr uint32_t OFF_RQ = OFF_ZW + 16384;
 constexpr uint32_t OFF_RK = OFF_RQ + 16384;
 constexpr uint32_t OFF_RV = OFF_RK + 16384;
@@ -82,21 +78,19 @@ constexpr uint32_t OFF_BAR = OFF_PART + 1024;   // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 64;     // tmem base, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // + alignment slack
-// Solve scratch inside the q/k/v staging (free between prep and the next load).
-constexpr int LDA = 65, LDX = 33;
-constexpr uint32_t OFF_AS = OFF_RQ;                     // float[64][65] A, strictly lower
-constexpr uint32_t OFF_TS = OFF_AS + 16896;             // float[64][65] T
-constexpr uint32_t OFF_XS = OFF_TS + 16896;             // float[32][33] block products
-static_assert(OFF_XS + 32 * LDX * 4 <= OFF_GN, "solve scratch overflows the staging area");
+// Solve scratch inside the q/k staging (free between prep and the next load).
+constexpr int LDA = 65, LDD = 17;
+constexpr uint32_t OFF_AS = OFF_RQ;             // float[64][65]    A, strictly lower
+constexpr uint32_t OFF_DS = OFF_AS + 16896;     // float[4][16][17] inverses of the diagonal blocks
+static_assert(OFF_DS + 4 * 16 * LDD * 4 <= OFF_RV, "solve scratch overlaps the v staging");
 
 // Tensor Memory columns (512 allocated).
 constexpr uint32_t TM_G = 0;      // [Etil;Qtil] Ktil^T : lanes 0-63 A, lanes 64-127 P   (64 cols)
-constexpr uint32_t TM_X = 64;     // [Etil;Qtil] S, then + [T;P] U : lanes 64-127 -> O    (64 cols)
-constexpr uint32_t TM_U = 128;    // [T;P] R : lanes 0-63 U                               (64 cols)
-constexpr uint32_t TM_D = 192;    // Ktil^T U                                             (64 cols)
-constexpr uint32_t TM_KT = 256;   // A operand Ktil^T: lane i, column s                   (64 cols)
-constexpr uint32_t TM_TP = 320;   // A operand [T;P]: lane t (P at 64+t), column s        (64 cols)
-constexpr uint32_t TM_KL = 384;   // A operand Ktil_lo^T (low TF32 part of Ktil^T)        (64 cols)
+constexpr uint32_t TM_X = 64;     // [Etil;Qtil] S, then + P U : lanes 64-127 -> O        (64 cols)
+constexpr uint32_t TM_D = 128;    // Ktil^T U                                             (64 cols)
+constexpr uint32_t TM_KT = 192;   // A operand Ktil_hi^T: lane i, column s                (64 cols)
+constexpr uint32_t TM_KL = 256;   // A operand Ktil_lo^T                                  (64 cols)
+constexpr uint32_t TM_P = 320;    // A operand: lanes 64-127 tril(P), lanes 0-63 zero     (64 cols)
 constexpr uint32_t TM_COLS = 512;
 
 enum { BAR_QKV = 0, BAR_A, BAR_B, BAR_W, BAR_MMA, NBARS };
@@ -108,7 +102,7 @@ constexpr uint32_t TX_W = 2 * 8192;
 
 // Element byte offsets inside the tiles.
 __device__ __forceinline__ uint32_t x_off(uint32_t r, uint32_t i) { return (i >> 5) * 16384u + swz128(r, (i & 31u) * 4u); }
-__device__ __forceinline__ uint32_t ru_off(uint32_t j, uint32_t t) { return (t >> 5) * 8192u + swz128(j, (t & 31u) * 4u); }
+__device__ __forceinline__ uint32_t u_off(uint32_t j, uint32_t t) { return (t >> 5) * 8192u + swz128(j, (t & 31u) * 4u); }
 __device__ __forceinline__ uint32_t zw_off(uint32_t t, uint32_t j) { return (j >> 5) * 8192u + swz128(t, (j & 31u) * 4u); }
 
 struct Maps {
@@ -123,6 +117,7 @@ struct Ctx {
 
 __device__ __forceinline__ float *fptr(const Ctx &c, uint32_t off) { return reinterpret_cast<float *>(c.sm + off); }
 __device__ __forceinline__ float &at(const Ctx &c, uint32_t off) { return *reinterpret_cast<float *>(c.sm + off); }
+__device__ __forceinline__ float4 &at4(const Ctx &c, uint32_t off) { return *reinterpret_cast<float4 *>(c.sm + off); }
 
 // TMA loads of one chunk's inputs (thread 0 only).
 __device__ __forceinline__ void load_qkv(const Ctx &c, const Maps &m, int h, int t0, int bidx, int col0) {
@@ -150,61 +145,82 @@ __device__ __forceinline__ float ldbf(const uint8_t *p) { return __bfloat162floa
 // Gate prep.  Thread (lane quarter qd, half th, lane l) owns key channel
 // i = 32 qd + l for tokens [32 th, 32 th + 32).  Cumulative decay is a running
 // FP32 product (exp of the cumulative log-decay up to rounding).  Padding tokens
-// (t >= n) have zero q, k, b, w, v from the TMA bounds fill and alpha forced to 1.
-__device__ __forceinline__ void prep(const Ctx &c, uint32_t tmem, int tid, int qd, int th, int lane, int n) {
+// (t >= n) have zero q, k, b from the TMA bounds fill and alpha forced to 1.
+// Tokens go in groups of 8; a group's loads are issued before the previous
+// group's stores so the in-place writes never stall the reads.
+__device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, int qd, int th, int lane, int n) {
     const int i = 32 * qd + lane;
     float *part = fptr(c, OFF_PART);
+    const uint32_t ci = (i >> 5) * 16384u;       // atom of channel i
+    const uint32_t cb = (i & 31) * 4u;           // byte in row
     float pa = 1.f;
-    for (int t = 32 * th; t < 32 * th + 32; ++t)
-        if (t < n) pa *= clamp_alpha(at(c, OFF_KS + x_off(t, i)));
+#pragma unroll
+    for (int tt = 0; tt < 32; ++tt) {
+        const int t = 32 * th + tt;
+        const float a = at(c, OFF_KS + ci + swz128(t, cb));
+        pa *= (t < n) ? clamp_alpha(a) : 1.f;
+    }
     part[th * 128 + i] = pa;
     __syncthreads();
     const float p0 = part[i], p1 = part[128 + i];
     if (th == 0) fptr(c, OFF_GN)[i] = p0 * p1;
     float g = th ? p0 : 1.f;
     float r = 1.f / g;
-    float kt[32], kl[32];
+    float av[8], kv[8], qv[8], bv[8];
+    auto load_group = [&](int g8) {
 #pragma unroll
-    for (int tt = 0; tt < 32; ++tt) {
-        const int t = 32 * th + tt;
-        const uint32_t o = x_off(t, i);
-        float a = (t < n) ? clamp_alpha(at(c, OFF_KS + o)) : 1.f;
-        g *= a;
-        r *= __fdividef(1.f, a);
-        const float kk = ldbf(c.sm + OFF_RK + t * 256 + i * 2);
-        const float qq = ldbf(c.sm + OFF_RQ + t * 256 + i * 2);
-        const float bb = at(c, OFF_X1 + o);
-        at(c, OFF_X1 + o) = to_tf32(bb * kk * g);
-        at(c, OFF_X1 + x_off(64 + t, i)) = to_tf32(qq * g);
-        const float kf = kk * r;
-        kt[tt] = to_tf32(kf);
-        kl[tt] = to_tf32(kf - kt[tt]);
-        at(c, OFF_KS + o) = kt[tt];
-    }
-    tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + TM_KT + 32 * th, kt);
-    tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + TM_KL + 32 * th, kl);
-    // Z = w * v in place over w (FP32; used only by the R epilogue).
-    const int j2 = tid & 31, tg = tid >> 5;
-    for (int m = 0; m < 8; ++m) {
-        const int t = tg + 8 * m;
-        float2 *pz = reinterpret_cast<float2 *>(c.sm + OFF_ZW + zw_off(t, 2 * j2));
-        const float2 w = *pz;
-        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(c.sm + OFF_RV + t * 128 + j2 * 4);
-        const float2 vf = __bfloat1622float2(v);
-        *pz = make_float2(w.x * vf.x, w.y * vf.y);
+        for (int u = 0; u < 8; ++u) {
+            const int t = 32 * th + 8 * g8 + u;
+            av[u] = at(c, OFF_KS + ci + swz128(t, cb));
+            bv[u] = at(c, OFF_X1 + ci + swz128(t, cb));
+            kv[u] = ldbf(c.sm + OFF_RK + t * 256 + i * 2);
+            qv[u] = ldbf(c.sm + OFF_RQ + t * 256 + i * 2);
+        }
+    };
+    load_group(0);
+#pragma unroll
+    for (int g8 = 0; g8 < 4; ++g8) {
+        float e[8], qt[8], kh[8], kl[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int t = 32 * th + 8 * g8 + u;
+            const float a = (t < n) ? clamp_alpha(av[u]) : 1.f;
+            g *= a;
+            r *= __fdividef(1.f, a);
+            e[u] = to_tf32(bv[u] * kv[u] * g);
+            qt[u] = to_tf32(qv[u] * g);
+            const float kf = kv[u] * r;
+            kh[u] = to_tf32(kf);
+            kl[u] = to_tf32(kf - kh[u]);
+        }
+        if (g8 < 3) load_group(g8 + 1);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int t = 32 * th + 8 * g8 + u;
+            at(c, OFF_X1 + ci + swz128(t, cb)) = e[u];
+            at(c, OFF_X1 + ci + swz128(64 + t, cb)) = qt[u];
+            at(c, OFF_KS + ci + swz128(t, cb)) = kh[u];
+        }
+        tmem_st8(tlane + TM_KT + 32 * th + 8 * g8, kh);
+        tmem_st8(tlane + TM_KL + 32 * th + 8 * g8, kl);
     }
 }
 
 // ---------------------------------------------------------------------------
-// T = (I + A)^{-1}, A strictly lower 64 x 64 (FP32, As), result in Ts (FP32,
-// zero above the diagonal).  16 x 16 diagonal blocks by forward substitution,
-// then T_ab = -T_aa (sum_c A_ac T_cb) for the 16- and 32-wide off-diagonal blocks.
-__device__ __forceinline__ void solve(const Ctx &c, int tid) {
+// Solve (I + A) U = R in FP32, A strictly lower 64 x 64 (As), R and U in the ZW
+// tile ([t][j], 64 value columns).  The inverses D_b of the four 16 x 16
+// diagonal blocks come first (forward substitution, one thread per column);
+// then, block by block, R'_b = R_b - sum_{c<b} A_bc U_c and U_b = D_b R'_b.
+// Thread (i, cg) owns row 16 b + i, columns 4 cg .. 4 cg + 3 of each block.
+__device__ __forceinline__ void fma4(float4 &acc, float a, const float4 &x) {
+    acc.x = fmaf(a, x.x, acc.x); acc.y = fmaf(a, x.y, acc.y); acc.z = fmaf(a, x.z, acc.z); acc.w = fmaf(a, x.w, acc.w);
+}
+
+__device__ __forceinline__ void solve_u(const Ctx &c, int tid) {
     const float *As = fptr(c, OFF_AS);
-    float *Ts = fptr(c, OFF_TS);
-    float *Xs = fptr(c, OFF_XS);
+    float *Ds = fptr(c, OFF_DS);
     if (tid < 64) {
-        const int a = tid >> 4, j = tid & 15, base = 16 * a;
+        const int b = tid >> 4, j = tid & 15, base = 16 * b;
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -214,53 +230,27 @@ __device__ __forceinline__ void solve(const Ctx &c, int tid) {
             x[i] = acc;
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) Ts[(base + i) * LDA + base + j] = x[i];
-    } else {
-        // zero the blocks above the diagonal: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-        for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
-            const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
-            const int a = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-            const int b = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            Ts[(16 * a + i) * LDA + 16 * b + j] = 0.f;
-        }
+        for (int i = 0; i < 16; ++i) Ds[(b * 16 + i) * LDD + j] = x[i];
     }
     __syncthreads();
-    // T_10 = -T_11 A_10 T_00 and T_32 = -T_33 A_32 T_22
-    for (int e = tid; e < 512; e += kThreads) {
-        const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
-        const int a = blk ? 3 : 1, b = a - 1;
-        float acc = 0.f;
+    const int i = tid >> 4, cg = tid & 15;
 #pragma unroll
-        for (int l = 0; l < 16; ++l) acc = fmaf(As[(16 * a + i) * LDA + 16 * b + l], Ts[(16 * b + l) * LDA + 16 * b + j], acc);
-        Xs[blk * 16 * LDX + i * LDX + j] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < 512; e += kThreads) {
-        const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
-        const int a = blk ? 3 : 1, b = a - 1;
-        float acc = 0.f;
+    for (int b = 0; b < 4; ++b) {
+        const int row = 16 * b + i;
+        const uint32_t my = OFF_ZW + zw_off(row, 4 * cg);
+        float4 acc = at4(c, my);
 #pragma unroll
-        for (int l = 0; l < 16; ++l) acc = fmaf(Ts[(16 * a + i) * LDA + 16 * a + l], Xs[blk * 16 * LDX + l * LDX + j], acc);
-        Ts[(16 * a + i) * LDA + 16 * b + j] = -acc;
+        for (int l = 0; l < 16 * b; ++l) fma4(acc, -As[row * LDA + l], at4(c, OFF_ZW + zw_off(l, 4 * cg)));
+        at4(c, my) = acc;
+        __syncthreads();
+        float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+            if (m <= i) fma4(u, Ds[(b * 16 + i) * LDD + m], at4(c, OFF_ZW + zw_off(16 * b + m, 4 * cg)));
+        __syncthreads();
+        at4(c, my) = u;
+        __syncthreads();
     }
-    __syncthreads();
-    // lower-left 32 x 32 block: T_BA = -T_BB A_BA T_AA
-    for (int e = tid; e < 1024; e += kThreads) {
-        const int i = e >> 5, j = e & 31;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) acc = fmaf(As[(32 + i) * LDA + l], Ts[l * LDA + j], acc);
-        Xs[i * LDX + j] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < 1024; e += kThreads) {
-        const int i = e >> 5, j = e & 31;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) acc = fmaf(Ts[(32 + i) * LDA + 32 + l], Xs[l * LDX + j], acc);
-        Ts[(32 + i) * LDA + j] = -acc;
-    }
-    __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -304,6 +294,12 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         load_alpha(c, maps, h, 0, bidx);
         load_b(c, maps, h, 0, bidx);
         load_w(c, maps, h, 0, bidx, col0);
+    }
+    if (srow < 64) {   // rows 0-63 of the P operand stay zero
+        float z[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z[j] = 0.f;
+        tmem_st32(tlane + TM_P + 32 * chh, z);
     }
 
     // State slice owned by this thread: key channel i = srow, value columns
@@ -349,8 +345,8 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         const uint32_t ph = ck & 1;
         const bool more = ck + 1 < nchunks;
         // ---- gate prep
-        if (!(ok = wait_all(BAR_QKV, ph) && wait_all(BAR_A, ph) && wait_all(BAR_B, ph) && wait_all(BAR_W, ph))) break;
-        prep(c, tmem, tid, qd, chh, lane, n);
+        if (!(ok = wait_all(BAR_QKV, ph) && wait_all(BAR_A, ph) && wait_all(BAR_B, ph))) break;
+        prep(c, tlane, qd, chh, lane, n);
         sync_for_mma();
         // ---- [Etil; Qtil] x [Ktil; S^T]^T -> TM_G (Gram) and TM_X (Etil S, Qtil S)
         if (tid == 0) {
@@ -363,7 +359,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             }
             mma_commit(c.bar[BAR_MMA]);
         }
-        if (!(ok = mma_wait())) break;
+        if (!(ok = mma_wait() && wait_all(BAR_W, ph))) break;
         if (tid == 0 && more) {     // X1 and the Ktil rows of KS are consumed: next b and alpha
             load_alpha(c, maps, h, t0 + kC, bidx);
             load_b(c, maps, h, t0 + kC, bidx);
@@ -371,7 +367,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         {
             float g[32];
             tmem_ld32(tlane + TM_G + 32 * chh, g);
-            if (srow < 64) {        // A row (strictly lower) and R = Z - Etil S
+            if (srow < 64) {        // A row (strictly lower) and R = w*v - Etil S, in place over w
                 float *As = fptr(c, OFF_AS);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
@@ -381,71 +377,58 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                 float x[32];
                 tmem_ld32(tlane + TM_X + 32 * chh, x);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
+                for (int j = 0; j < 32; j += 4) {
                     const int col = 32 * chh + j;
-                    const float rr = at(c, OFF_ZW + zw_off(srow, col)) - x[j];
-                    const float hi = to_tf32(rr);
-                    at(c, OFF_RU + ru_off(col, srow)) = hi;
-                    at(c, OFF_RL + ru_off(col, srow)) = to_tf32(rr - hi);
+                    float4 &wr = at4(c, OFF_ZW + zw_off(srow, col));
+                    const float4 w = wr;
+                    const uint2 vb = *reinterpret_cast<const uint2 *>(c.sm + OFF_RV + srow * 128 + col * 2);
+                    const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.x));
+                    const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.y));
+                    wr = make_float4(w.x * v01.x - x[j], w.y * v01.y - x[j + 1], w.z * v23.x - x[j + 2],
+                                     w.w * v23.y - x[j + 3]);
                 }
             } else {                // P row (lower incl. diagonal) -> A operand in TMEM
                 const int t = srow - 64;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) g[j] = (32 * chh + j <= t) ? to_tf32(g[j]) : 0.f;
-                tmem_st32(tlane + TM_TP + 32 * chh, g);
+                tmem_st32(tlane + TM_P + 32 * chh, g);
+            }
+        }
+        __syncthreads();
+        solve_u(c, tid);
+        // U (FP32, ZW) -> U_hi, U_lo tiles as [j][t]
+        {
+            const int t = srow >> 1;                       // token row; two threads per row
+            const int j0 = 32 * (srow & 1) + 16 * chh;     // 16 columns each
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                const float4 u = at4(c, OFF_ZW + zw_off(t, j0 + j));
+                const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float hi = to_tf32(uu[e]);
+                    at(c, OFF_UH + u_off(j0 + j + e, t)) = hi;
+                    at(c, OFF_UL + u_off(j0 + j + e, t)) = to_tf32(uu[e] - hi);
+                }
             }
         }
         sync_for_mma();
-        if (tid == 0 && more) load_w(c, maps, h, t0 + kC, bidx, col0);   // Z consumed
-        solve(c, tid);
-        if (srow < 64) {            // T rows -> A operand in TMEM
-            float tv[32];
-            const float *Ts = fptr(c, OFF_TS);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) tv[j] = to_tf32(Ts[srow * LDA + 32 * chh + j]);
-            tmem_st32(tlane + TM_TP + 32 * chh, tv);
-        }
-        sync_for_mma();
-        // ---- U = [T; P] R (lanes 0-63)
+        // ---- Ktil^T U -> TM_D (split);  P U_hi accumulated onto TM_X (lanes 64-127 become O)
         if (tid == 0) {
-            if (more) load_qkv(c, maps, h, t0 + kC, bidx, col0);         // staging free again
+            if (more) {                  // solve scratch and ZW consumed: next q, k, v and w
+                load_qkv(c, maps, h, t0 + kC, bidx, col0);
+                load_w(c, maps, h, t0 + kC, bidx, col0);
+            }
             tc_fence_after();
             const uint32_t id = idesc_tf32(128, 64, 0, 0);
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-                mma_tf32_ts(tmem + TM_U, tmem + TM_TP + 8 * kk, sdesc_sw128(c.sa + OFF_RU + koff, 16, 1024), id, kk > 0);
-                mma_tf32_ts(tmem + TM_U, tmem + TM_TP + 8 * kk, sdesc_sw128(c.sa + OFF_RL + koff, 16, 1024), id, 1);
-            }
-            mma_commit(c.bar[BAR_MMA]);
-        }
-        if (!(ok = mma_wait())) break;
-        if (srow < 64) {            // U -> RU (transposed)
-            float u[32];
-            tmem_ld32(tlane + TM_U + 32 * chh, u);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float hi = to_tf32(u[j]);
-                at(c, OFF_RU + ru_off(32 * chh + j, srow)) = hi;
-                at(c, OFF_RL + ru_off(32 * chh + j, srow)) = to_tf32(u[j] - hi);
-            }
-        }
-        sync_for_mma();
-        // ---- Ktil^T U -> TM_D;  [T; P] U accumulated onto TM_X (lanes 64-127 become O)
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_tf32(128, 64, 0, 0);
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-                const uint64_t uh = sdesc_sw128(c.sa + OFF_RU + koff, 16, 1024);
-                const uint64_t ul = sdesc_sw128(c.sa + OFF_RL + koff, 16, 1024);
+                const uint64_t uh = sdesc_sw128(c.sa + OFF_UH + koff, 16, 1024);
+                const uint64_t ul = sdesc_sw128(c.sa + OFF_UL + koff, 16, 1024);
                 mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, uh, id, kk > 0);
                 mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, ul, id, 1);
                 mma_tf32_ts(tmem + TM_D, tmem + TM_KL + 8 * kk, uh, id, 1);
-            }
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-                mma_tf32_ts(tmem + TM_X, tmem + TM_TP + 8 * kk, sdesc_sw128(c.sa + OFF_RU + koff, 16, 1024), id, 1);
-                mma_tf32_ts(tmem + TM_X, tmem + TM_TP + 8 * kk, sdesc_sw128(c.sa + OFF_RL + koff, 16, 1024), id, 1);
+                mma_tf32_ts(tmem + TM_X, tmem + TM_P + 8 * kk, uh, id, 1);
             }
             mma_commit(c.bar[BAR_MMA]);
         }
