@@ -185,7 +185,22 @@ def run_ours(args):
     g.load_library(rebuild_if_stale=(world == 1))
     stream = torch.cuda.current_stream(dev)
 
-    # ---- prefill workload (every rank its own replica; seed differs per rank)
+    B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
+    ms_step = e2e_ms = dec_ms = float("nan")
+    h2d = d2h = 0
+    clk = None
+    if args.workload in ("all", "prefill"):
+        ms_step, e2e_ms, h2d, d2h, clk = run_prefill(args, torch, dist, g, world, rank, dev, stream)
+    if args.workload in ("all", "decode"):
+        dec_ms = run_decode(args, torch, dist, g, world, rank, dev, stream)
+    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_prefill(args, torch, dist, g, world, rank, dev, stream):
+    """Device-timed prefill steps and the end-to-end variant; returns timings."""
     B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
     x = gi.chunk_inputs(**PREFILL, seed=rank)
     d = device_inputs(torch, x, dev)
@@ -207,7 +222,7 @@ def run_ours(args):
     step()
     torch.cuda.synchronize()
     per = max(time.perf_counter() - t_est, 1e-5)
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         for _ in range(int(min(4000, 1.2 / per))):
             step()
         ev0.record(stream)
@@ -222,8 +237,6 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_total = float(t.item())
     ms_step = ms_total / args.steps
-    tokens_per_step = B * T
-    value = tokens_per_step * world / (ms_step / 1e3)
 
     # ---- e2e: pinned host buffers, copies inside the timed region
     host = {n: d[n].cpu().pin_memory() for n in d}
@@ -253,11 +266,15 @@ def run_ours(args):
         t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    del host, o_h, S_h
-
-    # ---- decode workload: 64 consecutive in-place steps, timed as one region
-    del d, o, ST
+    del host, o_h, S_h, d, o, ST
     torch.cuda.empty_cache()
+    return ms_step, e2e_ms, h2d, d2h, clk
+
+
+def run_decode(args, torch, dist, g, world, rank, dev, stream):
+    """64 consecutive in-place decode steps timed as one region; returns ms per step."""
+    dv = DECODE["dv"]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     xd = gi.decode_inputs(**DECODE, seed=rank)
     steps_d = DECODE["steps"]
     Bd, Hd = DECODE["B"], DECODE["H"]
@@ -285,7 +302,21 @@ def run_ours(args):
         t = torch.tensor([dec_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dec_ms = float(t.item())
+    del dd, S0d, Sd, od, views
+    torch.cuda.empty_cache()
+    return dec_ms
 
+
+def _num(x):
+    return None if x != x else x      # NaN (workload not run) -> null
+
+
+def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk):
+    B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
+    Bd, Hd = DECODE["B"], DECODE["H"]
+    steps_d = DECODE["steps"]
+    reps = 3
+    value = B * T * world / (ms_step / 1e3)
     hbm, hbm_src = measured_peaks()
     pre_bytes = prefill_bytes(B, T, H, dk, dv)
     pre_gbs = pre_bytes / (ms_step / 1e3) / 1e9
@@ -301,33 +332,31 @@ def run_ours(args):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC, "value": _num(value), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": _num(ms_step), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; recipe in gdn2_inputs.py)",
             "config": {"workload": "GDN-2 chunkwise prefill B=4 T=4096 H=16 d_k=d_v=128 chunk=64, S0=0",
                        "global_batch": B * world, "seq_len": T, "heads": H, "d_k": dk, "d_v": dv,
                        "dtypes": "q/k/v/o bf16, alpha/b/w fp32, state fp32, fp32 accumulation",
                        "l2": "inputs (675 MB per call) larger than the 126 MB L2; no flush",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-            "e2e": {"value": B * T * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "roofline": {"bound": "hbm", "achieved": pre_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": pre_gbs / hbm, "traffic": traffic.get("gdn2_chunk"),
+            "e2e": {"value": _num(B * T * world / (e2e_ms / 1e3)), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": _num(e2e_ms)},
+            "roofline": {"bound": "hbm", "achieved": _num(pre_gbs), "peak": hbm, "unit": "GB/s",
+                         "frac": _num(pre_gbs / hbm), "traffic": traffic.get("gdn2_chunk"),
                          "kernel": "gdn2 chunkwise prefill", "algorithmic_bytes_per_launch": pre_bytes,
-                         "peak_source": f"{hbm_src} HBM copy bandwidth", "frac_of_8TBps": pre_gbs / 8000.0},
-            "decode": {"metric": "GDN-2 decode state GB/s @B256 H16 d128", "value": st_gbs, "unit": "GB/s",
-                       "us_per_step": dec_ms * 1e3, "steps": steps_d * reps,
-                       "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
-                                    "frac": dec_gbs / hbm, "traffic": traffic.get("gdn2_decode"),
-                                    "algorithmic_bytes_per_launch": dec_bytes, "frac_of_8TBps": dec_gbs / 8000.0}},
+                         "peak_source": f"{hbm_src} HBM copy bandwidth", "frac_of_8TBps": _num(pre_gbs / 8000.0)},
+            "decode": {"metric": "GDN-2 decode state GB/s @B256 H16 d128", "value": _num(st_gbs), "unit": "GB/s",
+                       "us_per_step": _num(dec_ms * 1e3), "steps": steps_d * reps,
+                       "roofline": {"bound": "hbm", "achieved": _num(dec_gbs), "peak": hbm, "unit": "GB/s",
+                                    "frac": _num(dec_gbs / hbm), "traffic": traffic.get("gdn2_decode"),
+                                    "algorithmic_bytes_per_launch": dec_bytes,
+                                    "frac_of_8TBps": _num(dec_gbs / 8000.0)}},
             "gpu_launches": args.steps,
-            "clocks": clk.summary(),
+            "clocks": clk.summary() if clk is not None else None,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
 
 
 def load_traffic():
@@ -384,6 +413,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["all", "prefill", "decode"], default="all",
+                    help="run only one workload's measurement (for profiling one kernel)")
     args = ap.parse_args()
     if args.impl == "ours":
         args.warmup = max(3, args.warmup)       # at least 3 untimed warm-up steps
