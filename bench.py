@@ -360,19 +360,22 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk):
 
 
 def load_traffic():
-    """Per-launch DRAM traffic from the committed ncu summary, if it matches the current sources."""
+    """Per-launch DRAM traffic from the committed ncu summary (profiles/traffic.json),
+    or None for a kernel whose sources changed since that capture."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return {}
     try:
         with open(path) as f:
             data = json.load(f)
-        import hashlib
         out = {}
         for name, rec in data.items():
-            src = os.path.join(ROOT, rec["source"])
-            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-            out[name] = rec["bytes_per_launch"] if h == rec.get("source_sha256_16") else None
+            m = hashlib.sha256()
+            for src in rec["sources"]:
+                with open(os.path.join(ROOT, src), "rb") as f:
+                    m.update(f.read())
+            out[name] = rec["bytes_per_launch"] if m.hexdigest()[:16] == rec["sources_sha256_16"] else None
         return out
     except (OSError, KeyError, ValueError):
         return {}
