@@ -10,8 +10,9 @@
 //   gamma_t = prod_{j<=t} alpha_j,  rho_t = 1/gamma_t          (per key channel, FP32)
 //   Etil = b*k*gamma,  Qtil = q*gamma,  Ktil = k*rho            (gate prep)
 //   [A | Etil S] and [P | Qtil S] = [Etil; Qtil] [Ktil; S^T]^T  (one tensor-core product)
+//   T = (I + strict_tril(A))^{-1}                                (FP32 blocked inversion)
 //   R = w*v - Etil S                                             (FP32 epilogue)
-//   (I + strict_tril(A)) U = R                                   (FP32 blocked forward substitution)
+//   U = T R                                                      (tensor core)
 //   O = Qtil S + tril(P) U                                       (tensor core, accumulated)
 //   S <- diag(gamma_n) (S + Ktil^T U)                            (tensor core + FP32 epilogue)
 //
@@ -19,9 +20,9 @@
 // is the token loop's arithmetic, re-associated.
 //
 // Precision: tensor-core operands are TF32 (10-bit mantissa); accumulation,
-// decay, R, the solve and the carried state are FP32.  The state update uses
-// split operands, x = x_hi + x_lo with both parts TF32:
-//   Ktil^T U = Ktil_hi^T U_hi + Ktil_hi^T U_lo + Ktil_lo^T U_hi,
+// decay, R, T and the carried state are FP32.  The state path uses split
+// operands, x = x_hi + x_lo with both parts TF32:
+//   T R = T R_hi + T R_lo,  Ktil^T U = Ktil_hi^T U_hi + Ktil_hi^T U_lo + Ktil_lo^T U_hi,
 // which carries about 21 bits of each operand (plain TF32 there lets the state
 // drift by ~0.7% of its RMS over 16K tokens; split, ~0.03%).  BF16 operands lose
 // too much: the read r = Sbar^T e nearly cancels the write z in the delta rule.
@@ -29,13 +30,15 @@
 // must stay below ~1e34 (sum of -ln alpha over one chunk <= 78 per key channel),
 // as documented in gdn2.h.
 //
-// Layout: one CTA per (batch, head, 64-column half of d_v); 256 threads (8
+// Layout: one CTA per (batch, head, 64-column half of d_v); 512 threads (16
 // warps) run the phases of a chunk in turn; thread 0 issues TMA loads and MMAs.
-// Every shared-memory MMA operand is K-major with the 128-byte swizzle.  The
-// operands needed transposed (Ktil^T, P) are written to Tensor Memory and read
-// from there as the A operand.  alpha, b and w are TMA-loaded straight into the
-// tiles they become and transformed in place; each next-chunk load is issued as
-// soon as its tile is consumed.
+// Warp w reads Tensor Memory lanes 32 (w % 4) .. +31 and owns the 16-column
+// quarter w / 4 of every 64-column accumulator.  Every shared-memory MMA operand
+// is K-major with the 128-byte swizzle; the operands needed transposed (Ktil^T,
+// [T; P]) are written to Tensor Memory and read from there as the A operand.
+// alpha, b and w are TMA-loaded straight into the tiles they become and
+// transformed in place; each next-chunk load is issued as soon as its tile is
+// consumed.
 #include <cudaTypedefs.h>
 #include <stdio.h>
 
@@ -53,16 +56,16 @@ using namespace sm100;
 constexpr int kC = 64;            // chunk length (tokens)
 constexpr int kDK = 128;          // key channels
 constexpr int kDVS = 64;          // value columns per CTA
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr long long kWaitLimit = 4000000000ll;   // ~2 s of SM cycles per wait
 
 // Shared-memory map (bytes from a 1024-aligned base).  MMA tiles hold TF32,
 // 32 elements per 128-byte swizzled row, K-major:
 //   X1  rows 0-63 Etil[t][i], rows 64-127 Qtil[t][i]         4 atoms x 16 KB (i = key channel)
 //   KS  rows 0-63 Ktil_hi[s][i], rows 64-127 S[i][j] as [j][i]  4 atoms x 16 KB
-//   UH  U_hi as [j][t]                                        2 atoms x 8 KB (t = token)
-//   UL  U_lo as [j][t]                                        2 atoms x 8 KB
-//   ZW  w, then R, then U, as [t][j] (FP32, same swizzle)     2 atoms x 8 KB
+//   UH  R_hi, later U_hi, as [j][t]                           2 atoms x 8 KB (t = token)
+//   UL  R_lo, later U_lo, as [j][t]                           2 atoms x 8 KB
+//   ZW  w as [t][j] (FP32, same swizzle; TMA destination)     2 atoms x 8 KB
 // and unswizzled BF16 staging of q, k (64 x 128) and v (64 x 64).
 constexpr uint32_t OFF_X1 = 0;
 constexpr uint32_t OFF_KS = OFF_X1 + 65536;
@@ -73,24 +76,29 @@ constexpr uint32_t OFF_RQ = OFF_ZW + 16384;
 constexpr uint32_t OFF_RK = OFF_RQ + 16384;
 constexpr uint32_t OFF_RV = OFF_RK + 16384;
 constexpr uint32_t OFF_GN = OFF_RV + 8192;      // float[128]   decay over the chunk
-constexpr uint32_t OFF_PART = OFF_GN + 512;     // float[2][128] half-chunk decay products
-constexpr uint32_t OFF_BAR = OFF_PART + 1024;   // mbarriers
+constexpr uint32_t OFF_PART = OFF_GN + 512;     // float[4][128] quarter-chunk decay products
+constexpr uint32_t OFF_BAR = OFF_PART + 2048;   // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 64;     // tmem base, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // + alignment slack
-// Solve scratch inside the q/k staging (free between prep and the next load).
-constexpr int LDA = 65, LDD = 17;
-constexpr uint32_t OFF_AS = OFF_RQ;             // float[64][65]    A, strictly lower
-constexpr uint32_t OFF_DS = OFF_AS + 16896;     // float[4][16][17] inverses of the diagonal blocks
-static_assert(OFF_DS + 4 * 16 * LDD * 4 <= OFF_RV, "solve scratch overlaps the v staging");
+// Inversion scratch inside the q/k/v staging (A is written after the prep has
+// consumed q and k; T only after the R epilogue has consumed v).
+constexpr int LDT = 66;
+constexpr uint32_t OFF_AT = OFF_RQ;                     // float[64][66]  A transposed: AT[s][t] = A[t][s]
+constexpr uint32_t OFF_TS = OFF_AT + 64 * LDT * 4;      // float[64][66]  T
+constexpr uint32_t OFF_XS = OFF_TS + 64 * LDT * 4;      // float[32][34]  block products
+constexpr int LDX = 34;
+static_assert(OFF_AT + 64 * LDT * 4 <= OFF_RV, "A scratch overlaps the v staging");
+static_assert(OFF_XS + 32 * LDX * 4 <= OFF_GN, "inversion scratch overflows the staging area");
 
 // Tensor Memory columns (512 allocated).
 constexpr uint32_t TM_G = 0;      // [Etil;Qtil] Ktil^T : lanes 0-63 A, lanes 64-127 P   (64 cols)
 constexpr uint32_t TM_X = 64;     // [Etil;Qtil] S, then + P U : lanes 64-127 -> O        (64 cols)
-constexpr uint32_t TM_D = 128;    // Ktil^T U                                             (64 cols)
-constexpr uint32_t TM_KT = 192;   // A operand Ktil_hi^T: lane i, column s                (64 cols)
-constexpr uint32_t TM_KL = 256;   // A operand Ktil_lo^T                                  (64 cols)
-constexpr uint32_t TM_P = 320;    // A operand: lanes 64-127 tril(P), lanes 0-63 zero     (64 cols)
+constexpr uint32_t TM_U = 128;    // [T;P] R : lanes 0-63 U                               (64 cols)
+constexpr uint32_t TM_D = 192;    // Ktil^T U                                             (64 cols)
+constexpr uint32_t TM_KT = 256;   // A operand Ktil_hi^T: lane i, column s                (64 cols)
+constexpr uint32_t TM_KL = 320;   // A operand Ktil_lo^T                                  (64 cols)
+constexpr uint32_t TM_TP = 384;   // A operand [T; P]: lane t (P at 64 + t), column s     (64 cols)
 constexpr uint32_t TM_COLS = 512;
 
 enum { BAR_QKV = 0, BAR_A, BAR_B, BAR_W, BAR_MMA, NBARS };
@@ -99,11 +107,6 @@ constexpr uint32_t TX_QKV = 16384 + 16384 + 8192;
 constexpr uint32_t TX_A = 4 * 8192;
 constexpr uint32_t TX_B = 4 * 8192;
 constexpr uint32_t TX_W = 2 * 8192;
-
-// Element byte offsets inside the tiles.
-__device__ __forceinline__ uint32_t x_off(uint32_t r, uint32_t i) { return (i >> 5) * 16384u + swz128(r, (i & 31u) * 4u); }
-__device__ __forceinline__ uint32_t u_off(uint32_t j, uint32_t t) { return (t >> 5) * 8192u + swz128(j, (t & 31u) * 4u); }
-__device__ __forceinline__ uint32_t zw_off(uint32_t t, uint32_t j) { return (j >> 5) * 8192u + swz128(t, (j & 31u) * 4u); }
 
 struct Maps {
     CUtensorMap q, k, v, alpha, b, w;
@@ -117,7 +120,19 @@ struct Ctx {
 
 __device__ __forceinline__ float *fptr(const Ctx &c, uint32_t off) { return reinterpret_cast<float *>(c.sm + off); }
 __device__ __forceinline__ float &at(const Ctx &c, uint32_t off) { return *reinterpret_cast<float *>(c.sm + off); }
+__device__ __forceinline__ float2 &at2(const Ctx &c, uint32_t off) { return *reinterpret_cast<float2 *>(c.sm + off); }
 __device__ __forceinline__ float4 &at4(const Ctx &c, uint32_t off) { return *reinterpret_cast<float4 *>(c.sm + off); }
+
+// Swizzled offsets of one fixed 4-byte column position in a tile with 128-byte
+// rows: element (row, byte cb) is at row*128 + sw[row % 8].  Indexing sw[] with
+// a compile-time row keeps the XOR out of the inner loops.
+struct Swz {
+    uint32_t o[8];
+    __device__ __forceinline__ explicit Swz(uint32_t cb) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[k] = ((((cb >> 4) ^ k) & 7u) << 4) | (cb & 15u);
+    }
+};
 
 // TMA loads of one chunk's inputs (thread 0 only).
 __device__ __forceinline__ void load_qkv(const Ctx &c, const Maps &m, int h, int t0, int bidx, int col0) {
@@ -142,83 +157,69 @@ __device__ __forceinline__ void load_w(const Ctx &c, const Maps &m, int h, int t
 __device__ __forceinline__ float ldbf(const uint8_t *p) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p)); }
 
 // ---------------------------------------------------------------------------
-// Gate prep.  Thread (lane quarter qd, half th, lane l) owns key channel
-// i = 32 qd + l for tokens [32 th, 32 th + 32).  Cumulative decay is a running
-// FP32 product (exp of the cumulative log-decay up to rounding).  Padding tokens
-// (t >= n) have zero q, k, b from the TMA bounds fill and alpha forced to 1.
-// Tokens go in groups of 8; a group's loads are issued before the previous
-// group's stores so the in-place writes never stall the reads.
-__device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, int qd, int th, int lane, int n) {
+// Gate prep.  Thread (lane quarter qd, token quarter cq, lane l) owns key
+// channel i = 32 qd + l for tokens [16 cq, 16 cq + 16).  Cumulative decay is a
+// running FP32 product (exp of the cumulative log-decay up to rounding).
+// Padding tokens (t >= n) have zero q, k, b from the TMA bounds fill and alpha
+// forced to 1.  All loads of the 16 tokens precede the in-place stores.
+__device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, int qd, int cq, int lane, int n) {
     const int i = 32 * qd + lane;
+    const Swz sw((i & 31) * 4u);
+    const uint32_t rbase = (i >> 5) * 16384u + cq * 16 * 128;   // atom of channel i, first row of the quarter
     float *part = fptr(c, OFF_PART);
-    const uint32_t ci = (i >> 5) * 16384u;       // atom of channel i
-    const uint32_t cb = (i & 31) * 4u;           // byte in row
+    float av[16], bv[16], kv[16], qv[16];
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) {
+        const uint32_t o = rbase + tt * 128 + sw.o[tt & 7];
+        av[tt] = at(c, OFF_KS + o);
+        bv[tt] = at(c, OFF_X1 + o);
+        const int t = 16 * cq + tt;
+        kv[tt] = ldbf(c.sm + OFF_RK + t * 256 + i * 2);
+        qv[tt] = ldbf(c.sm + OFF_RQ + t * 256 + i * 2);
+    }
     float pa = 1.f;
 #pragma unroll
-    for (int tt = 0; tt < 32; ++tt) {
-        const int t = 32 * th + tt;
-        const float a = at(c, OFF_KS + ci + swz128(t, cb));
-        pa *= (t < n) ? clamp_alpha(a) : 1.f;
+    for (int tt = 0; tt < 16; ++tt) {
+        av[tt] = (16 * cq + tt < n) ? clamp_alpha(av[tt]) : 1.f;
+        pa *= av[tt];
     }
-    part[th * 128 + i] = pa;
+    part[cq * 128 + i] = pa;
     __syncthreads();
-    const float p0 = part[i], p1 = part[128 + i];
-    if (th == 0) fptr(c, OFF_GN)[i] = p0 * p1;
-    float g = th ? p0 : 1.f;
-    float r = 1.f / g;
-    float av[8], kv[8], qv[8], bv[8];
-    auto load_group = [&](int g8) {
+    float g = 1.f, tot = 1.f;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = 32 * th + 8 * g8 + u;
-            av[u] = at(c, OFF_KS + ci + swz128(t, cb));
-            bv[u] = at(c, OFF_X1 + ci + swz128(t, cb));
-            kv[u] = ldbf(c.sm + OFF_RK + t * 256 + i * 2);
-            qv[u] = ldbf(c.sm + OFF_RQ + t * 256 + i * 2);
-        }
-    };
-    load_group(0);
-#pragma unroll
-    for (int g8 = 0; g8 < 4; ++g8) {
-        float e[8], qt[8], kh[8], kl[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = 32 * th + 8 * g8 + u;
-            const float a = (t < n) ? clamp_alpha(av[u]) : 1.f;
-            g *= a;
-            r *= __fdividef(1.f, a);
-            e[u] = to_tf32(bv[u] * kv[u] * g);
-            qt[u] = to_tf32(qv[u] * g);
-            const float kf = kv[u] * r;
-            kh[u] = to_tf32(kf);
-            kl[u] = to_tf32(kf - kh[u]);
-        }
-        if (g8 < 3) load_group(g8 + 1);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = 32 * th + 8 * g8 + u;
-            at(c, OFF_X1 + ci + swz128(t, cb)) = e[u];
-            at(c, OFF_X1 + ci + swz128(64 + t, cb)) = qt[u];
-            at(c, OFF_KS + ci + swz128(t, cb)) = kh[u];
-        }
-        tmem_st8(tlane + TM_KT + 32 * th + 8 * g8, kh);
-        tmem_st8(tlane + TM_KL + 32 * th + 8 * g8, kl);
+    for (int q2 = 0; q2 < 4; ++q2) {
+        const float p = part[q2 * 128 + i];
+        g = (q2 < cq) ? g * p : g;
+        tot *= p;
     }
+    if (cq == 0) fptr(c, OFF_GN)[i] = tot;
+    float r = 1.f / g;
+    float kh[16], kl[16];
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) {
+        g *= av[tt];
+        r *= __fdividef(1.f, av[tt]);
+        const uint32_t o = rbase + tt * 128 + sw.o[tt & 7];
+        at(c, OFF_X1 + o) = to_tf32(bv[tt] * kv[tt] * g);
+        at(c, OFF_X1 + o + 64 * 128) = to_tf32(qv[tt] * g);      // Qtil: rows 64-127, same swizzle phase
+        const float kf = kv[tt] * r;
+        kh[tt] = to_tf32(kf);
+        kl[tt] = to_tf32(kf - kh[tt]);
+        at(c, OFF_KS + o) = kh[tt];
+    }
+    tmem_st16(tlane + TM_KT + 16 * cq, kh);
+    tmem_st16(tlane + TM_KL + 16 * cq, kl);
 }
 
 // ---------------------------------------------------------------------------
-// Solve (I + A) U = R in FP32, A strictly lower 64 x 64 (As), R and U in the ZW
-// tile ([t][j], 64 value columns).  The inverses D_b of the four 16 x 16
-// diagonal blocks come first (forward substitution, one thread per column);
-// then, block by block, R'_b = R_b - sum_{c<b} A_bc U_c and U_b = D_b R'_b.
-// Thread (i, cg) owns row 16 b + i, columns 4 cg .. 4 cg + 3 of each block.
-__device__ __forceinline__ void fma4(float4 &acc, float a, const float4 &x) {
-    acc.x = fmaf(a, x.x, acc.x); acc.y = fmaf(a, x.y, acc.y); acc.z = fmaf(a, x.z, acc.z); acc.w = fmaf(a, x.w, acc.w);
-}
-
-__device__ __forceinline__ void solve_u(const Ctx &c, int tid) {
-    const float *As = fptr(c, OFF_AS);
-    float *Ds = fptr(c, OFF_DS);
+// T = (I + A)^{-1} in FP32, A strictly lower 64 x 64 given transposed (AT[s][t]).
+// 16 x 16 diagonal blocks D_b by forward substitution; then T_10 = -D_1 A_10 D_0,
+// T_32 = -D_3 A_32 D_2; then the lower-left 32 x 32 block T_BA = -T_BB A_BA T_AA.
+// Result in Ts (row-major, zero above the diagonal).
+__device__ __forceinline__ void invert(const Ctx &c, int tid) {
+    const float *AT = fptr(c, OFF_AT);
+    float *Ts = fptr(c, OFF_TS);
+    float *Xs = fptr(c, OFF_XS);
     if (tid < 64) {
         const int b = tid >> 4, j = tid & 15, base = 16 * b;
         float x[16];
@@ -226,30 +227,82 @@ __device__ __forceinline__ void solve_u(const Ctx &c, int tid) {
         for (int i = 0; i < 16; ++i) {
             float acc = (i == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int l = 0; l < i; ++l) acc = fmaf(-As[(base + i) * LDA + base + l], x[l], acc);
+            for (int l = 0; l < i; ++l) acc = fmaf(-AT[(base + l) * LDT + base + i], x[l], acc);
             x[i] = acc;
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) Ds[(b * 16 + i) * LDD + j] = x[i];
+        for (int i = 0; i < 16; ++i) Ts[(base + i) * LDT + base + j] = x[i];
+    } else {
+        // zero the blocks above the diagonal: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+        for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
+            const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
+            const int a = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int b = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            Ts[(16 * a + i) * LDT + 16 * b + j] = 0.f;
+        }
     }
     __syncthreads();
-    const int i = tid >> 4, cg = tid & 15;
+    {   // X = A_{a,a-1} D_{a-1} for a = 1, 3 (one output per thread)
+        const int blk = tid >> 8, i = (tid >> 4) & 15, j = tid & 15;
+        const int a = blk ? 3 : 1, b = a - 1;
+        float acc = 0.f;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        const int row = 16 * b + i;
-        const uint32_t my = OFF_ZW + zw_off(row, 4 * cg);
-        float4 acc = at4(c, my);
+        for (int l = 0; l < 16; ++l) acc = fmaf(AT[(16 * b + l) * LDT + 16 * a + i], Ts[(16 * b + l) * LDT + 16 * b + j], acc);
+        Xs[blk * 16 * LDX + i * LDX + j] = acc;
+    }
+    __syncthreads();
+    {   // T_{a,a-1} = -D_a X
+        const int blk = tid >> 8, i = (tid >> 4) & 15, j = tid & 15;
+        const int a = blk ? 3 : 1, b = a - 1;
+        float acc = 0.f;
 #pragma unroll
-        for (int l = 0; l < 16 * b; ++l) fma4(acc, -As[row * LDA + l], at4(c, OFF_ZW + zw_off(l, 4 * cg)));
-        at4(c, my) = acc;
-        __syncthreads();
-        float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int l = 0; l < 16; ++l) acc = fmaf(Ts[(16 * a + i) * LDT + 16 * a + l], Xs[blk * 16 * LDX + l * LDX + j], acc);
+        Ts[(16 * a + i) * LDT + 16 * b + j] = -acc;
+    }
+    __syncthreads();
+    // Y = A_BA T_AA (32 x 32): 256 threads, 2 x 2 outputs each
+    if (tid < 256) {
+        const int i = 2 * (tid >> 4), j = 2 * (tid & 15);
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll 8
+        for (int l = 0; l < 32; ++l) {
+            const float2 a = *reinterpret_cast<const float2 *>(AT + l * LDT + 32 + i);   // A[32+i][l], A[33+i][l]
+            const float2 t = *reinterpret_cast<const float2 *>(Ts + l * LDT + j);         // T[l][j], T[l][j+1]
+            y00 = fmaf(a.x, t.x, y00); y01 = fmaf(a.x, t.y, y01);
+            y10 = fmaf(a.y, t.x, y10); y11 = fmaf(a.y, t.y, y11);
+        }
+        *reinterpret_cast<float2 *>(Xs + i * LDX + j) = make_float2(y00, y01);
+        *reinterpret_cast<float2 *>(Xs + (i + 1) * LDX + j) = make_float2(y10, y11);
+    }
+    __syncthreads();
+    // T_BA = -T_BB Y
+    if (tid < 256) {
+        const int i = 2 * (tid >> 4), j = 2 * (tid & 15);
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll 8
+        for (int l = 0; l < 32; ++l) {
+            const float a0 = Ts[(32 + i) * LDT + 32 + l], a1 = Ts[(33 + i) * LDT + 32 + l];
+            const float2 y = *reinterpret_cast<const float2 *>(Xs + l * LDX + j);
+            y00 = fmaf(a0, y.x, y00); y01 = fmaf(a0, y.y, y01);
+            y10 = fmaf(a1, y.x, y10); y11 = fmaf(a1, y.y, y11);
+        }
+        *reinterpret_cast<float2 *>(Ts + (32 + i) * LDT + j) = make_float2(-y00, -y01);
+        *reinterpret_cast<float2 *>(Ts + (33 + i) * LDT + j) = make_float2(-y10, -y11);
+    }
+    __syncthreads();
+}
+
+// Split x into TF32 hi + lo parts and store both into the [j][t] tiles UH / UL
+// at token t (this thread's TMEM lane), columns 16 cq .. 16 cq + 15.
+__device__ __forceinline__ void store_split_jt(const Ctx &c, const float (&x)[16], int t, int cq) {
+    const Swz sw((t & 31) * 4u);
+    const uint32_t base = (t >> 5) * 8192u + cq * 16 * 128;
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
-            if (m <= i) fma4(u, Ds[(b * 16 + i) * LDD + m], at4(c, OFF_ZW + zw_off(16 * b + m, 4 * cg)));
-        __syncthreads();
-        at4(c, my) = u;
-        __syncthreads();
+    for (int j = 0; j < 16; ++j) {
+        const uint32_t o = base + j * 128 + sw.o[j & 7];
+        const float hi = to_tf32(x[j]);
+        at(c, OFF_UH + o) = hi;
+        at(c, OFF_UL + o) = to_tf32(x[j] - hi);
     }
 }
 
@@ -266,7 +319,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
     volatile uint32_t *abort_flag = misc + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qd = warp & 3, chh = warp >> 2;          // TMEM lane quarter, column half
+    const int qd = warp & 3, cq = warp >> 2;            // TMEM lane quarter, 16-column quarter
     const int head = blockIdx.x >> 1, half = blockIdx.x & 1;
     const int bidx = head / H, h = head % H;
     const int col0 = half * kDVS;
@@ -295,27 +348,27 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         load_b(c, maps, h, 0, bidx);
         load_w(c, maps, h, 0, bidx, col0);
     }
-    if (srow < 64) {   // rows 0-63 of the P operand stay zero
-        float z[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) z[j] = 0.f;
-        tmem_st32(tlane + TM_P + 32 * chh, z);
-    }
 
     // State slice owned by this thread: key channel i = srow, value columns
-    // col0 + 32*chh + [0, 32).  FP32 in registers across all chunks; its TF32
+    // col0 + 16 cq + [0, 16).  FP32 in registers across all chunks; its TF32
     // copy is KS rows 64 + j (j = local column), channel i.
-    float S[32];
+    const Swz ssw((srow & 31) * 4u);
+    const uint32_t sbase = OFF_KS + (srow >> 5) * 16384u + (64 + 16 * cq) * 128;
+    float S[16];
     {
-        const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 32 * chh;
+        const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 16 * cq;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
+        for (int j = 0; j < 16; j += 4) {
             float4 x = S0 ? *reinterpret_cast<const float4 *>(S0 + off + j) : make_float4(0.f, 0.f, 0.f, 0.f);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) at(c, OFF_KS + x_off(64 + 32 * chh + j, srow)) = to_tf32(S[j]);
+        for (int j = 0; j < 16; ++j) at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(S[j]);
     }
+
+    // Shared-memory descriptors (start address advanced per K step).
+    const uint64_t dX1 = sdesc_sw128(c.sa + OFF_X1, 16, 1024), dKS = sdesc_sw128(c.sa + OFF_KS, 16, 1024);
+    const uint64_t dUH = sdesc_sw128(c.sa + OFF_UH, 16, 1024), dUL = sdesc_sw128(c.sa + OFF_UL, 16, 1024);
 
     uint32_t mma_phase = 0;
     bool ok = true;
@@ -346,16 +399,16 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         const bool more = ck + 1 < nchunks;
         // ---- gate prep
         if (!(ok = wait_all(BAR_QKV, ph) && wait_all(BAR_A, ph) && wait_all(BAR_B, ph))) break;
-        prep(c, tlane, qd, chh, lane, n);
+        prep(c, tlane, qd, cq, lane, n);
         sync_for_mma();
         // ---- [Etil; Qtil] x [Ktil; S^T]^T -> TM_G (Gram) and TM_X (Etil S, Qtil S)
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id = idesc_tf32(128, 128, 0, 0);
+#pragma unroll
             for (int kk = 0; kk < 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_tf32(tmem + TM_G, sdesc_sw128(c.sa + OFF_X1 + koff, 16, 1024),
-                         sdesc_sw128(c.sa + OFF_KS + koff, 16, 1024), id, kk > 0);
+                const uint32_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                mma_tf32(tmem + TM_G, dX1 + koff, dKS + koff, id, kk > 0);
             }
             mma_commit(c.bar[BAR_MMA]);
         }
@@ -365,92 +418,103 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             load_b(c, maps, h, t0 + kC, bidx);
         }
         {
-            float g[32];
-            tmem_ld32(tlane + TM_G + 32 * chh, g);
-            if (srow < 64) {        // A row (strictly lower) and R = w*v - Etil S, in place over w
-                float *As = fptr(c, OFF_AS);
+            float g[16];
+            tmem_ld16(tlane + TM_G + 16 * cq, g);
+            if (srow < 64) {        // A row (strictly lower, transposed into AT) and R = w*v - Etil S
+                float *AT = fptr(c, OFF_AT);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int s = 32 * chh + j;
-                    As[srow * LDA + s] = (s < srow) ? g[j] : 0.f;
+                for (int j = 0; j < 16; ++j) {
+                    const int s = 16 * cq + j;
+                    AT[s * LDT + srow] = (s < srow) ? g[j] : 0.f;
                 }
-                float x[32];
-                tmem_ld32(tlane + TM_X + 32 * chh, x);
+                float x[16];
+                tmem_ld16(tlane + TM_X + 16 * cq, x);
+                const int ch = (16 * cq) >> 2;          // first 16-byte chunk of this quarter's columns
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const int col = 32 * chh + j;
-                    float4 &wr = at4(c, OFF_ZW + zw_off(srow, col));
-                    const float4 w = wr;
-                    const uint2 vb = *reinterpret_cast<const uint2 *>(c.sm + OFF_RV + srow * 128 + col * 2);
+                for (int m = 0; m < 4; ++m) {
+                    const int cc = ch + m;              // chunk among the 16 of a row (two 8-chunk atoms)
+                    const uint32_t zo = (cc >> 3) * 8192u + srow * 128 + ((((cc & 7) ^ (srow & 7))) << 4);
+                    const float4 w = at4(c, OFF_ZW + zo);
+                    const uint2 vb = *reinterpret_cast<const uint2 *>(c.sm + OFF_RV + srow * 128 + (4 * cc) * 2);
                     const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.x));
                     const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.y));
-                    wr = make_float4(w.x * v01.x - x[j], w.y * v01.y - x[j + 1], w.z * v23.x - x[j + 2],
-                                     w.w * v23.y - x[j + 3]);
+                    x[4 * m] = w.x * v01.x - x[4 * m];
+                    x[4 * m + 1] = w.y * v01.y - x[4 * m + 1];
+                    x[4 * m + 2] = w.z * v23.x - x[4 * m + 2];
+                    x[4 * m + 3] = w.w * v23.y - x[4 * m + 3];
                 }
+                store_split_jt(c, x, srow, cq);
             } else {                // P row (lower incl. diagonal) -> A operand in TMEM
                 const int t = srow - 64;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) g[j] = (32 * chh + j <= t) ? to_tf32(g[j]) : 0.f;
-                tmem_st32(tlane + TM_P + 32 * chh, g);
+                for (int j = 0; j < 16; ++j) g[j] = (16 * cq + j <= t) ? to_tf32(g[j]) : 0.f;
+                tmem_st16(tlane + TM_TP + 16 * cq, g);
             }
         }
         __syncthreads();
-        solve_u(c, tid);
-        // U (FP32, ZW) -> U_hi, U_lo tiles as [j][t]
-        {
-            const int t = srow >> 1;                       // token row; two threads per row
-            const int j0 = 32 * (srow & 1) + 16 * chh;     // 16 columns each
+        if (tid == 0 && more) load_w(c, maps, h, t0 + kC, bidx, col0);   // w consumed
+        invert(c, tid);
+        if (srow < 64) {            // T rows -> A operand in TMEM
+            float tv[16];
+            const float *Ts = fptr(c, OFF_TS);
 #pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-                const float4 u = at4(c, OFF_ZW + zw_off(t, j0 + j));
-                const float uu[4] = {u.x, u.y, u.z, u.w};
+            for (int j = 0; j < 16; ++j) tv[j] = to_tf32(Ts[srow * LDT + 16 * cq + j]);
+            tmem_st16(tlane + TM_TP + 16 * cq, tv);
+        }
+        sync_for_mma();
+        // ---- U = [T; P] (R_hi + R_lo) -> TM_U (lanes 0-63)
+        if (tid == 0) {
+            if (more) load_qkv(c, maps, h, t0 + kC, bidx, col0);         // inversion scratch free
+            tc_fence_after();
+            const uint32_t id = idesc_tf32(128, 64, 0, 0);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float hi = to_tf32(uu[e]);
-                    at(c, OFF_UH + u_off(j0 + j + e, t)) = hi;
-                    at(c, OFF_UL + u_off(j0 + j + e, t)) = to_tf32(uu[e] - hi);
-                }
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                mma_tf32_ts(tmem + TM_U, tmem + TM_TP + 8 * kk, dUH + koff, id, kk > 0);
+                mma_tf32_ts(tmem + TM_U, tmem + TM_TP + 8 * kk, dUL + koff, id, 1);
             }
+            mma_commit(c.bar[BAR_MMA]);
+        }
+        if (!(ok = mma_wait())) break;
+        if (srow < 64) {            // U -> U_hi, U_lo
+            float u[16];
+            tmem_ld16(tlane + TM_U + 16 * cq, u);
+            store_split_jt(c, u, srow, cq);
         }
         sync_for_mma();
         // ---- Ktil^T U -> TM_D (split);  P U_hi accumulated onto TM_X (lanes 64-127 become O)
         if (tid == 0) {
-            if (more) {                  // solve scratch and ZW consumed: next q, k, v and w
-                load_qkv(c, maps, h, t0 + kC, bidx, col0);
-                load_w(c, maps, h, t0 + kC, bidx, col0);
-            }
             tc_fence_after();
             const uint32_t id = idesc_tf32(128, 64, 0, 0);
+#pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-                const uint64_t uh = sdesc_sw128(c.sa + OFF_UH + koff, 16, 1024);
-                const uint64_t ul = sdesc_sw128(c.sa + OFF_UL + koff, 16, 1024);
-                mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, uh, id, kk > 0);
-                mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, ul, id, 1);
-                mma_tf32_ts(tmem + TM_D, tmem + TM_KL + 8 * kk, uh, id, 1);
-                mma_tf32_ts(tmem + TM_X, tmem + TM_P + 8 * kk, uh, id, 1);
+                const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, dUH + koff, id, kk > 0);
+                mma_tf32_ts(tmem + TM_D, tmem + TM_KT + 8 * kk, dUL + koff, id, 1);
+                mma_tf32_ts(tmem + TM_D, tmem + TM_KL + 8 * kk, dUH + koff, id, 1);
+                mma_tf32_ts(tmem + TM_X, tmem + TM_TP + 8 * kk, dUH + koff, id, 1);
             }
             mma_commit(c.bar[BAR_MMA]);
         }
         if (!(ok = mma_wait())) break;
         {   // state: S <- gamma_n (S + Ktil^T U); TF32 operand copy for the next chunk
-            float d[32];
-            tmem_ld32(tlane + TM_D + 32 * chh, d);
+            float d[16];
+            tmem_ld16(tlane + TM_D + 16 * cq, d);
             const float gn = fptr(c, OFF_GN)[srow];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 S[j] = gn * (S[j] + d[j]);
-                at(c, OFF_KS + x_off(64 + 32 * chh + j, srow)) = to_tf32(S[j]);
+                at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(S[j]);
             }
         }
         if (srow >= 64) {           // outputs from lanes 64-127 of TM_X
-            float v[32];
-            tmem_ld32(tlane + TM_X + 32 * chh, v);
+            float v[16];
+            tmem_ld16(tlane + TM_X + 16 * cq, v);
             const int t = srow - 64;
             if (t < n) {
-                __nv_bfloat16 *dst = o + (((size_t)bidx * T + t0 + t) * H + h) * 128 + col0 + 32 * chh;
+                __nv_bfloat16 *dst = o + (((size_t)bidx * T + t0 + t) * H + h) * 128 + col0 + 16 * cq;
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
+                for (int j = 0; j < 16; j += 8) {
                     uint4 pk;
                     __nv_bfloat162 p0 = __floats2bfloat162_rn(v[j], v[j + 1]);
                     __nv_bfloat162 p1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
@@ -468,9 +532,9 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
     }
 
     if (ok && S_T) {
-        const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 32 * chh;
+        const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 16 * cq;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
+        for (int j = 0; j < 16; j += 4)
             *reinterpret_cast<float4 *>(S_T + off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
     if (!ok && tid == 0) {
