@@ -372,8 +372,10 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
 
     uint32_t mma_phase = 0;
     bool ok = true;
+    // One lane polls the mbarrier; the other warps wait at the CTA barrier, which
+    // costs them no issue slots.  The barrier also publishes the TMA-written data.
     auto wait_all = [&](int which, uint32_t parity) {
-        if (!mbar_wait(c.bar[which], parity, kWaitLimit)) {
+        if (tid == 0 && !mbar_wait(c.bar[which], parity, kWaitLimit)) {
             *abort_flag = 1;
             atomicExch(&g_device_error, 1u + (unsigned)which);
         }
