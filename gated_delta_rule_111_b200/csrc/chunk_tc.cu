@@ -32,10 +32,10 @@
 //
 // Organisation: one CTA per (batch, head, 64-column half of d_v), 18 warps in
 // four roles that run concurrently and hand work over through mbarriers:
-//   warp 0      TMA producer (alpha, b into their operand tiles; w, v staging)
+//   warp 0      TMA producer (alpha, b into their operand tiles; q, k staged
+//               as BF16 over the inversion scratch; w, v staging)
 //   warp 1      MMA issuer (one thread, every tcgen05 instruction)
-//   warps 2-9   key side: gate prep, Gram epilogue, blocked inversion of
-//               (I + A); prefetch q and k of the next chunk into registers
+//   warps 2-9   key side: gate prep, Gram epilogue, blocked inversion of (I + A)
 //   warps 10-17 state side: R, U and state/output epilogues; owns the FP32 state
 // The key side of chunk c+1 runs while the state chain of chunk c runs; the
 // key factor Ktil^T and [T; P] are double-buffered in Tensor Memory for that.
@@ -71,6 +71,8 @@ constexpr long long kWaitLimit = 4000000000ll;   // ~2 s of SM cycles per wait
 //   UL  R_lo, later U_lo, as [j][t]                           2 atoms x 8 KB
 //   ZW  w as [t][j] (FP32, same swizzle; TMA destination)     2 atoms x 8 KB
 //   RV  v as [t][j] (BF16, unswizzled; TMA destination)
+//   QK  q, k of the next chunk as BF16 [a][t][32] (a = channel block of 32), 16 KB
+//       each: TMA destinations, read by the gate prep; the same bytes then hold
 //   AS  A, then T in place (FP32 [64][66]);  XS block products (FP32 [32][34])
 constexpr uint32_t OFF_X1 = 0;
 constexpr uint32_t OFF_KS = OFF_X1 + 65536;
@@ -78,15 +80,18 @@ constexpr uint32_t OFF_UH = OFF_KS + 65536;
 constexpr uint32_t OFF_UL = OFF_UH + 16384;
 constexpr uint32_t OFF_ZW = OFF_UL + 16384;
 constexpr uint32_t OFF_RV = OFF_ZW + 16384;
-constexpr int LDA = 66, LDX = 34;
-constexpr uint32_t OFF_AS = OFF_RV + 8192;
-constexpr uint32_t OFF_XS = OFF_AS + 64 * LDA * 4;
-constexpr uint32_t OFF_GN = OFF_XS + 32 * LDX * 4;     // float[2][128] decay over the chunk (by buffer)
+constexpr uint32_t OFF_GN = OFF_RV + 8192;             // float[2][128] decay over the chunk (by buffer)
 constexpr uint32_t OFF_PART = OFF_GN + 1024;           // float[2][128] half-chunk decay products
 constexpr uint32_t OFF_BAR = OFF_PART + 1024;          // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;           // tmem base, abort flag
-constexpr uint32_t SMEM_USED = OFF_MISC + 16;
+constexpr int LDA = 66, LDX = 34;
+constexpr uint32_t OFF_QK = OFF_MISC + 768;            // 1024-aligned
+constexpr uint32_t OFF_AS = OFF_QK;
+constexpr uint32_t OFF_XS = OFF_AS + 64 * LDA * 4;
+constexpr uint32_t SMEM_USED = OFF_QK + 32768;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
+static_assert(OFF_QK % 1024 == 0 && OFF_XS + 32 * LDX * 4 <= SMEM_USED, "shared-memory map");
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 
 // Tensor Memory columns (512 allocated).
 constexpr uint32_t TM_G = 0;        // Gram: lanes 0-63 A, lanes 64-127 P                 (64 cols)
@@ -97,15 +102,16 @@ constexpr uint32_t TM_TP = 320;     // 2 buffers: A operand [T; P], lane t, colu
 constexpr uint32_t TM_COLS = 512;
 
 enum {
-    B_FULL_AB = 0, B_FULL_WV, B_X1_FREE, B_WV_FREE, B_KPREP, B_G_FULL, B_TP_READY, B_S_READY,
+    B_FULL_AB = 0, B_FULL_WV, B_FULL_QK, B_X1_FREE, B_WV_FREE, B_KPREP, B_G_FULL, B_TP_READY, B_S_READY,
     B_X_FULL, B_R_READY, B_U_FULL, B_U_READY, B_D_FULL, B_KT_FREE0, B_KT_FREE1, NBARS
 };
 
 constexpr uint32_t TX_AB = 8 * 8192;
+constexpr uint32_t TX_QK = 8 * 4096;
 constexpr uint32_t TX_WV = 2 * 8192 + 8192;
 
 struct Maps {
-    CUtensorMap v, alpha, b, w;
+    CUtensorMap q, k, v, alpha, b, w;
 };
 
 struct Ctx {
@@ -154,30 +160,6 @@ __device__ __forceinline__ bool solo_wait(const Ctx &c, int which, uint32_t pari
 // Key side.  Thread (lane quarter qd, half kh, lane l) owns key channel
 // i = 32 qd + l for tokens [32 kh, 32 kh + 32) in the gate prep, and TMEM lane
 // 32 qd + l, columns [32 kh, 32 kh + 32) in the Gram epilogue.
-struct KeyRegs {
-    uint32_t q[16], k[16];   // BF16 pairs (tokens 2m, 2m+1) of this thread's channel
-};
-
-__device__ __forceinline__ void prefetch_qk(KeyRegs &r, const __nv_bfloat16 *q, const __nv_bfloat16 *k, int bidx,
-                                            int T, int H, int h, int t0, int kh, int i) {
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-        uint32_t qq = 0, kk = 0;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int t = t0 + 32 * kh + 2 * m + e;
-            if (t < T) {
-                const size_t off = (((size_t)bidx * T + t) * H + h) * kDK + i;
-                const uint32_t qb = __ldg(reinterpret_cast<const unsigned short *>(q) + off);
-                const uint32_t kb = __ldg(reinterpret_cast<const unsigned short *>(k) + off);
-                qq |= qb << (16 * e);
-                kk |= kb << (16 * e);
-            }
-        }
-        r.q[m] = qq;
-        r.k[m] = kk;
-    }
-}
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
@@ -185,8 +167,8 @@ __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 
 // log-decay up to rounding); Etil, Qtil into X1, Ktil into KS (rows 0-63) and
 // its transpose into Tensor Memory.  Padding tokens (t >= n): zero b from the
 // TMA bounds fill, zero q, k, alpha forced to 1.
-__device__ __forceinline__ void prep(const Ctx &c, const KeyRegs &kr, uint32_t tlane, uint32_t kt_col, int kb,
-                                     int qd, int kh, int lane, int n) {
+__device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, uint32_t kt_col, int kb, int qd, int kh,
+                                     int lane, int n) {
     const int i = 32 * qd + lane;
     const Swz sw((i & 31) * 4u);
     const uint32_t rbase = (i >> 5) * 16384u + kh * 32 * 128;
@@ -199,6 +181,8 @@ __device__ __forceinline__ void prep(const Ctx &c, const KeyRegs &kr, uint32_t t
     }
     part[kh * 128 + i] = pa;
     named_bar(kBarK, kGroup);
+    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(c.sm + OFF_QK) + (i >> 5) * 2048 + kh * 1024 + (i & 31);
+    const __nv_bfloat16 *ks = qs + 8192;
     const float p0 = part[i], p1 = part[128 + i];
     if (kh == 0) fptr(c, OFF_GN)[kb * 128 + i] = p0 * p1;
     float g = kh ? p0 : 1.f;
@@ -218,9 +202,7 @@ __device__ __forceinline__ void prep(const Ctx &c, const KeyRegs &kr, uint32_t t
             const float a = (32 * kh + tt < n) ? clamp_alpha(av[u]) : 1.f;
             g *= a;
             r *= __fdividef(1.f, a);
-            const uint32_t qp = kr.q[tt >> 1], kp = kr.k[tt >> 1];
-            const float qq = (tt & 1) ? bf_hi(qp) : bf_lo(qp);
-            const float kk = (tt & 1) ? bf_hi(kp) : bf_lo(kp);
+            const float qq = __bfloat162float(qs[tt * 32]), kk = __bfloat162float(ks[tt * 32]);
             const uint32_t o = rbase + tt * 128 + sw.o[u];
             at(c, OFF_X1 + o) = to_tf32(bv[u] * kk * g);
             at(c, OFF_X1 + o + 64 * 128) = to_tf32(qq * g);          // Qtil rows 64-127, same swizzle phase
@@ -238,17 +220,16 @@ __device__ __forceinline__ void prep(const Ctx &c, const KeyRegs &kr, uint32_t t
 __device__ __forceinline__ void invert(const Ctx &c, int ktid) {
     float *As = fptr(c, OFF_AS);
     float *Xs = fptr(c, OFF_XS);
+    // Column j of D_b: x = e_j, then x_i -= A_il x_l for l < i (x_l final once reached).
     float x[16];
     const int b = ktid >> 4, j = ktid & 15, base = 16 * b;
     if (ktid < 64) {
-        float acc[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = (i == j) ? 1.f : 0.f;
+        for (int i = 0; i < 16; ++i) x[i] = (i == j) ? 1.f : 0.f;
 #pragma unroll
-        for (int l = 0; l < 16; ++l) {
-            x[l] = acc[l];
+        for (int l = 0; l < 15; ++l) {
 #pragma unroll
-            for (int i = l + 1; i < 16; ++i) acc[i] = fmaf(-As[(base + i) * LDA + base + l], x[l], acc[i]);
+            for (int i = l + 1; i < 16; ++i) x[i] = fmaf(-As[(base + i) * LDA + base + l], x[l], x[i]);
         }
     }
     named_bar(kBarK, kGroup);
@@ -327,12 +308,13 @@ __device__ __forceinline__ void store_split_jt(const Ctx &c, const float (&x)[32
 
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
-chunk_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16 *__restrict__ qg,
-                const __nv_bfloat16 *__restrict__ kg, const float *S0, __nv_bfloat16 *__restrict__ o, float *S_T,
+chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat16 *__restrict__ o, float *S_T,
                 int T, int H) {
     extern __shared__ uint8_t smem_raw[];
     Ctx c;
-    c.sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Align by offsetting the __shared__ array itself (not through an integer
+    // cast) so that the compiler keeps every access in the shared window.
+    c.sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     c.sa = smem_u32(c.sm);
     uint32_t *misc = reinterpret_cast<uint32_t *>(c.sm + OFF_MISC);
     c.abort_flag = misc + 1;
@@ -347,6 +329,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16 *__restri
         for (int i = 0; i < NBARS; ++i) mbar_init(c.bar(i), 1);
         fence_mbar_init();
         *c.abort_flag = 0;
+        tma_prefetch_map(&maps.q); tma_prefetch_map(&maps.k);
         tma_prefetch_map(&maps.v); tma_prefetch_map(&maps.alpha);
         tma_prefetch_map(&maps.b); tma_prefetch_map(&maps.w);
     }
@@ -369,6 +352,16 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16 *__restri
                 for (int a = 0; a < 4; ++a) {
                     tma_load_4d(c.sa + OFF_KS + a * 16384, &maps.alpha, 32 * a, h, ck * kC, bidx, fb);
                     tma_load_4d(c.sa + OFF_X1 + a * 16384, &maps.b, 32 * a, h, ck * kC, bidx, fb);
+                }
+            }
+        } else if (lane == 2) {     // q, k -> QK (over the inversion scratch of the previous chunk)
+            for (int ck = 0; ck < nchunks; ++ck) {
+                if (ck > 0 && !solo_wait(c, B_TP_READY, (ck - 1) & 1)) break;
+                const uint32_t fb = c.bar(B_FULL_QK);
+                mbar_expect_tx(fb, TX_QK);
+                for (int a = 0; a < 4; ++a) {
+                    tma_load_4d(c.sa + OFF_QK + a * 4096, &maps.q, 32 * a, h, ck * kC, bidx, fb);
+                    tma_load_4d(c.sa + OFF_QK + 16384 + a * 4096, &maps.k, 32 * a, h, ck * kC, bidx, fb);
                 }
             }
         } else if (lane == 1) {     // w -> ZW, v -> RV
@@ -443,14 +436,12 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16 *__restri
         const int srow = 32 * qd + lane;
         const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);
         const bool el = ktid == 0;
-        KeyRegs kr;
-        prefetch_qk(kr, qg, kg, bidx, T, H, h, 0, kh, srow);
         for (int ck = 0; ck < nchunks; ++ck) {
             const uint32_t ph = ck & 1;
             const int t0 = ck * kC, n = min(kC, T - t0);
-            if (!group_wait(c, B_FULL_AB, ph, el, kBarK)) break;
+            if (!group_wait(c, B_FULL_AB, ph, el, kBarK) || !group_wait(c, B_FULL_QK, ph, el, kBarK)) break;
             if (ck >= 2 && !group_wait(c, ph ? B_KT_FREE1 : B_KT_FREE0, ((ck - 2) >> 1) & 1, el, kBarK)) break;
-            prep(c, kr, tlane, TM_KT + 64 * ph, ph, qd, kh, lane, n);
+            prep(c, tlane, TM_KT + 64 * ph, ph, qd, kh, lane, n);
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
@@ -493,7 +484,6 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16 *__restri
             tc_fence_before();
             named_bar(kBarK, kGroup);
             if (el) mbar_arrive(c.bar(B_TP_READY));
-            if (ck + 1 < nchunks) prefetch_qk(kr, qg, kg, bidx, T, H, h, t0 + kC, kh, srow);
         }
     } else {
         // ------------------------------------------------ state side
@@ -610,6 +600,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16 *__restri
     if (tid == 0 && *c.abort_flag) {
         (void)mbar_wait(c.bar(B_FULL_AB), 0, kWaitLimit / 8);
         (void)mbar_wait(c.bar(B_FULL_WV), 0, kWaitLimit / 8);
+        (void)mbar_wait(c.bar(B_FULL_QK), 0, kWaitLimit / 8);
     }
     if (warp == 0) {
         __syncwarp();
@@ -666,7 +657,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     using namespace tc;
     Maps m;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    if (!make_map(&m.v, v, BF, 2, B, T, H, 128, 64, false) ||
+    if (!make_map(&m.q, q, BF, 2, B, T, H, kDK, 32, false) || !make_map(&m.k, k, BF, 2, B, T, H, kDK, 32, false) ||
+        !make_map(&m.v, v, BF, 2, B, T, H, 128, 64, false) ||
         !make_map(&m.alpha, alpha, F32, 4, B, T, H, kDK, 32, true) ||
         !make_map(&m.b, b, F32, 4, B, T, H, kDK, 32, true) || !make_map(&m.w, w, F32, 4, B, T, H, 128, 32, true))
         return cudaErrorInvalidValue;
@@ -677,9 +669,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
         attr_set = true;
     }
     const unsigned grid = 2u * (unsigned)B * (unsigned)H;
-    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(m, static_cast<const __nv_bfloat16 *>(q),
-                                                            static_cast<const __nv_bfloat16 *>(k), S0,
-                                                            static_cast<__nv_bfloat16 *>(o), S_T, T, H);
+    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(m, S0, static_cast<__nv_bfloat16 *>(o), S_T, T, H);
     return cudaGetLastError();
 }
 
