@@ -70,7 +70,7 @@ constexpr long long kWaitLimit = 4000000000ll;   // ~2 s of SM cycles per wait
 //   UH  R_hi, later U_hi, as [j][t]                           2 atoms x 8 KB (t = token)
 //   UL  R_lo, later U_lo, as [j][t]                           2 atoms x 8 KB
 //   ZW  w as [t][j] (FP32, same swizzle; TMA destination)     2 atoms x 8 KB
-//   RV  v as [t][j] (BF16, unswizzled; TMA destination)
+//   RV  v as [t][j] (BF16, same swizzle; TMA destination)
 //   QK  q, k of the next chunk as BF16 [a][t][32] (a = channel block of 32), 16 KB
 //       each: TMA destinations, read by the gate prep; the same bytes then hold
 //   AS  A, then T in place (FP32 [64][66]);  XS block products (FP32 [32][34])
@@ -353,6 +353,11 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                     tma_load_4d(c.sa + OFF_KS + a * 16384, &maps.alpha, 32 * a, h, ck * kC, bidx, fb);
                     tma_load_4d(c.sa + OFF_X1 + a * 16384, &maps.b, 32 * a, h, ck * kC, bidx, fb);
                 }
+                if (ck + 1 < nchunks)       // the next chunk's tiles into L2 while this one is processed
+                    for (int a = 0; a < 4; ++a) {
+                        tma_prefetch_4d(&maps.alpha, 32 * a, h, (ck + 1) * kC, bidx);
+                        tma_prefetch_4d(&maps.b, 32 * a, h, (ck + 1) * kC, bidx);
+                    }
             }
         } else if (lane == 2) {     // q, k -> QK (over the inversion scratch of the previous chunk)
             for (int ck = 0; ck < nchunks; ++ck) {
@@ -363,6 +368,11 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                     tma_load_4d(c.sa + OFF_QK + a * 4096, &maps.q, 32 * a, h, ck * kC, bidx, fb);
                     tma_load_4d(c.sa + OFF_QK + 16384 + a * 4096, &maps.k, 32 * a, h, ck * kC, bidx, fb);
                 }
+                if (ck + 1 < nchunks)
+                    for (int a = 0; a < 4; ++a) {
+                        tma_prefetch_4d(&maps.q, 32 * a, h, (ck + 1) * kC, bidx);
+                        tma_prefetch_4d(&maps.k, 32 * a, h, (ck + 1) * kC, bidx);
+                    }
             }
         } else if (lane == 1) {     // w -> ZW, v -> RV
             for (int ck = 0; ck < nchunks; ++ck) {
@@ -372,6 +382,10 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                 for (int a = 0; a < 2; ++a)
                     tma_load_4d(c.sa + OFF_ZW + a * 8192, &maps.w, col0 + 32 * a, h, ck * kC, bidx, fb);
                 tma_load_4d(c.sa + OFF_RV, &maps.v, col0, h, ck * kC, bidx, fb);
+                if (ck + 1 < nchunks) {
+                    for (int a = 0; a < 2; ++a) tma_prefetch_4d(&maps.w, col0 + 32 * a, h, (ck + 1) * kC, bidx);
+                    tma_prefetch_4d(&maps.v, col0, h, (ck + 1) * kC, bidx);
+                }
             }
         }
         __syncwarp();
@@ -518,15 +532,20 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                 float x[32];
                 tmem_ld32(tlane + TM_X + 32 * sh, x);
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int cc = 8 * sh + m;                 // 16-byte chunk (4 columns) among 16 per row
-                    const uint32_t zo = (cc >> 3) * 8192u + srow * 128 + (((cc & 7) ^ (srow & 7)) << 4);
-                    const float4 w = at4(c, OFF_ZW + zo);
-                    const uint2 vb = *reinterpret_cast<const uint2 *>(c.sm + OFF_RV + srow * 128 + cc * 8);
-                    x[4 * m] = w.x * bf_lo(vb.x) - x[4 * m];
-                    x[4 * m + 1] = w.y * bf_hi(vb.x) - x[4 * m + 1];
-                    x[4 * m + 2] = w.z * bf_lo(vb.y) - x[4 * m + 2];
-                    x[4 * m + 3] = w.w * bf_hi(vb.y) - x[4 * m + 3];
+                for (int p = 0; p < 4; ++p) {                  // columns 32 sh + 8 p .. + 7
+                    const uint32_t sw7 = srow & 7;
+                    const uint4 vb = *reinterpret_cast<const uint4 *>(c.sm + OFF_RV + srow * 128 + (((4 * sh + p) ^ sw7) << 4));
+                    const float4 w0 = at4(c, OFF_ZW + sh * 8192u + srow * 128 + (((2 * p) ^ sw7) << 4));
+                    const float4 w1 = at4(c, OFF_ZW + sh * 8192u + srow * 128 + (((2 * p + 1) ^ sw7) << 4));
+                    float *xp = x + 8 * p;
+                    xp[0] = w0.x * bf_lo(vb.x) - xp[0];
+                    xp[1] = w0.y * bf_hi(vb.x) - xp[1];
+                    xp[2] = w0.z * bf_lo(vb.y) - xp[2];
+                    xp[3] = w0.w * bf_hi(vb.y) - xp[3];
+                    xp[4] = w1.x * bf_lo(vb.z) - xp[4];
+                    xp[5] = w1.y * bf_hi(vb.z) - xp[5];
+                    xp[6] = w1.z * bf_lo(vb.w) - xp[6];
+                    xp[7] = w1.w * bf_hi(vb.w) - xp[7];
                 }
                 store_split_jt(c, x, srow, sh);
             }
@@ -658,7 +677,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     Maps m;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     if (!make_map(&m.q, q, BF, 2, B, T, H, kDK, 32, false) || !make_map(&m.k, k, BF, 2, B, T, H, kDK, 32, false) ||
-        !make_map(&m.v, v, BF, 2, B, T, H, 128, 64, false) ||
+        !make_map(&m.v, v, BF, 2, B, T, H, 128, 64, true) ||
         !make_map(&m.alpha, alpha, F32, 4, B, T, H, kDK, 32, true) ||
         !make_map(&m.b, b, F32, 4, B, T, H, kDK, 32, true) || !make_map(&m.w, w, F32, 4, B, T, H, 128, 32, true))
         return cudaErrorInvalidValue;
