@@ -166,21 +166,28 @@ __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 
 // Gate prep: cumulative decay as running FP32 products (exp of the cumulative
 // log-decay up to rounding); Etil, Qtil into X1, Ktil into KS (rows 0-63) and
 // its transpose into Tensor Memory.  Padding tokens (t >= n): zero b from the
-// TMA bounds fill, zero q, k, alpha forced to 1.
-__device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, uint32_t kt_col, int kb, int qd, int kh,
-                                     int lane, int n) {
+// TMA bounds fill, zero q, k, alpha forced to 1.  prep_decay forms each
+// thread's product of alpha over its 32 tokens (needs only alpha).
+__device__ __forceinline__ void prep_decay(const Ctx &c, int qd, int kh, int lane, int n) {
     const int i = 32 * qd + lane;
     const Swz sw((i & 31) * 4u);
     const uint32_t rbase = (i >> 5) * 16384u + kh * 32 * 128;
-    float *part = fptr(c, OFF_PART);
     float pa = 1.f;
 #pragma unroll
     for (int tt = 0; tt < 32; ++tt) {
         const float a = at(c, OFF_KS + rbase + tt * 128 + sw.o[tt & 7]);
         pa *= (32 * kh + tt < n) ? clamp_alpha(a) : 1.f;
     }
-    part[kh * 128 + i] = pa;
-    named_bar(kBarK, kGroup);
+    fptr(c, OFF_PART)[kh * 128 + i] = pa;
+}
+
+// Gate prep proper (after prep_decay and a group barrier).
+__device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, uint32_t kt_col, int kb, int qd, int kh,
+                                     int lane, int n) {
+    const int i = 32 * qd + lane;
+    const Swz sw((i & 31) * 4u);
+    const uint32_t rbase = (i >> 5) * 16384u + kh * 32 * 128;
+    const float *part = fptr(c, OFF_PART);
     const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(c.sm + OFF_QK) + (i >> 5) * 2048 + kh * 1024 + (i & 31);
     const __nv_bfloat16 *ks = qs + 8192;
     const float p0 = part[i], p1 = part[128 + i];
@@ -214,50 +221,26 @@ __device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, uint32_t kt_c
 }
 
 // T = (I + A)^{-1} in FP32, in place in AS (A strictly lower, zero above the
-// diagonal).  16 x 16 diagonal blocks by forward substitution (right-looking,
-// so each step's dependency is one FMA); T_10 = -D_1 A_10 D_0 and
-// T_32 = -D_3 A_32 D_2; then T_BA = -T_BB A_BA T_AA for the lower-left 32 x 32.
+// diagonal).  The two 32 x 32 diagonal blocks T_AA, T_BB by forward
+// substitution (right-looking: column j of a block per thread, each step's
+// dependency one FMA); then T_BA = -T_BB A_BA T_AA for the lower-left block.
 __device__ __forceinline__ void invert(const Ctx &c, int ktid) {
     float *As = fptr(c, OFF_AS);
     float *Xs = fptr(c, OFF_XS);
-    // Column j of D_b: x = e_j, then x_i -= A_il x_l for l < i (x_l final once reached).
-    float x[16];
-    const int b = ktid >> 4, j = ktid & 15, base = 16 * b;
     if (ktid < 64) {
+        const int base = 32 * (ktid >> 5), j = ktid & 31;
+        float x[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = (i == j) ? 1.f : 0.f;
+        for (int i = 0; i < 32; ++i) x[i] = (i == j) ? 1.f : 0.f;
 #pragma unroll
-        for (int l = 0; l < 15; ++l) {
+        for (int l = 0; l < 31; ++l) {
+            const float xl = x[l];
 #pragma unroll
-            for (int i = l + 1; i < 16; ++i) x[i] = fmaf(-As[(base + i) * LDA + base + l], x[l], x[i]);
+            for (int i = l + 1; i < 32; ++i) x[i] = fmaf(-As[(base + i) * LDA + base + l], xl, x[i]);
         }
-    }
-    named_bar(kBarK, kGroup);
-    if (ktid < 64) {
+        __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) As[(base + i) * LDA + base + j] = x[i];
-    }
-    named_bar(kBarK, kGroup);
-    // X = A_{a,a-1} D_{a-1}, a = 1, 3
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-        const int e = ktid + kGroup * m, blk = e >> 8, i = (e >> 4) & 15, jj = e & 15;
-        const int a = blk ? 3 : 1, bb = a - 1;
-        float s = 0.f;
-#pragma unroll
-        for (int l = 0; l < 16; ++l) s = fmaf(As[(16 * a + i) * LDA + 16 * bb + l], As[(16 * bb + l) * LDA + 16 * bb + jj], s);
-        Xs[(blk * 16 + i) * LDX + jj] = s;
-    }
-    named_bar(kBarK, kGroup);
-    // T_{a,a-1} = -D_a X
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-        const int e = ktid + kGroup * m, blk = e >> 8, i = (e >> 4) & 15, jj = e & 15;
-        const int a = blk ? 3 : 1, bb = a - 1;
-        float s = 0.f;
-#pragma unroll
-        for (int l = 0; l < 16; ++l) s = fmaf(As[(16 * a + i) * LDA + 16 * a + l], Xs[(blk * 16 + l) * LDX + jj], s);
-        As[(16 * a + i) * LDA + 16 * bb + jj] = -s;
+        for (int i = 0; i < 32; ++i) As[(base + i) * LDA + base + j] = x[i];
     }
     named_bar(kBarK, kGroup);
     // Y = A_BA T_AA (32 x 32), 2 x 2 outputs per thread
@@ -453,7 +436,9 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
         for (int ck = 0; ck < nchunks; ++ck) {
             const uint32_t ph = ck & 1;
             const int t0 = ck * kC, n = min(kC, T - t0);
-            if (!group_wait(c, B_FULL_AB, ph, el, kBarK) || !group_wait(c, B_FULL_QK, ph, el, kBarK)) break;
+            if (!group_wait(c, B_FULL_AB, ph, el, kBarK)) break;
+            prep_decay(c, qd, kh, lane, n);
+            if (!group_wait(c, B_FULL_QK, ph, el, kBarK)) break;
             if (ck >= 2 && !group_wait(c, ph ? B_KT_FREE1 : B_KT_FREE0, ((ck - 2) >> 1) & 1, el, kBarK)) break;
             prep(c, tlane, TM_KT + 64 * ph, ph, qd, kh, lane, n);
             tmem_wait_st();
