@@ -32,13 +32,17 @@
 //
 // Organisation: one CTA per (batch, head, 64-column half of d_v), 18 warps in
 // four roles that run concurrently and hand work over through mbarriers:
-//   warp 0      TMA producer (alpha, b into their operand tiles; q, k staged
-//               as BF16 over the inversion scratch; w, v staging)
+//   warp 0      TMA producer (alpha, b into their operand tiles; q, k into a
+//               BF16 staging tile; L2 prefetch of the next chunk's tiles)
 //   warp 1      MMA issuer (one thread, every tcgen05 instruction)
 //   warps 2-9   key side: gate prep, Gram epilogue, blocked inversion of (I + A)
-//   warps 10-17 state side: R, U and state/output epilogues; owns the FP32 state
+//   warps 10-17 state side: R, U and state/output epilogues (w, v read
+//               straight from global memory into registers)
 // The key side of chunk c+1 runs while the state chain of chunk c runs; the
 // key factor Ktil^T and [T; P] are double-buffered in Tensor Memory for that.
+// The FP32 state itself lives in Tensor Memory: the state-update MMA
+// accumulates Ktil^T U onto it, the epilogue scales it by the chunk decay and
+// writes the TF32 copy that the next chunk's MMAs read.
 // Shared-memory MMA operands are K-major with the 128-byte swizzle; operands
 // needed transposed (Ktil^T, [T; P]) are read from Tensor Memory as operand A.
 #include <cudaTypedefs.h>
@@ -69,46 +73,41 @@ constexpr long long kWaitLimit = 4000000000ll;   // ~2 s of SM cycles per wait
 //   KS  rows 0-63 Ktil[s][i], rows 64-127 S[i][j] as [j][i]    4 atoms x 16 KB
 //   UH  R_hi, later U_hi, as [j][t]                           2 atoms x 8 KB (t = token)
 //   UL  R_lo, later U_lo, as [j][t]                           2 atoms x 8 KB
-//   ZW  w as [t][j] (FP32, same swizzle; TMA destination)     2 atoms x 8 KB
-//   RV  v as [t][j] (BF16, same swizzle; TMA destination)
-//   QK  q, k of the next chunk as BF16 [a][t][32] (a = channel block of 32), 16 KB
-//       each: TMA destinations, read by the gate prep; the same bytes then hold
+//   QK  q, k as BF16 [a][t][32] (a = channel block of 32), 16 KB each: TMA
+//       destinations, read by the gate prep
 //   AS  A, then T in place (FP32 [64][66]);  XS block products (FP32 [32][34])
 constexpr uint32_t OFF_X1 = 0;
 constexpr uint32_t OFF_KS = OFF_X1 + 65536;
 constexpr uint32_t OFF_UH = OFF_KS + 65536;
 constexpr uint32_t OFF_UL = OFF_UH + 16384;
-constexpr uint32_t OFF_ZW = OFF_UL + 16384;
-constexpr uint32_t OFF_RV = OFF_ZW + 16384;
-constexpr uint32_t OFF_GN = OFF_RV + 8192;             // float[2][128] decay over the chunk (by buffer)
+constexpr uint32_t OFF_GN = OFF_UL + 16384;            // float[2][128] decay over the chunk (by buffer)
 constexpr uint32_t OFF_PART = OFF_GN + 1024;           // float[2][128] half-chunk decay products
 constexpr uint32_t OFF_BAR = OFF_PART + 1024;          // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;           // tmem base, abort flag
 constexpr int LDA = 66, LDX = 34;
-constexpr uint32_t OFF_QK = OFF_MISC + 768;            // 1024-aligned
-constexpr uint32_t OFF_AS = OFF_QK;
+constexpr uint32_t OFF_QK = (OFF_MISC + 16 + 1023) / 1024 * 1024;
+constexpr uint32_t OFF_AS = OFF_QK + 32768;
 constexpr uint32_t OFF_XS = OFF_AS + 64 * LDA * 4;
-constexpr uint32_t SMEM_USED = OFF_QK + 32768;
+constexpr uint32_t SMEM_USED = OFF_XS + 32 * LDX * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
-static_assert(OFF_QK % 1024 == 0 && OFF_XS + 32 * LDX * 4 <= SMEM_USED, "shared-memory map");
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 
 // Tensor Memory columns (512 allocated).
 constexpr uint32_t TM_G = 0;        // Gram: lanes 0-63 A, lanes 64-127 P                 (64 cols)
 constexpr uint32_t TM_X = 64;       // [Etil;Qtil] S, then + P U: lanes 64-127 -> O       (64 cols)
-constexpr uint32_t TM_UD = 128;     // U = T R (lanes 0-63), then Ktil^T U                (64 cols)
+constexpr uint32_t TM_U = 128;      // U = T R (lanes 0-63)                                (64 cols)
 constexpr uint32_t TM_KT = 192;     // 2 buffers: A operand Ktil^T, lane i, column s      (2 x 64 cols)
 constexpr uint32_t TM_TP = 320;     // 2 buffers: A operand [T; P], lane t, column s      (2 x 64 cols)
+constexpr uint32_t TM_S = 448;      // FP32 state S[i][j], lane i, column j               (64 cols)
 constexpr uint32_t TM_COLS = 512;
 
 enum {
-    B_FULL_AB = 0, B_FULL_WV, B_FULL_QK, B_X1_FREE, B_WV_FREE, B_KPREP, B_G_FULL, B_TP_READY, B_S_READY,
-    B_X_FULL, B_R_READY, B_U_FULL, B_U_READY, B_D_FULL, B_KT_FREE0, B_KT_FREE1, NBARS
+    B_FULL_AB = 0, B_FULL_QK, B_X1_FREE, B_KPREP, B_G_FULL, B_DIAG_DONE, B_TP_READY, B_S_READY,
+    B_X_FULL, B_R_READY, B_U_FULL, B_U_READY, B_D_FULL, B_O_FULL, B_KT_FREE0, B_KT_FREE1, NBARS
 };
 
 constexpr uint32_t TX_AB = 8 * 8192;
 constexpr uint32_t TX_QK = 8 * 4096;
-constexpr uint32_t TX_WV = 2 * 8192 + 8192;
 
 struct Maps {
     CUtensorMap q, k, v, alpha, b, w;
@@ -221,12 +220,12 @@ __device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, uint32_t kt_c
 }
 
 // T = (I + A)^{-1} in FP32, in place in AS (A strictly lower, zero above the
-// diagonal).  The two 32 x 32 diagonal blocks T_AA, T_BB by forward
-// substitution (right-looking: column j of a block per thread, each step's
-// dependency one FMA); then T_BA = -T_BB A_BA T_AA for the lower-left block.
-__device__ __forceinline__ void invert(const Ctx &c, int ktid) {
+// diagonal), in two parts.  invert_diag (key side): the 32 x 32 diagonal
+// blocks T_AA, T_BB by forward substitution (right-looking: column j of a block
+// per thread, each step's dependency one FMA).  invert_offdiag (state side,
+// which is otherwise waiting for T): T_BA = -T_BB A_BA T_AA.
+__device__ __forceinline__ void invert_diag(const Ctx &c, int ktid) {
     float *As = fptr(c, OFF_AS);
-    float *Xs = fptr(c, OFF_XS);
     if (ktid < 64) {
         const int base = 32 * (ktid >> 5), j = ktid & 31;
         float x[32];
@@ -242,10 +241,14 @@ __device__ __forceinline__ void invert(const Ctx &c, int ktid) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) As[(base + i) * LDA + base + j] = x[i];
     }
-    named_bar(kBarK, kGroup);
+}
+// gtid: thread index within the 256-thread group that runs this; bar_id: its barrier.
+__device__ __forceinline__ void invert_offdiag(const Ctx &c, int gtid, uint32_t bar_id) {
+    float *As = fptr(c, OFF_AS);
+    float *Xs = fptr(c, OFF_XS);
     // Y = A_BA T_AA (32 x 32), 2 x 2 outputs per thread
     {
-        const int i = 2 * (ktid >> 4), jj = 2 * (ktid & 15);
+        const int i = 2 * (gtid >> 4), jj = 2 * (gtid & 15);
         float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 8
         for (int l = 0; l < 32; ++l) {
@@ -257,10 +260,10 @@ __device__ __forceinline__ void invert(const Ctx &c, int ktid) {
         *reinterpret_cast<float2 *>(Xs + i * LDX + jj) = make_float2(y00, y01);
         *reinterpret_cast<float2 *>(Xs + (i + 1) * LDX + jj) = make_float2(y10, y11);
     }
-    named_bar(kBarK, kGroup);
+    named_bar(bar_id, kGroup);
     // T_BA = -T_BB Y
     {
-        const int i = 2 * (ktid >> 4), jj = 2 * (ktid & 15);
+        const int i = 2 * (gtid >> 4), jj = 2 * (gtid & 15);
         float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 8
         for (int l = 0; l < 32; ++l) {
@@ -272,7 +275,7 @@ __device__ __forceinline__ void invert(const Ctx &c, int ktid) {
         *reinterpret_cast<float2 *>(As + (32 + i) * LDA + jj) = make_float2(-y00, -y01);
         *reinterpret_cast<float2 *>(As + (33 + i) * LDA + jj) = make_float2(-y10, -y11);
     }
-    named_bar(kBarK, kGroup);
+    named_bar(bar_id, kGroup);
 }
 
 // Split 32 values into TF32 hi + lo parts and store both into the [j][t] tiles
@@ -291,7 +294,8 @@ __device__ __forceinline__ void store_split_jt(const Ctx &c, const float (&x)[32
 
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
-chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat16 *__restrict__ o, float *S_T,
+chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
+                const __nv_bfloat16 *__restrict__ vg, const float *S0, __nv_bfloat16 *__restrict__ o, float *S_T,
                 int T, int H) {
     extern __shared__ uint8_t smem_raw[];
     Ctx c;
@@ -336,15 +340,18 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                     tma_load_4d(c.sa + OFF_KS + a * 16384, &maps.alpha, 32 * a, h, ck * kC, bidx, fb);
                     tma_load_4d(c.sa + OFF_X1 + a * 16384, &maps.b, 32 * a, h, ck * kC, bidx, fb);
                 }
-                if (ck + 1 < nchunks)       // the next chunk's tiles into L2 while this one is processed
+                if (ck + 1 < nchunks) {     // the next chunk's tiles into L2 while this one is processed
                     for (int a = 0; a < 4; ++a) {
                         tma_prefetch_4d(&maps.alpha, 32 * a, h, (ck + 1) * kC, bidx);
                         tma_prefetch_4d(&maps.b, 32 * a, h, (ck + 1) * kC, bidx);
                     }
+                    for (int a = 0; a < 2; ++a) tma_prefetch_4d(&maps.w, col0 + 32 * a, h, (ck + 1) * kC, bidx);
+                    tma_prefetch_4d(&maps.v, col0, h, (ck + 1) * kC, bidx);
+                }
             }
-        } else if (lane == 2) {     // q, k -> QK (over the inversion scratch of the previous chunk)
+        } else if (lane == 1) {     // q, k -> QK once the gate prep has consumed the previous chunk's
             for (int ck = 0; ck < nchunks; ++ck) {
-                if (ck > 0 && !solo_wait(c, B_TP_READY, (ck - 1) & 1)) break;
+                if (ck > 0 && !solo_wait(c, B_KPREP, (ck - 1) & 1)) break;
                 const uint32_t fb = c.bar(B_FULL_QK);
                 mbar_expect_tx(fb, TX_QK);
                 for (int a = 0; a < 4; ++a) {
@@ -356,19 +363,6 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                         tma_prefetch_4d(&maps.q, 32 * a, h, (ck + 1) * kC, bidx);
                         tma_prefetch_4d(&maps.k, 32 * a, h, (ck + 1) * kC, bidx);
                     }
-            }
-        } else if (lane == 1) {     // w -> ZW, v -> RV
-            for (int ck = 0; ck < nchunks; ++ck) {
-                if (ck > 0 && !solo_wait(c, B_WV_FREE, (ck - 1) & 1)) break;
-                const uint32_t fb = c.bar(B_FULL_WV);
-                mbar_expect_tx(fb, TX_WV);
-                for (int a = 0; a < 2; ++a)
-                    tma_load_4d(c.sa + OFF_ZW + a * 8192, &maps.w, col0 + 32 * a, h, ck * kC, bidx, fb);
-                tma_load_4d(c.sa + OFF_RV, &maps.v, col0, h, ck * kC, bidx, fb);
-                if (ck + 1 < nchunks) {
-                    for (int a = 0; a < 2; ++a) tma_prefetch_4d(&maps.w, col0 + 32 * a, h, (ck + 1) * kC, bidx);
-                    tma_prefetch_4d(&maps.v, col0, h, (ck + 1) * kC, bidx);
-                }
             }
         }
         __syncwarp();
@@ -408,22 +402,27 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                    mma_tf32_ts(tmem + TM_UD, tp + 8 * kk, dUH + koff, id, kk > 0);
-                    mma_tf32_ts(tmem + TM_UD, tp + 8 * kk, dUL + koff, id, 1);
+                    mma_tf32_ts(tmem + TM_U, tp + 8 * kk, dUH + koff, id, kk > 0);
+                    mma_tf32_ts(tmem + TM_U, tp + 8 * kk, dUL + koff, id, 1);
                 }
                 mma_commit(c.bar(B_U_FULL));
-                // Ktil^T (U_hi + U_lo) -> TM_UD;  P U_hi accumulated onto TM_X
+                // S + Ktil^T (U_hi + U_lo) accumulated onto the state;  then P U_hi onto TM_X
                 if (!solo_wait(c, B_U_READY, ph)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                    mma_tf32_ts(tmem + TM_UD, kt + 8 * kk, dUH + koff, id, kk > 0);
-                    mma_tf32_ts(tmem + TM_UD, kt + 8 * kk, dUL + koff, id, 1);
-                    mma_tf32_ts(tmem + TM_X, tp + 8 * kk, dUH + koff, id, 1);
+                    mma_tf32_ts(tmem + TM_S, kt + 8 * kk, dUH + koff, id, 1);
+                    mma_tf32_ts(tmem + TM_S, kt + 8 * kk, dUL + koff, id, 1);
                 }
                 mma_commit(c.bar(B_D_FULL));
-                mma_commit(c.bar(ph ? B_KT_FREE1 : B_KT_FREE0));
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                    mma_tf32_ts(tmem + TM_X, tp + 8 * kk, dUH + koff, id, 1);
+                }
+                mma_commit(c.bar(B_O_FULL));
+                mma_commit(c.bar(ph ? B_KT_FREE1 : B_KT_FREE0));     // Ktil^T and [T; P] of this parity
             }
         }
         __syncwarp();
@@ -446,8 +445,10 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             tc_fence_before();
             named_bar(kBarK, kGroup);
             if (el) mbar_arrive(c.bar(B_KPREP));
-            // Gram epilogue: A (rows 0-63, strictly lower) -> AS; P (rows 64-127) -> [T; P] operand
+            // Gram epilogue: A (rows 0-63, strictly lower) -> AS; P (rows 64-127) -> [T; P] operand.
+            // AS is free once the state side has copied out the previous chunk's T.
             if (!group_wait(c, B_G_FULL, ph, el, kBarK)) break;
+            if (ck >= 1 && !group_wait(c, B_TP_READY, (ck - 1) & 1, el, kBarK)) break;
             tc_fence_after();
             {
                 float g[32];
@@ -468,32 +469,23 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                 }
             }
             named_bar(kBarK, kGroup);
-            invert(c, ktid);
-            if (srow < 64) {        // T rows -> [T; P] operand
-                float tv[32];
-                const float *As = fptr(c, OFF_AS);
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int s = 32 * kh + jj;
-                    tv[jj] = (s <= srow) ? to_tf32(As[srow * LDA + s]) : 0.f;
-                }
-                tmem_st32_nowait(tlane + TM_TP + 64 * ph + 32 * kh, tv);
-            }
+            invert_diag(c, ktid);
             tmem_wait_st();
             tc_fence_before();
             named_bar(kBarK, kGroup);
-            if (el) mbar_arrive(c.bar(B_TP_READY));
+            if (el) mbar_arrive(c.bar(B_DIAG_DONE));
         }
     } else {
         // ------------------------------------------------ state side
         const int stid = tid - 320, qd = warp & 3, sh = (warp - 10) >> 2;
         const int srow = 32 * qd + lane;
         const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);
+        const uint32_t ts = tlane + TM_S + 32 * sh;        // this thread's state row, 32 columns
         const bool el = stid == 0;
         const Swz ssw((srow & 31) * 4u);
         const uint32_t sbase = OFF_KS + (srow >> 5) * 16384u + (64 + 32 * sh) * 128;   // S rows of KS
-        float S[32];
-        {
+        {   // S0 -> Tensor Memory and its TF32 copy
+            float S[32];
             const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 32 * sh;
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
@@ -502,26 +494,47 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j) at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(S[j]);
+            tmem_st32_nowait(ts, S);
+            tmem_wait_st();
         }
         fence_proxy_async_smem();
+        tc_fence_before();
         named_bar(kBarS, kGroup);
         if (el) mbar_arrive(c.bar(B_S_READY));
         bool done_ok = true;
         for (int ck = 0; ck < nchunks; ++ck) {
             const uint32_t ph = ck & 1;
             const int t0 = ck * kC, n = min(kC, T - t0);
+            // w, v of this thread's token (lanes 0-63) and columns, straight into registers;
+            // the loads complete while the MMA below runs.  Padding tokens read as zero.
+            float4 wr[8];
+            uint4 vr[4];
+            if (srow < 64) {
+                if (srow < n) {
+                    const size_t row = (((size_t)bidx * T + t0 + srow) * H + h) * 128 + col0 + 32 * sh;
+                    const float4 *wp = reinterpret_cast<const float4 *>(wg + row);
+                    const uint4 *vp = reinterpret_cast<const uint4 *>(vg + row);
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) wr[m] = __ldg(wp + m);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) vr[m] = __ldg(vp + m);
+                } else {
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) wr[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) vr[m] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
             // R = w*v - Etil S (lanes 0-63) -> R_hi, R_lo
-            if (!group_wait(c, B_X_FULL, ph, el, kBarS) || !group_wait(c, B_FULL_WV, ph, el, kBarS)) { done_ok = false; break; }
+            if (!group_wait(c, B_X_FULL, ph, el, kBarS)) { done_ok = false; break; }
             tc_fence_after();
             if (srow < 64) {
                 float x[32];
                 tmem_ld32(tlane + TM_X + 32 * sh, x);
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {                  // columns 32 sh + 8 p .. + 7
-                    const uint32_t sw7 = srow & 7;
-                    const uint4 vb = *reinterpret_cast<const uint4 *>(c.sm + OFF_RV + srow * 128 + (((4 * sh + p) ^ sw7) << 4));
-                    const float4 w0 = at4(c, OFF_ZW + sh * 8192u + srow * 128 + (((2 * p) ^ sw7) << 4));
-                    const float4 w1 = at4(c, OFF_ZW + sh * 8192u + srow * 128 + (((2 * p + 1) ^ sw7) << 4));
+                    const uint4 vb = vr[p];
+                    const float4 w0 = wr[2 * p], w1 = wr[2 * p + 1];
                     float *xp = x + 8 * p;
                     xp[0] = w0.x * bf_lo(vb.x) - xp[0];
                     xp[1] = w0.y * bf_hi(vb.x) - xp[1];
@@ -537,32 +550,54 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarS, kGroup);
-            if (el) { mbar_arrive(c.bar(B_R_READY)); mbar_arrive(c.bar(B_WV_FREE)); }
+            if (el) mbar_arrive(c.bar(B_R_READY));
+            // finish T = (I + A)^{-1} and copy it, TF32, into rows 0-63 of the [T; P] operand
+            if (!group_wait(c, B_DIAG_DONE, ph, el, kBarS)) { done_ok = false; break; }
+            tc_fence_after();
+            invert_offdiag(c, stid, kBarS);
+            if (srow < 64) {
+                float tv[32];
+                const float *As = fptr(c, OFF_AS);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int s = 32 * sh + jj;
+                    tv[jj] = (s <= srow) ? to_tf32(As[srow * LDA + s]) : 0.f;
+                }
+                tmem_st32_nowait(tlane + TM_TP + 64 * ph + 32 * sh, tv);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar(kBarS, kGroup);
+            if (el) mbar_arrive(c.bar(B_TP_READY));
             // U -> U_hi, U_lo
             if (!group_wait(c, B_U_FULL, ph, el, kBarS)) { done_ok = false; break; }
             tc_fence_after();
             if (srow < 64) {
                 float u[32];
-                tmem_ld32(tlane + TM_UD + 32 * sh, u);
+                tmem_ld32(tlane + TM_U + 32 * sh, u);
                 store_split_jt(c, u, srow, sh);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarS, kGroup);
             if (el) mbar_arrive(c.bar(B_U_READY));
-            // state S <- gamma_n (S + Ktil^T U) and its TF32 copy; outputs (lanes 64-127 of TM_X)
+            // state S <- gamma_n (S + Ktil^T U), in Tensor Memory, and its TF32 copy
             if (!group_wait(c, B_D_FULL, ph, el, kBarS)) { done_ok = false; break; }
             tc_fence_after();
             {
                 float d[32];
-                tmem_ld32(tlane + TM_UD + 32 * sh, d);
+                tmem_ld32(ts, d);
                 const float gn = fptr(c, OFF_GN)[ph * 128 + srow];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    S[j] = gn * (S[j] + d[j]);
-                    at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(S[j]);
+                    d[j] *= gn;
+                    at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(d[j]);
                 }
+                tmem_st32_nowait(ts, d);
             }
+            // outputs: lanes 64-127 of TM_X
+            if (!group_wait(c, B_O_FULL, ph, el, kBarS)) { done_ok = false; break; }
+            tc_fence_after();
             if (srow >= 64) {
                 float v[32];
                 tmem_ld32(tlane + TM_X + 32 * sh, v);
@@ -584,12 +619,15 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
                     }
                 }
             }
+            tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarS, kGroup);
             if (el) mbar_arrive(c.bar(B_S_READY));
         }
         if (done_ok && *c.abort_flag == 0 && S_T) {
+            float S[32];
+            tmem_ld32(ts, S);
             const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 32 * sh;
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
@@ -603,7 +641,6 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *S0, __nv_bfloat1
     __syncthreads();
     if (tid == 0 && *c.abort_flag) {
         (void)mbar_wait(c.bar(B_FULL_AB), 0, kWaitLimit / 8);
-        (void)mbar_wait(c.bar(B_FULL_WV), 0, kWaitLimit / 8);
         (void)mbar_wait(c.bar(B_FULL_QK), 0, kWaitLimit / 8);
     }
     if (warp == 0) {
@@ -673,7 +710,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
         attr_set = true;
     }
     const unsigned grid = 2u * (unsigned)B * (unsigned)H;
-    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(m, S0, static_cast<__nv_bfloat16 *>(o), S_T, T, H);
+    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(m, w, static_cast<const __nv_bfloat16 *>(v), S0,
+                                                            static_cast<__nv_bfloat16 *>(o), S_T, T, H);
     return cudaGetLastError();
 }
 
