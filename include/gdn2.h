@@ -51,7 +51,7 @@ extern "C" {
 typedef enum {
     GDN2_OK = 0,
     GDN2_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative size, aliasing not allowed */
-    GDN2_ERR_UNSUPPORTED = 2,  /* head size or dtype this build does not implement */
+    GDN2_ERR_UNSUPPORTED = 2,  /* head size or dtype the library does not implement */
     GDN2_ERR_CUDA = 3          /* a CUDA runtime call or kernel launch failed */
 } gdn2_status;
 
