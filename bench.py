@@ -79,6 +79,30 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(x, torch, dist, world, device):
+    """The largest of every rank's ``x`` (one all-reduce; every rank calls it
+    in the same order).  With one rank, ``x`` itself."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sync_ranks(torch, dist, world):
+    """Device idle, then all ranks meet (brackets every timed region)."""
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+
+def job_tokens_per_s(B, T, world, ms):
+    """Whole-job throughput: every rank runs one B x T replica per step, so the
+    job processes B*T*world tokens in the slowest rank's time."""
+    return B * T * world / (ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
 def oracle_tokens_per_s(budget_s=12.0, max_heads=None):
@@ -212,9 +236,7 @@ def run_prefill(args, torch, dist, g, world, rank, dev, stream):
 
     for _ in range(args.warmup):
         step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    sync_ranks(torch, dist, world)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # nvidia-smi samples every 100 ms: keep the GPU busy with the same step for
     # about a second before the timed region so the samples see it under load.
@@ -225,17 +247,13 @@ def run_prefill(args, torch, dist, g, world, rank, dev, stream):
     with ClockSampler(dev.index) as clk:
         for _ in range(int(min(4000, 1.2 / per))):
             step()
+        sync_ranks(torch, dist, world)
         ev0.record(stream)
         for _ in range(args.steps):
             step()
         ev1.record(stream)
-        torch.cuda.synchronize()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        dist.barrier()
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+        sync_ranks(torch, dist, world)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), torch, dist, world, dev)
     ms_step = ms_total / args.steps
 
     # ---- e2e: pinned host buffers, copies inside the timed region
@@ -254,18 +272,14 @@ def run_prefill(args, torch, dist, g, world, rank, dev, stream):
 
     for _ in range(2):
         e2e_step()
-    torch.cuda.synchronize()
+    sync_ranks(torch, dist, world)
     e2e_steps = max(2, min(args.steps, 5))
     ev0.record(stream)
     for _ in range(e2e_steps):
         e2e_step()
     ev1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    sync_ranks(torch, dist, world)
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, torch, dist, world, dev)
     del host, o_h, S_h, d, o, ST
     torch.cuda.empty_cache()
     return ms_step, e2e_ms, h2d, d2h, clk
@@ -290,18 +304,14 @@ def run_decode(args, torch, dist, g, world, rank, dev, stream):
 
     for _ in range(max(args.warmup, 1)):
         decode_run()
-    torch.cuda.synchronize()
+    sync_ranks(torch, dist, world)
     reps = 3
     ev0.record(stream)
     for _ in range(reps):
         decode_run()
     ev1.record(stream)
-    torch.cuda.synchronize()
-    dec_ms = ev0.elapsed_time(ev1) / (reps * steps_d)
-    if world > 1:
-        t = torch.tensor([dec_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dec_ms = float(t.item())
+    sync_ranks(torch, dist, world)
+    dec_ms = max_over_ranks(ev0.elapsed_time(ev1) / (reps * steps_d), torch, dist, world, dev)
     del dd, S0d, Sd, od, views
     torch.cuda.empty_cache()
     return dec_ms
@@ -316,7 +326,7 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk):
     Bd, Hd = DECODE["B"], DECODE["H"]
     steps_d = DECODE["steps"]
     reps = 3
-    value = B * T * world / (ms_step / 1e3)
+    value = job_tokens_per_s(B, T, world, ms_step)
     hbm, hbm_src = measured_peaks()
     pre_bytes = prefill_bytes(B, T, H, dk, dv)
     pre_gbs = pre_bytes / (ms_step / 1e3) / 1e9
@@ -340,7 +350,7 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk):
                        "dtypes": "q/k/v/o bf16, alpha/b/w fp32, state fp32, fp32 accumulation",
                        "l2": "inputs (675 MB per call) larger than the 126 MB L2; no flush",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-            "e2e": {"value": _num(B * T * world / (e2e_ms / 1e3)), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": _num(job_tokens_per_s(B, T, world, e2e_ms)), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": _num(e2e_ms)},
             "roofline": {"bound": "hbm", "achieved": _num(pre_gbs), "peak": hbm, "unit": "GB/s",
                          "frac": _num(pre_gbs / hbm), "traffic": traffic.get("gdn2_chunk"),
