@@ -152,6 +152,28 @@ def test_small_full(g, dtype, T, d):
     assert rel(ST, S_ref) <= (TOL_FP32 if dtype == "fp32" else TOL_BF16_S)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("dk,dv", [(128, 64), (64, 128)])
+def test_prefill_unequal_head_sizes(g, dtype, dk, dv):
+    """d_k != d_v (the FP32 CUDA-core prefill): several chunks, ragged tail, S0."""
+    x = gi.chunk_inputs(2, 129, 2, dk, dv, dtype=dtype, seed=dk + 3 * dv, s0_std=0.05)
+    o, ST = run_chunk(g, x)
+    o_ref, S_ref = oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], x["S0"])
+    check_o(o, o_ref, dtype)
+    assert rel(ST, S_ref) <= (TOL_FP32 if dtype == "fp32" else TOL_BF16_S)
+
+
+def test_multi_wave_grid(g):
+    """More CTAs than SMs (B=12, H=16: 384 column-half CTAs on 148 SMs, about three
+    waves), ragged tail, nonzero S0: every output of every head checked, so each SM
+    runs several CTAs one after another through the same Tensor Memory."""
+    x = gi.chunk_inputs(12, 130, 16, 128, 128, dtype="bf16", seed=77, s0_std=0.05)
+    o, ST = run_chunk(g, x)
+    o_ref, S_ref = oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], x["S0"])
+    check_o(o, o_ref, "bf16")
+    assert rel(ST, S_ref) <= TOL_BF16_S
+
+
 def test_delta_identity_fp32(g):
     """b = 1, w = 1, unit keys, q = k: every output equals v (the delta rule writes the error)."""
     x = gi.chunk_inputs(1, 130, 2, 128, 128, dtype="fp32", seed=9, s0_std=0.1)
