@@ -163,6 +163,32 @@ def test_prefill_unequal_head_sizes(g, dtype, dk, dv):
     assert rel(ST, S_ref) <= (TOL_FP32 if dtype == "fp32" else TOL_BF16_S)
 
 
+def _gate_case(case, seed):
+    """B=1, T=500, H=4, d=128, BF16, S0 != 0, with the gates pushed to an edge of their range."""
+    x = gi.chunk_inputs(1, 500, 4, 128, 128, dtype="bf16", seed=seed, s0_std=0.05)
+    rng = np.random.default_rng(seed + 1000)
+    if case == "strong_decay":
+        # -ln(alpha) in [1.0, 1.2]: up to 76.8 per 64-token chunk, just inside the documented
+        # bound (78) for the tensor-core path; gamma falls to ~1e-33 within a chunk.
+        x["alpha"] = np.exp(-rng.uniform(1.0, 1.2, x["alpha"].shape)).astype(np.float32)
+    elif case == "no_decay":
+        x["alpha"] = np.ones_like(x["alpha"])
+    elif case == "erase_to_2":
+        # erase gate over [0, 2], the range of the pages' gate ablation
+        x["b"] = (2.0 * x["b"]).astype(np.float32)
+    return x
+
+
+@pytest.mark.parametrize("case", ["strong_decay", "no_decay", "erase_to_2"])
+def test_gate_edges(g, case):
+    """Every output and the final state, against the oracle, at the edges of the gate ranges."""
+    x = _gate_case(case, seed={"strong_decay": 31, "no_decay": 32, "erase_to_2": 33}[case])
+    o, ST = run_chunk(g, x)
+    o_ref, S_ref = oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], x["S0"])
+    check_o(o, o_ref, "bf16")
+    assert rel(ST, S_ref) <= TOL_BF16_S
+
+
 def test_multi_wave_grid(g):
     """More CTAs than SMs (B=12, H=16: 384 column-half CTAs on 148 SMs, about three
     waves), ragged tail, nonzero S0: every output of every head checked, so each SM
@@ -306,6 +332,25 @@ def test_decode_small(g, dtype, dk, dv):
         o_ref, S_ref = oracle.gdn2_step(*(x[n][s] for n in ("q", "k", "v", "alpha", "b", "w")), S_ref)
         check_o(o[s], o_ref, dtype)
     assert rel(S, S_ref) <= tol_s
+
+
+@pytest.mark.parametrize("case", ["strong_decay", "no_decay", "erase_to_2"])
+def test_decode_gate_edges(g, case):
+    """Decode steps at the edges of the gate ranges (as test_gate_edges), every output."""
+    x = gi.decode_inputs(8, 3, 4, 128, 128, dtype="bf16", seed=41, s0_std=0.1)
+    rng = np.random.default_rng(42)
+    if case == "strong_decay":
+        x["alpha"] = np.exp(-rng.uniform(1.0, 1.2, x["alpha"].shape)).astype(np.float32)
+    elif case == "no_decay":
+        x["alpha"] = np.ones_like(x["alpha"])
+    else:
+        x["b"] = (2.0 * x["b"]).astype(np.float32)
+    o, S = run_decode(g, x, 8)
+    S_ref = x["S0"].astype(np.float64)
+    for s in range(8):
+        o_ref, S_ref = oracle.gdn2_step(*(x[n][s] for n in ("q", "k", "v", "alpha", "b", "w")), S_ref)
+        check_o(o[s], o_ref, "bf16")
+    assert rel(S, S_ref) <= TOL_BF16_S
 
 
 def test_decode_b256_64_steps_sampled(g):
