@@ -1,0 +1,62 @@
+"""The bench's JSON line keeps its contract: every key the harness reads, with
+values derived from the timings as documented (CPU; synthetic timings)."""
+import argparse
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+class _Clocks:
+    def summary(self):
+        return {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 10}
+
+
+def _line(capsys, world=1, ms=0.5, e2e=12.0, dec=0.085):
+    args = argparse.Namespace(steps=20, warmup=5, no_cpu_baseline=True, cpu_budget=1.0)
+    bench.report(args, world, 0, ms, e2e, 604_000_000, 71_000_000, dec, _Clocks())
+    out = capsys.readouterr().out.strip().splitlines()
+    assert len(out) == 1
+    return json.loads(out[0])
+
+
+def test_keys_and_types(capsys):
+    d = _line(capsys)
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "e2e", "roofline", "gpu_launches", "clocks",
+              "cpu_baseline", "decode"):
+        assert k in d, k
+    assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["vs_baseline"] is None
+    assert d["steps"] == 20 and d["warmup"] == 5 and d["n_gpus"] == 1 and d["gpu_launches"] == 20
+    assert "workload" in d["config"]
+    for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
+        assert k in d["e2e"], k
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in d["roofline"], k
+    assert d["roofline"]["bound"] == "hbm" and d["roofline"]["unit"] == "GB/s"
+    assert d["clocks"]["sm_mhz"] == 1965.0
+
+
+def test_values_follow_the_timings(capsys):
+    d = _line(capsys, ms=0.5, e2e=12.0)
+    P = bench.PREFILL
+    tokens = P["B"] * P["T"]
+    assert d["value"] == pytest.approx(tokens / 0.5e-3)
+    assert d["e2e"]["value"] == pytest.approx(tokens / 12.0e-3)
+    algo = bench.prefill_bytes(P["B"], P["T"], P["H"], P["dk"], P["dv"])
+    assert algo == 675_282_944                     # 2,560 B per token-head + the FP32 final state
+    r = d["roofline"]
+    assert r["achieved"] == pytest.approx(algo / 0.5e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+
+
+def test_job_value_scales_with_ranks(capsys):
+    one = _line(capsys, world=1, ms=0.5)
+    four = _line(capsys, world=4, ms=0.5)
+    assert four["value"] == pytest.approx(4 * one["value"])
+    assert four["n_gpus"] == 4 and four["config"]["global_batch"] == 4 * bench.PREFILL["B"]
