@@ -118,3 +118,12 @@ def test_product_package_does_not_import_oracle():
     for p in list(pkg.rglob("*.py")) + list(pkg.rglob("*.cu")) + list(pkg.rglob("*.cuh")):
         text = p.read_text()
         assert "oracle" not in text.replace("oracle-free", ""), f"{p} mentions the oracle"
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the compiled library the binding raises; there is no fallback path."""
+    from gated_delta_rule_111_b200 import build as b
+    monkeypatch.setattr(g, "_lib", None)
+    monkeypatch.setattr(b, "LIB", str(tmp_path / "libgdn2.so"))
+    with pytest.raises(ImportError, match="libgdn2.so not found"):
+        g.load_library(rebuild_if_stale=False)
