@@ -54,6 +54,28 @@ def prefill_bytes(B, T, H, dk, dv):
     return tok * (2 * dk * 2 + dv * 2 + 2 * dk * 4 + dv * 4 + dv * 2) + B * H * dk * dv * 4  # + S_T
 
 
+def prefill_mma_flops(B, T, H, dk=128, dv=128, C=64):
+    """Tensor-core FLOPs one tensor-core prefill launch executes (TF32 MMAs as issued:
+    per CTA = (batch, head, d_v/2 columns) and chunk: Gram [Etil;Qtil]Ktil^T 2C x C x dk,
+    [Etil;Qtil]S 2C x dv/2 x dk, U = [T;P](R_hi + R_lo) 2 x 2C x dv/2 x C, state update
+    Ktil^T(U_hi + U_lo) 2 x dk x dv/2 x C, P U_hi 2C x dv/2 x C)."""
+    n = dv // 2
+    macs = 2 * C * C * dk + 2 * C * n * dk + 2 * (2 * C * n * C) + 2 * (dk * n * C) + 2 * C * n * C
+    chunks = -(-T // C)
+    return 2 * macs * chunks * 2 * B * H
+
+
+TF32_PER_BF16 = 1.1 / 2.25       # nominal dense TF32 / BF16 tensor rates on B200
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]) * TF32_PER_BF16, "measured bf16 burst x nominal tf32/bf16"
+    return 1590.0 * TF32_PER_BF16, "fallback bf16 x nominal tf32/bf16"
+
+
 def decode_bytes(B, H, dk, dv):
     bh = B * H
     return bh * (2 * dk * dv * 4 + (2 * dk + dv) * 2 + (2 * dk + dv) * 4 + dv * 2)
@@ -334,6 +356,8 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk):
     dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
     st_gbs = state_bytes(Bd, Hd, dk, dv) / (dec_ms / 1e3) / 1e9
     traffic = load_traffic()
+    tflops = prefill_mma_flops(B, T, H, dk, dv) / (ms_step / 1e3) / 1e12
+    tpeak, tsrc = measured_tensor_peak()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -356,6 +380,9 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk):
                          "frac": _num(pre_gbs / hbm), "traffic": traffic.get("gdn2_chunk"),
                          "kernel": "gdn2 chunkwise prefill", "algorithmic_bytes_per_launch": pre_bytes,
                          "peak_source": f"{hbm_src} HBM copy bandwidth", "frac_of_8TBps": _num(pre_gbs / 8000.0)},
+            "tensor_secondary": {"achieved": _num(tflops), "peak": tpeak, "unit": "TFLOP/s", "dtype": "tf32",
+                                 "frac": _num(tflops / tpeak), "flops_per_launch": prefill_mma_flops(B, T, H, dk, dv),
+                                 "peak_source": tsrc},
             "decode": {"metric": "GDN-2 decode state GB/s @B256 H16 d128", "value": _num(st_gbs), "unit": "GB/s",
                        "us_per_step": _num(dec_ms * 1e3), "steps": steps_d * reps,
                        "roofline": {"bound": "hbm", "achieved": _num(dec_gbs), "peak": hbm, "unit": "GB/s",

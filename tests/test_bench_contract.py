@@ -60,3 +60,12 @@ def test_job_value_scales_with_ranks(capsys):
     four = _line(capsys, world=4, ms=0.5)
     assert four["value"] == pytest.approx(4 * one["value"])
     assert four["n_gpus"] == 4 and four["config"]["global_batch"] == 4 * bench.PREFILL["B"]
+
+
+def test_tensor_secondary(capsys):
+    d = _line(capsys, ms=0.5)
+    t = d["tensor_secondary"]
+    # 4.72 M MACs per CTA and chunk; 128 CTAs x 64 chunks for B=4, T=4096, H=16
+    assert t["flops_per_launch"] == 2 * 4_718_592 * 64 * 128
+    assert t["achieved"] == pytest.approx(t["flops_per_launch"] / 0.5e-3 / 1e12)
+    assert t["frac"] == pytest.approx(t["achieved"] / t["peak"]) and t["dtype"] == "tf32"
