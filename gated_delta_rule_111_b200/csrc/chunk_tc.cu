@@ -166,7 +166,9 @@ __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 
 // log-decay up to rounding); Etil, Qtil into X1, Ktil into KS (rows 0-63) and
 // its transpose into Tensor Memory.  Padding tokens (t >= n): zero b from the
 // TMA bounds fill, zero q, k, alpha forced to 1.  prep_decay forms each
-// thread's product of alpha over its 32 tokens (needs only alpha).
+// thread's product of alpha over its 32 tokens (needs only alpha).  kFull: the
+// chunk has all 64 tokens, so no token needs the padding test.
+template <bool kFull>
 __device__ __forceinline__ void prep_decay(const Ctx &c, int qd, int kh, int lane, int n) {
     const int i = 32 * qd + lane;
     const Swz sw((i & 31) * 4u);
@@ -175,12 +177,13 @@ __device__ __forceinline__ void prep_decay(const Ctx &c, int qd, int kh, int lan
 #pragma unroll
     for (int tt = 0; tt < 32; ++tt) {
         const float a = at(c, OFF_KS + rbase + tt * 128 + sw.o[tt & 7]);
-        pa *= (32 * kh + tt < n) ? clamp_alpha(a) : 1.f;
+        pa *= (kFull || 32 * kh + tt < n) ? clamp_alpha(a) : 1.f;
     }
     fptr(c, OFF_PART)[kh * 128 + i] = pa;
 }
 
 // Gate prep proper (after prep_decay and a group barrier).
+template <bool kFull>
 __device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, uint32_t kt_col, int kb, int qd, int kh,
                                      int lane, int n) {
     const int i = 32 * qd + lane;
@@ -205,7 +208,7 @@ __device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, uint32_t kt_c
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int tt = 8 * grp + u;
-            const float a = (32 * kh + tt < n) ? clamp_alpha(av[u]) : 1.f;
+            const float a = (kFull || 32 * kh + tt < n) ? clamp_alpha(av[u]) : 1.f;
             g *= a;
             r *= __fdividef(1.f, a);
             const float qq = __bfloat162float(qs[tt * 32]), kk = __bfloat162float(ks[tt * 32]);
@@ -436,10 +439,12 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
             const uint32_t ph = ck & 1;
             const int t0 = ck * kC, n = min(kC, T - t0);
             if (!group_wait(c, B_FULL_AB, ph, el, kBarK)) break;
-            prep_decay(c, qd, kh, lane, n);
+            if (n == kC) prep_decay<true>(c, qd, kh, lane, n);
+            else prep_decay<false>(c, qd, kh, lane, n);
             if (!group_wait(c, B_FULL_QK, ph, el, kBarK)) break;
             if (ck >= 2 && !group_wait(c, ph ? B_KT_FREE1 : B_KT_FREE0, ((ck - 2) >> 1) & 1, el, kBarK)) break;
-            prep(c, tlane, TM_KT + 64 * ph, ph, qd, kh, lane, n);
+            if (n == kC) prep<true>(c, tlane, TM_KT + 64 * ph, ph, qd, kh, lane, n);
+            else prep<false>(c, tlane, TM_KT + 64 * ph, ph, qd, kh, lane, n);
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
