@@ -282,16 +282,19 @@ __device__ __forceinline__ void invert_offdiag(const Ctx &c, int gtid, uint32_t 
 }
 
 // Split 32 values into TF32 hi + lo parts and store both into the [j][t] tiles
-// UH / UL at token t, columns 32 sh .. 32 sh + 31.
+// UH / UL at token t, columns 32 sh .. 32 sh + 31.  hi keeps the top 10
+// mantissa bits (a TF32 value exactly), lo = x - hi is exact in FP32 and
+// below one TF32 unit of x; the tensor core reads lo to TF32 by dropping its
+// low bits, so hi + lo carries x to within 2^-20 of |x|.
 __device__ __forceinline__ void store_split_jt(const Ctx &c, const float (&x)[32], int t, int sh) {
     const Swz sw((t & 31) * 4u);
     const uint32_t base = (t >> 5) * 8192u + sh * 32 * 128;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const uint32_t o = base + j * 128 + sw.o[j & 7];
-        const float hi = to_tf32(x[j]);
+        const float hi = __uint_as_float(__float_as_uint(x[j]) & 0xFFFFE000u);
         at(c, OFF_UH + o) = hi;
-        at(c, OFF_UL + o) = to_tf32(x[j] - hi);
+        at(c, OFF_UL + o) = x[j] - hi;
     }
 }
 
