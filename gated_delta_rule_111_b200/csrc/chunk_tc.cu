@@ -563,14 +563,11 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
             if (!group_wait(c, B_DIAG_DONE, ph, el, kBarS)) { done_ok = false; break; }
             tc_fence_after();
             invert_offdiag(c, stid, kBarS);
-            if (srow < 64) {
+            if (srow < 64) {        // AS holds exact zeros above the diagonal of T
                 float tv[32];
-                const float *As = fptr(c, OFF_AS);
+                const float *As = fptr(c, OFF_AS) + srow * LDA + 32 * sh;
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int s = 32 * sh + jj;
-                    tv[jj] = (s <= srow) ? to_tf32(As[srow * LDA + s]) : 0.f;
-                }
+                for (int jj = 0; jj < 32; ++jj) tv[jj] = to_tf32(As[jj]);
                 tmem_st32_nowait(tlane + TM_TP + 64 * ph + 32 * sh, tv);
             }
             tmem_wait_st();
