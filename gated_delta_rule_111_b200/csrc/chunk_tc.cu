@@ -462,13 +462,14 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
                 float g[32];
                 tmem_ld32(tlane + TM_G + 32 * kh, g);
                 if (srow < 64) {
-                    float *As = fptr(c, OFF_AS);
+                    // The diagonal 32 x 32 blocks are only read strictly below their diagonal and are
+                    // then overwritten by T_AA, T_BB; A_BA lies wholly below the diagonal.  Only the
+                    // block above the diagonal (rows 0-31, columns 32-63) needs its zeros.
+                    float2 *dst = reinterpret_cast<float2 *>(fptr(c, OFF_AS) + srow * LDA + 32 * kh);
+                    const bool upper = srow < 32 && kh == 1;
 #pragma unroll
-                    for (int jj = 0; jj < 32; jj += 2) {
-                        const int s = 32 * kh + jj;
-                        *reinterpret_cast<float2 *>(As + srow * LDA + s) =
-                            make_float2((s < srow) ? g[jj] : 0.f, (s + 1 < srow) ? g[jj + 1] : 0.f);
-                    }
+                    for (int jj = 0; jj < 32; jj += 2)
+                        dst[jj >> 1] = upper ? make_float2(0.f, 0.f) : make_float2(g[jj], g[jj + 1]);
                 } else {
                     const int t = srow - 64;
 #pragma unroll
