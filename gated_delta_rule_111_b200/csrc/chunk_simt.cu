@@ -1,10 +1,11 @@
 // Chunkwise prefill of the Gated DeltaNet-2 recurrence on CUDA cores, in FP32.
 //
 // "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention"
-// (iplexlaw.co.kr analysis), "Token processing and parallel training": 64-token
-// chunks; the cumulative channel-wise decay is absorbed into the erase factors,
-// leaving a triangular solve and dense products per chunk; decay, state and
-// solve are kept in FP32.
+// (iplexlaw.co.kr analysis), "Token processing and parallel training": the
+// sequence is cut into 64-token blocks; the per-channel decay accumulated since
+// the block start is folded into the erase-side and key-side factors, so each
+// block costs one unit-triangular system plus matrix products; decay, state and
+// the triangular system are carried in FP32.
 //
 // This kernel is the FP32 path (q/k/v in FP32, tolerance 1e-4) and the path for
 // every head size the tensor-core kernel does not cover.  Within a chunk of n

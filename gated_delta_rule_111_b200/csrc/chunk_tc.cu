@@ -2,10 +2,11 @@
 // cores (tcgen05, TF32 operands, FP32 accumulation in Tensor Memory).
 //
 // "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention"
-// (iplexlaw.co.kr analysis), "Token processing and parallel training":
-// 64-token chunks, the cumulative channel-wise decay absorbed into asymmetric
-// erase factors, triangular solves and dense products inside each chunk, FP32
-// decay and state/solve precision.  Per chunk of n tokens from state S:
+// (iplexlaw.co.kr analysis), "Token processing and parallel training": the
+// sequence is cut into 64-token blocks; the per-channel decay accumulated since
+// the block start is folded into the erase-side and key-side factors, so each
+// block costs one unit-triangular system plus matrix products; decay, state and
+// the triangular system are carried in FP32.  Per chunk of n tokens from state S:
 //
 //   gamma_t = prod_{j<=t} alpha_j,  rho_t = 1/gamma_t          (per key channel, FP32)
 //   Etil = b*k*gamma,  Qtil = q*gamma,  Ktil = k*rho            (gate prep)

@@ -10,7 +10,7 @@
  *     z    = w_t (.) v_t                  write vector (value channels)
  *     r    = Sbar^T e                     old read at the erase address
  *     S_t  = Sbar + k_t (z - r)^T         delta write
- *     o_t  = S_t^T q_t                    the query reads the updated state
+ *     o_t  = S_t^T q_t                    output from the state after this token's update
  *
  * Two entry points compute exactly this, in the two execution modes the pages
  * describe ("Token processing and parallel training": chunkwise WY with 64-token
@@ -61,10 +61,10 @@ typedef enum {
 } gdn2_dtype;
 
 /*
- * Chunkwise prefill ("Token processing and parallel training": 64-token chunks,
- * cumulative channel-wise decay absorbed into asymmetric erase factors,
- * triangular solves and dense products within each chunk, FP32 decay and
- * state/solve precision).
+ * Chunkwise prefill ("Token processing and parallel training": 64-token blocks;
+ * the per-channel decay accumulated inside a block is folded into the erase-side
+ * and key-side factors, leaving one unit-triangular system and matrix products
+ * per block; decay, state and the triangular system in FP32).
  *
  *   q, k      [B][T][H][d_k]  dt            read
  *   v         [B][T][H][d_v]  dt            read

@@ -56,7 +56,7 @@ static void load_state(double *S, const double *S0, int b, int h, int H, int dk,
  *   e    = b_t (.) k_t,  z = w_t (.) v_t   erase (key side) and write (value side)
  *   r    = Sbar^T e                        old read at the erase address
  *   S_t  = Sbar + k_t (z - r)^T            delta write
- *   o_t  = S_t^T q_t                       the query reads the updated state
+ *   o_t  = S_t^T q_t                       output from the state after this token's update
  * S0 may be NULL (zeros); ST may be NULL (not returned).
  */
 void oracle_gdn2(int B, int T, int H, int dk, int dv,

@@ -1,10 +1,11 @@
 """The chunkwise algebra the CUDA kernels implement, checked in FP64 against the
 token-by-token oracle (CPU only).
 
-"Token processing and parallel training" (Gated DeltaNet-2 analysis) sketches
-the parallel form: 64-token chunks, cumulative channel-wise decay absorbed into
-asymmetric erase factors, a triangular solve and dense products per chunk.  Our
-re-derivation, per chunk of n tokens starting from state S:
+"Token processing and parallel training" (Gated DeltaNet-2 analysis) outlines
+the parallel form only: 64-token blocks whose accumulated per-channel decay is
+folded into the erase-side and key-side factors, so that each block needs one
+unit-triangular system and matrix products.  Our re-derivation, per chunk of n
+tokens starting from state S:
 
   gamma_t = prod_{j<=t} alpha_j  (per key channel),   rho_t = 1 / gamma_t
   Etil = e * gamma,  Qtil = q * gamma,  Ktil = k * rho        (e = b*k, z = w*v)
