@@ -3,15 +3,16 @@
 The oracle is tied to facts outside itself, from "Gated DeltaNet-2: Decoupling
 Erase and Write in Linear Attention" (iplexlaw.co.kr analysis) and plain algebra:
 
-* KDA reduction -- tying both gates to one scalar beta recovers KDA ("Independent
-  decisions on two axes"); checked against a separately coded transition-matrix
-  recurrence (I - beta k k^T) diag(alpha) S + beta k v^T.
+* KDA reduction -- when the erase and write gates are both the same per-token
+  scalar beta, the method is KDA ("Independent decisions on two axes"); checked
+  against a separately coded transition-matrix recurrence
+  (I - beta k k^T) diag(alpha) S + beta k v^T.
 * Gated DeltaNet reduction -- scalar decay on top of the tie recovers Gated
   DeltaNet; checked against alpha (I - beta k k^T) S + beta k v^T.
 * Delta-rule identity -- with b = 1 and a unit key, S_t^T k_t = z_t exactly for any
   decay and prior state (S_t^T k = Sbar^T k + (k^T k)(z - Sbar^T k)); with q = k the
-  output is w*v.  ("DeltaNet updates the difference between an incoming value and
-  the state's current read", "From a growing cache to a fixed state".)
+  output is w*v.  (The delta rule writes the gap between the new value and what the
+  state currently returns for the key: "From a growing cache to a fixed state".)
 * b = 0 -- no erase, so the output is a decayed causal linear-attention sum,
   computed by an explicit O(T^2) loop.
 * alpha = 1, b = 0, w = 1 -- plain causal linear attention tril(Q K^T) V, a
