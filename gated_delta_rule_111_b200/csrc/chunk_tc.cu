@@ -36,9 +36,11 @@
 //   warp 0      TMA producer (alpha, b into their operand tiles; q, k into a
 //               BF16 staging tile; L2 prefetch of the next chunk's tiles)
 //   warp 1      MMA issuer (one thread, every tcgen05 instruction)
-//   warps 2-9   key side: gate prep, Gram epilogue, blocked inversion of (I + A)
-//   warps 10-17 state side: R, U and state/output epilogues (w, v read
-//               straight from global memory into registers)
+//   warps 2-9   key side: gate prep, Gram epilogue, the diagonal 32 x 32
+//               blocks of T = (I + A)^{-1}
+//   warps 10-17 state side: R epilogue (w, v read straight from global memory
+//               into registers), the off-diagonal block of T and its copy into
+//               Tensor Memory, U, state and output epilogues
 // The key side of chunk c+1 runs while the state chain of chunk c runs; the
 // key factor Ktil^T and [T; P] are double-buffered in Tensor Memory for that.
 // The FP32 state itself lives in Tensor Memory: the state-update MMA
