@@ -106,7 +106,7 @@ constexpr uint32_t TM_COLS = 512;
 
 enum {
     B_FULL_AB = 0, B_FULL_QK, B_X1_FREE, B_KPREP, B_G_FULL, B_DIAG_DONE, B_TP_READY, B_S_READY,
-    B_X_FULL, B_R_READY, B_U_FULL, B_U_READY, B_D_FULL, B_O_FULL, B_KT_FREE0, B_KT_FREE1, NBARS
+    B_X_FULL, B_R_READY, B_U_FULL, B_U_READY, B_D_FULL, B_O_FULL, B_KT_FREE0, B_KT_FREE1, B_DRAIN, NBARS
 };
 
 constexpr uint32_t TX_AB = 8 * 8192;
@@ -340,11 +340,15 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
+        // Each lane finally waits (bounded) for the last copy it issued, so that no copy
+        // into shared memory is still in flight when the CTA ends, also after a give-up.
         if (lane == 0) {            // alpha -> KS rows 0-63, b -> X1 rows 0-63
+            int last = -1;
             for (int ck = 0; ck < nchunks; ++ck) {
                 if (ck > 0 && !solo_wait(c, B_X1_FREE, (ck - 1) & 1)) break;
                 const uint32_t fb = c.bar(B_FULL_AB);
                 mbar_expect_tx(fb, TX_AB);
+                last = ck;
                 for (int a = 0; a < 4; ++a) {
                     tma_load_4d(c.sa + OFF_KS + a * 16384, &maps.alpha, 32 * a, h, ck * kC, bidx, fb);
                     tma_load_4d(c.sa + OFF_X1 + a * 16384, &maps.b, 32 * a, h, ck * kC, bidx, fb);
@@ -358,11 +362,14 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
                     tma_prefetch_4d(&maps.v, col0, h, (ck + 1) * kC, bidx);
                 }
             }
+            if (last >= 0) (void)mbar_wait(c.bar(B_FULL_AB), last & 1, kWaitLimit / 8);
         } else if (lane == 1) {     // q, k -> QK once the gate prep has consumed the previous chunk's
+            int last = -1;
             for (int ck = 0; ck < nchunks; ++ck) {
                 if (ck > 0 && !solo_wait(c, B_KPREP, (ck - 1) & 1)) break;
                 const uint32_t fb = c.bar(B_FULL_QK);
                 mbar_expect_tx(fb, TX_QK);
+                last = ck;
                 for (int a = 0; a < 4; ++a) {
                     tma_load_4d(c.sa + OFF_QK + a * 4096, &maps.q, 32 * a, h, ck * kC, bidx, fb);
                     tma_load_4d(c.sa + OFF_QK + 16384 + a * 4096, &maps.k, 32 * a, h, ck * kC, bidx, fb);
@@ -373,6 +380,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
                         tma_prefetch_4d(&maps.k, 32 * a, h, (ck + 1) * kC, bidx);
                     }
             }
+            if (last >= 0) (void)mbar_wait(c.bar(B_FULL_QK), last & 1, kWaitLimit / 8);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -433,6 +441,9 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
                 mma_commit(c.bar(B_O_FULL));
                 mma_commit(c.bar(ph ? B_KT_FREE1 : B_KT_FREE0));     // Ktil^T and [T; P] of this parity
             }
+            // Every MMA issued above has completed before Tensor Memory is released (bounded).
+            mma_commit(c.bar(B_DRAIN));
+            (void)mbar_wait(c.bar(B_DRAIN), 0, kWaitLimit / 8);
         }
         __syncwarp();
     } else if (warp < 10) {
@@ -644,14 +655,10 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
         }
     }
 
-    // Every role has finished or given up.  Drain copies that may still be in
-    // flight after a give-up (bounded), then release Tensor Memory.
+    // Every role has finished or given up, and the producer and MMA lanes have seen
+    // their last copy and MMA complete: release Tensor Memory.
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *c.abort_flag) {
-        (void)mbar_wait(c.bar(B_FULL_AB), 0, kWaitLimit / 8);
-        (void)mbar_wait(c.bar(B_FULL_QK), 0, kWaitLimit / 8);
-    }
     if (warp == 0) {
         __syncwarp();
         tc_fence_after();
