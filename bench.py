@@ -43,6 +43,7 @@ import gdn2_inputs as gi  # noqa: E402
 
 PREFILL = gi.PREFILL_4K
 DECODE = gi.DECODE_B256
+LONG = gi.LONG_RAGGED
 BYTES_PER_TOKEN_HEAD = 2560        # q,k,v bf16 (768) + alpha,b,w fp32 (1536) + o bf16 (256)
 METRIC = "GDN-2 chunk fwd tokens/s @H16 d128 T4K"
 UNIT = "tokens/s"
@@ -239,7 +240,10 @@ def run_ours(args):
         ms_step, e2e_ms, h2d, d2h, clk = run_prefill(args, torch, dist, g, world, rank, dev, stream)
     if args.workload in ("all", "decode"):
         dec_ms = run_decode(args, torch, dist, g, world, rank, dev, stream)
-    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk)
+    long_ms = float("nan")
+    if args.workload in ("all", "long"):
+        long_ms = run_long(args, torch, dist, g, world, rank, dev, stream)
+    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -339,11 +343,40 @@ def run_decode(args, torch, dist, g, world, rank, dev, stream):
     return dec_ms
 
 
+def run_long(args, torch, dist, g, world, rank, dev, stream):
+    """One prefill call on the long ragged workload (B=1, T=65,573, H=16, S0 != 0): latency
+    bound (32 CTAs, 1,025 chunks each), reported for the record; returns ms per call."""
+    x = gi.chunk_inputs(**LONG, seed=rank)
+    d = device_inputs(torch, x, dev)
+    S0 = torch.from_numpy(x["S0"]).to(dev)
+    del x
+    B, T, H, dv = LONG["B"], LONG["T"], LONG["H"], LONG["dv"]
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    ST = torch.empty_like(S0)
+
+    def call():
+        g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], S0, o=o, S_T=ST, stream=stream)
+
+    call()
+    sync_ranks(torch, dist, world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    ev0.record(stream)
+    for _ in range(reps):
+        call()
+    ev1.record(stream)
+    sync_ranks(torch, dist, world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / reps, torch, dist, world, dev)
+    del d, S0, o, ST
+    torch.cuda.empty_cache()
+    return ms
+
+
 def _num(x):
     return None if x != x else x      # NaN (workload not run) -> null
 
 
-def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk):
+def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=float("nan")):
     B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
     Bd, Hd = DECODE["B"], DECODE["H"]
     steps_d = DECODE["steps"]
@@ -389,6 +422,10 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk):
                                     "frac": _num(dec_gbs / hbm), "traffic": traffic.get("gdn2_decode"),
                                     "algorithmic_bytes_per_launch": dec_bytes,
                                     "frac_of_8TBps": _num(dec_gbs / 8000.0)}},
+            "long_ragged": {"workload": "B=1 T=65573 H=16 d_k=d_v=128, S0 != 0 (ragged last chunk)",
+                            "ms_per_call": _num(long_ms),
+                            "tokens_per_s": _num(LONG["B"] * LONG["T"] * world / (long_ms / 1e3)),
+                            "note": "latency bound: 32 CTAs walk 1,025 chunks each; reported, no target"},
             "gpu_launches": args.steps,
             "clocks": clk.summary() if clk is not None else None,
             "cpu_baseline": cpu,
@@ -453,7 +490,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "long"], default="all",
                     help="run only one workload's measurement (for profiling one kernel)")
     args = ap.parse_args()
     if args.impl == "ours":

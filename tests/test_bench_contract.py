@@ -29,7 +29,7 @@ def test_keys_and_types(capsys):
     d = _line(capsys)
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
               "scaling", "vs_baseline", "dtype", "data", "config", "e2e", "roofline", "gpu_launches", "clocks",
-              "cpu_baseline", "decode"):
+              "cpu_baseline", "decode", "long_ragged"):
         assert k in d, k
     assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["vs_baseline"] is None
     assert d["steps"] == 20 and d["warmup"] == 5 and d["n_gpus"] == 1 and d["gpu_launches"] == 20
