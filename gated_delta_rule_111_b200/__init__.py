@@ -19,7 +19,8 @@ import torch
 
 from . import build as _build
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_recurrent_step", "gdn2_device_error", "library_path", "load_library", "exported_symbols",
+__all__ = ["gdn2_chunk_fwd", "gdn2_recurrent_step", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
+           "load_library", "exported_symbols",
            "GDN2_OK", "GDN2_ERR_INVALID_ARG", "GDN2_ERR_UNSUPPORTED", "GDN2_ERR_CUDA", "Gdn2Error"]
 
 GDN2_OK, GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_CUDA = 0, 1, 2, 3
@@ -60,6 +61,8 @@ def load_library(rebuild_if_stale: bool = True) -> ctypes.CDLL:
     lib.gdn2_version.restype = i
     lib.gdn2_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
     lib.gdn2_device_error.restype = i
+    lib.gdn2_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.gdn2_set_wait_limit.restype = i
     _lib = lib
     return lib
 
@@ -114,6 +117,11 @@ def gdn2_device_error(clear: bool = True) -> int:
     return int(code.value)
 
 
+def gdn2_set_wait_limit(cycles: int = 0) -> None:
+    """Test hook: SM cycles before a kernel's internal wait gives up (0 = default, ~2 s)."""
+    _check(load_library().gdn2_set_wait_limit(int(cycles)))
+
+
 def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, *, o=None, S_T=None, output_final_state=True,
                    stream=None):
     """Chunkwise prefill.  q,k [B,T,H,dk], v [B,T,H,dv] (bf16 or fp32); alpha,b [B,T,H,dk] and
@@ -140,8 +148,9 @@ def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, *, o=None, S_T=None, output_fi
         S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     elif S_T is not None:
         _need(S_T, "S_T", torch.float32, (B, H, dk, dv), dev)
-    _check(lib.gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
-                              _ptr(S_T), B, T, H, dk, dv, code, _stream(stream, dev)))
+    with torch.cuda.device(dev):
+        _check(lib.gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                                  _ptr(S_T), B, T, H, dk, dv, code, _stream(stream, dev)))
     return o, S_T
 
 
@@ -164,6 +173,7 @@ def gdn2_recurrent_step(q, k, v, alpha, b, w, S, *, o=None, stream=None):
         o = torch.empty((B, H, dv), dtype=dt, device=dev)
     else:
         _need(o, "o", dt, (B, H, dv), dev)
-    _check(lib.gdn2_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
-                                   B, H, dk, dv, code, _stream(stream, dev)))
+    with torch.cuda.device(dev):
+        _check(lib.gdn2_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
+                                       B, H, dk, dv, code, _stream(stream, dev)))
     return o

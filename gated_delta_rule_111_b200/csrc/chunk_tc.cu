@@ -3,53 +3,63 @@
 //
 // "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention"
 // (iplexlaw.co.kr analysis), "Token processing and parallel training": the
-// sequence is cut into 64-token blocks; the per-channel decay accumulated since
-// the block start is folded into the erase-side and key-side factors, so each
-// block costs one unit-triangular system plus matrix products; decay, state and
-// the triangular system are carried in FP32.  Per chunk of n tokens from state S:
+// sequence is cut into blocks of up to 64 tokens; the per-channel decay
+// accumulated since the block start is folded into the erase-side and key-side
+// factors, so each block costs one unit-triangular system plus matrix
+// products; decay, state and the triangular system are carried in FP32.  Per
+// chunk of n tokens from state S:
 //
-//   gamma_t = prod_{j<=t} alpha_j,  rho_t = 1/gamma_t          (per key channel, FP32)
-//   Etil = b*k*gamma,  Qtil = q*gamma,  Ktil = k*rho            (gate prep)
-//   [A; P] = [Etil; Qtil] Ktil^T                                 (Gram, tensor core)
-//   T = (I + strict_tril(A))^{-1}                                (FP32 blocked inversion)
-//   [Etil S; Qtil S]                                             (tensor core)
-//   R = w*v - Etil S                                             (FP32 epilogue)
-//   U = T R                                                      (tensor core)
-//   O = Qtil S + tril(P) U                                       (tensor core, accumulated)
-//   S <- diag(gamma_n) (S + Ktil^T U)                            (tensor core + FP32 epilogue)
+//   gamma_t = prod_{j<=t} alpha_j                                (per key channel, FP32)
+//   Etil = b*k*gamma,  Qtil = q*gamma,  Ktil = k / gamma          (gate prep)
+//   [A; P] = [Etil; Qtil] Ktil^T                                  (Gram, tensor core)
+//   T = (I + strict_tril(A))^{-1}                                 (FP32 blocked inversion)
+//   [Etil S; Qtil S]                                              (tensor core)
+//   R = w*v - Etil S                                              (FP32 epilogue)
+//   U = T R                                                       (tensor core)
+//   O = Qtil S + tril(P) U                                        (tensor core, accumulated)
+//   S <- diag(gamma_n) (S + Ktil^T U)                             (tensor core + FP32 epilogue)
 //
 // U holds the per-token corrections z_t - r_t of the token recurrence, so this
 // is the token loop's arithmetic, re-associated.
 //
+// Chunk length.  Ktil = k / gamma grows inside a chunk as the decay deepens.
+// A chunk is therefore cut short, to n <= 64 tokens, where the decay
+// accumulated since its first token would fall below 2^-64 in some key
+// channel; the next chunk starts at the cut.  Every factor then stays within
+// [2^-64, 2^64] of its input, for every alpha in (0, 1] (values of alpha below
+// 2^-64 are taken as 2^-64, which changes a decayed state row by less than
+// 2^-64 of its size).  On ordinary gates (a few to some tens of nats of decay
+// per 64 tokens) no chunk is cut; a chunk of one token is always exact.
+//
 // Precision: tensor-core operands are TF32 (10-bit mantissa); accumulation,
 // decay, R, T and the carried state are FP32.  R and U enter their products as
-// split operands, x = x_hi + x_lo with both parts TF32 (T R = T R_hi + T R_lo,
-// Ktil^T U = Ktil^T U_hi + Ktil^T U_lo), which keeps the carried state within
-// ~0.3% of its RMS over 16K tokens (plain TF32 there: ~0.7%).  BF16 operands
-// lose too much: the read r = Sbar^T e nearly cancels the write z in the delta
-// rule.  The key factor Ktil = k / gamma grows within a chunk as
-// exp(-sum ln alpha); it must stay below ~1e34 (sum of -ln alpha over one chunk
-// <= 78 per key channel), as documented in gdn2.h.
+// split operands, x = x_hi + x_lo with both parts TF32, which keeps the carried
+// state within a few 1e-3 of its RMS over 16K tokens.
 //
-// Organisation: one CTA per (batch, head, 64-column half of d_v), 18 warps in
-// four roles that run concurrently and hand work over through mbarriers:
-//   warp 0      TMA producer (alpha, b into their operand tiles; q, k into a
-//               BF16 staging tile; L2 prefetch of the next chunk's tiles)
-//   warp 1      MMA issuer (one thread, every tcgen05 instruction)
-//   warps 2-9   key side: gate prep, Gram epilogue, the diagonal 32 x 32
-//               blocks of T = (I + A)^{-1}
-//   warps 10-17 state side: R epilogue (w, v read straight from global memory
-//               into registers), the off-diagonal block of T and its copy into
-//               Tensor Memory, U, state and output epilogues
-// The key side of chunk c+1 runs while the state chain of chunk c runs; the
-// key factor Ktil^T and [T; P] are double-buffered in Tensor Memory for that.
-// The FP32 state itself lives in Tensor Memory: the state-update MMA
-// accumulates Ktil^T U onto it, the epilogue scales it by the chunk decay and
-// writes the TF32 copy that the next chunk's MMAs read.
-// Shared-memory MMA operands are K-major with the 128-byte swizzle; operands
-// needed transposed (Ktil^T, [T; P]) are read from Tensor Memory as operand A.
+// Organisation: one CTA per (sequence, head, 64-column half of d_v), 17 warps
+// in three roles that run concurrently and hand work over through mbarriers:
+//   warp 0      MMA issuer: one thread issues every tcgen05 instruction, in
+//               whichever order their inputs become ready
+//   warps 1-8   key side, one chunk ahead of the state side.  alpha, b, q, k
+//               arrive by TMA in 128-byte-swizzled tiles; a thread per key
+//               channel forms the decay products and the chunk length and
+//               turns the tiles in place into Qtil and Etil, writes Ktil (the
+//               Gram's B operand) and Ktil^T into Tensor Memory (the state
+//               update's A operand); a thread per token then moves the rows
+//               of [Etil; Qtil] into Tensor Memory (the A operand of the Gram
+//               and X products); Gram epilogue; the whole inversion
+//               T = (I + A)^{-1}
+//   warps 9-16  state side: R epilogue (w, v straight from global memory into
+//               registers), U, state and output epilogues
+// The state chain of a chunk is X -> R -> U -> state update; everything that
+// does not depend on the state (gate prep, Gram, T) is done one chunk ahead.
+// The FP32 state lives in Tensor Memory: the state-update MMA accumulates
+// Ktil^T U onto it, the epilogue scales it by the chunk decay and writes the
+// TF32 copy that the next chunk's X product reads.
 #include <cudaTypedefs.h>
 #include <stdio.h>
+
+#include <atomic>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -62,70 +72,100 @@ namespace tc {
 
 using namespace sm100;
 
-constexpr int kC = 64;            // chunk length (tokens)
+constexpr int kC = 64;            // longest chunk (tokens)
 constexpr int kDK = 128;          // key channels
+constexpr int kDV = 128;          // value channels of a head
 constexpr int kDVS = 64;          // value columns per CTA
-constexpr int kThreads = 576;     // 18 warps
+constexpr int kThreads = 544;     // 17 warps
 constexpr int kGroup = 256;       // threads in each of the two compute groups
-constexpr uint32_t kBarK = 1, kBarS = 2;   // named hardware barriers of the groups
-constexpr long long kWaitLimit = 4000000000ll;   // ~2 s of SM cycles per wait
+constexpr uint32_t kBarK = 1, kBarS = 2;        // named hardware barriers of the groups
+constexpr float kGammaMin = 5.42101086e-20f;   // 2^-64: floor of the decay spanned by one chunk
+constexpr long long kDrainLimit = 4000000000ll; // ~2 s: end-of-kernel waits for in-flight MMAs
 
-// Shared-memory map (bytes from a 1024-aligned base).  MMA tiles hold TF32,
-// 32 elements per 128-byte swizzled row, K-major:
-//   X1  rows 0-63 Etil[t][i], rows 64-127 Qtil[t][i]         4 atoms x 16 KB (i = key channel)
-//   KS  rows 0-63 Ktil[s][i], rows 64-127 S[i][j] as [j][i]    4 atoms x 16 KB
-//   UH  R_hi, later U_hi, as [j][t]                           2 atoms x 8 KB (t = token)
-//   UL  R_lo, later U_lo, as [j][t]                           2 atoms x 8 KB
-//   QK  q, k as BF16 [a][t][32] (a = channel block of 32), 16 KB each: TMA
-//       destinations, read by the gate prep
+// Shared-memory map (bytes from a 1024-aligned base).  Tiles hold 64 rows of
+// 128 swizzled bytes per block (8 KB):
+//   AT  alpha[t][i] as TMA delivers it (4 channel blocks of FP32), turned in
+//       place into Qtil (TF32)
+//   BT  b[t][i], turned in place into Etil (TF32)
+//   QT  q[t][i], KT  k[t][i] (BF16, 2 blocks of 64 channels each)
+//   KG  Ktil[s][i] (TF32, 4 channel blocks): B operand of the Gram (K-major)
+//   SC  S[i][j] as [j][i] (TF32, 4 channel blocks): B operand of the X product
+//   UH  R_hi, later U_hi, as [j][t] (2 token blocks);  UL  R_lo, later U_lo
 //   AS  A, then T in place (FP32 [64][66]);  XS block products (FP32 [32][34])
-constexpr uint32_t OFF_X1 = 0;
-constexpr uint32_t OFF_KS = OFF_X1 + 65536;
-constexpr uint32_t OFF_UH = OFF_KS + 65536;
-constexpr uint32_t OFF_UL = OFF_UH + 16384;
-constexpr uint32_t OFF_GN = OFF_UL + 16384;            // float[2][128] decay over the chunk (by buffer)
-constexpr uint32_t OFF_PART = OFF_GN + 1024;           // float[2][128] half-chunk decay products
-constexpr uint32_t OFF_BAR = OFF_PART + 1024;          // mbarriers
-constexpr uint32_t OFF_MISC = OFF_BAR + 256;           // tmem base, abort flag
+constexpr uint32_t TILE = 8192;
+constexpr uint32_t OFF_AT = 0;
+constexpr uint32_t OFF_BT = OFF_AT + 4 * TILE;
+constexpr uint32_t OFF_QT = OFF_BT + 4 * TILE;
+constexpr uint32_t OFF_KT = OFF_QT + 2 * TILE;
+constexpr uint32_t OFF_KG = OFF_KT + 2 * TILE;
+constexpr uint32_t OFF_SC = OFF_KG + 4 * TILE;
+constexpr uint32_t OFF_UH = OFF_SC + 4 * TILE;
+constexpr uint32_t OFF_UL = OFF_UH + 2 * TILE;
 constexpr int LDA = 66, LDX = 34;
-constexpr uint32_t OFF_QK = (OFF_MISC + 16 + 1023) / 1024 * 1024;
-constexpr uint32_t OFF_AS = OFF_QK + 32768;
+constexpr uint32_t OFF_AS = OFF_UL + 2 * TILE;
 constexpr uint32_t OFF_XS = OFF_AS + 64 * LDA * 4;
-constexpr uint32_t SMEM_USED = OFF_XS + 32 * LDX * 4;
+// Per-chunk record handed from the key side to the issuer and the state side.
+struct ChunkRec {
+    int t0, n, last, pad;
+    float gn[kDK];                // decay over the chunk, per key channel
+};
+constexpr int kRecSlots = 4;
+constexpr uint32_t OFF_REC = OFF_XS + 32 * LDX * 4;
+constexpr uint32_t OFF_PART = OFF_REC + kRecSlots * sizeof(ChunkRec);   // float[128]
+constexpr uint32_t OFF_BAR = OFF_PART + 512;                             // mbarriers
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;   // [0] tmem base, [1] abort flag, [2] first cut
+constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+static_assert(OFF_REC % 16 == 0 && sizeof(ChunkRec) % 16 == 0, "record alignment");
+constexpr uint32_t TX_AB = 8 * TILE;                   // alpha and b of one chunk
+constexpr uint32_t TX_QK = 4 * TILE;                   // q and k of one chunk
 
 // Tensor Memory columns (512 allocated).
-constexpr uint32_t TM_G = 0;        // Gram: lanes 0-63 A, lanes 64-127 P                 (64 cols)
-constexpr uint32_t TM_X = 64;       // [Etil;Qtil] S, then + P U: lanes 64-127 -> O       (64 cols)
-constexpr uint32_t TM_U = 128;      // U = T R (lanes 0-63)                                (64 cols)
-constexpr uint32_t TM_KT = 192;     // 2 buffers: A operand Ktil^T, lane i, column s      (2 x 64 cols)
-constexpr uint32_t TM_TP = 320;     // 2 buffers: A operand [T; P], lane t, column s      (2 x 64 cols)
-constexpr uint32_t TM_S = 448;      // FP32 state S[i][j], lane i, column j               (64 cols)
+constexpr uint32_t TM_EQ = 0;       // A operand [Etil; Qtil]: lane t (0-63 Etil, 64-127 Qtil), column i  (128 cols)
+constexpr uint32_t TM_X = 128;      // [Etil;Qtil] S, then + P U: lanes 64-127 -> O                     (64 cols)
+constexpr uint32_t TM_U = 192;      // U = T R (lanes 0-63)                                             (64 cols)
+constexpr uint32_t TM_S = 256;      // FP32 state S[i][j], lane i, column j                             (64 cols)
+constexpr uint32_t TM_TP = 320;     // 2 buffers: the Gram [A; P], then the A operand [T; P]            (2 x 64 cols)
+constexpr uint32_t TM_KH = 448;     // A operand Ktil^T, lane i, column s                               (64 cols)
 constexpr uint32_t TM_COLS = 512;
 
 enum {
-    B_FULL_AB = 0, B_FULL_QK, B_X1_FREE, B_KPREP, B_G_FULL, B_DIAG_DONE, B_TP_READY, B_S_READY,
-    B_X_FULL, B_R_READY, B_U_FULL, B_U_READY, B_D_FULL, B_O_FULL, B_KT_FREE0, B_KT_FREE1, B_DRAIN, NBARS
+    B_KPREP = 0, B_G_FULL, B_S_READY, B_X_FULL, B_R_READY, B_TP_READY0, B_TP_READY1, B_U_FULL, B_U_READY,
+    B_D_FULL, B_O_FULL, B_KH_READY, B_KH_FREE, B_TP_FREE0, B_TP_FREE1, B_RR0, B_RR1, B_RR2, B_RR3,
+    B_FULL_AB, B_FULL_QK, B_DRAIN, NBARS
 };
+static_assert(NBARS * 8 <= 256, "barrier area");
 
-constexpr uint32_t TX_AB = 8 * 8192;
-constexpr uint32_t TX_QK = 8 * 4096;
-
+// Flat token index space: token t of sequence s is row (tok * H + h) of every
+// per-token tensor, tok = s * T + t (fixed length) or the packed index (varlen).
 struct Maps {
-    CUtensorMap q, k, v, alpha, b, w;
+    CUtensorMap q, k, v, alpha, b, w;    // 3-D {channel, head, token}, used for L2 prefetch
+};
+struct Params {
+    const __nv_bfloat16 *q, *k, *v;
+    const float *alpha, *b, *w;
+    const float *S0;
+    __nv_bfloat16 *o;
+    float *S_T;
+    const int *cu_seqlens;    // nullptr: nseq sequences of T tokens; else packed offsets [nseq + 1]
+    int T, H;
+    long long wait_limit;     // SM cycles before a pipeline wait gives up
 };
 
 struct Ctx {
     uint8_t *sm;          // 1024-aligned shared base (generic pointer)
     uint32_t sa;          // same, shared-window address
     volatile uint32_t *abort_flag;
+    long long limit;
     __device__ __forceinline__ uint32_t bar(int i) const { return sa + OFF_BAR + 8 * i; }
 };
 
 __device__ __forceinline__ float *fptr(const Ctx &c, uint32_t off) { return reinterpret_cast<float *>(c.sm + off); }
 __device__ __forceinline__ float &at(const Ctx &c, uint32_t off) { return *reinterpret_cast<float *>(c.sm + off); }
-__device__ __forceinline__ float4 &at4(const Ctx &c, uint32_t off) { return *reinterpret_cast<float4 *>(c.sm + off); }
+__device__ __forceinline__ ChunkRec &rec(const Ctx &c, int ck) {
+    return reinterpret_cast<ChunkRec *>(c.sm + OFF_REC)[ck & (kRecSlots - 1)];
+}
 
 // Swizzled offsets of one fixed 4-byte column position in a tile with 128-byte
 // rows: element (row, byte cb) is at row*128 + o[row % 8].
@@ -137,99 +177,166 @@ struct Swz {
     }
 };
 
-// A wait whose outcome is uniform across a compute group: one thread polls the
-// mbarrier (bounded), the group meets at its named barrier, all read the flag.
-__device__ __forceinline__ bool group_wait(const Ctx &c, int which, uint32_t parity, bool elected, uint32_t bar_id) {
-    if (elected && *c.abort_flag == 0 && !mbar_wait(c.bar(which), parity, kWaitLimit)) {
-        *c.abort_flag = 1;
-        atomicExch(&g_device_error, 1u + (unsigned)which);
-    }
-    named_bar(bar_id, kGroup);
-    return *c.abort_flag == 0;
+__device__ __forceinline__ void record_abort(const Ctx &c, int which) {
+    *c.abort_flag = 1;
+    atomicExch(&g_device_error, 1u + (unsigned)which);
 }
-// Bounded wait for a single thread (producer, MMA issuer).
+// A wait whose outcome is uniform across a compute group: one thread polls the
+// mbarrier (bounded), and the group's barrier ORs the failure over all of it.
+__device__ __forceinline__ bool group_wait(const Ctx &c, int which, uint32_t parity, bool elected, uint32_t bar_id) {
+    bool fail = false;
+    if (elected) {
+        if (*c.abort_flag) fail = true;
+        else if (!mbar_wait(c.bar(which), parity, c.limit)) { record_abort(c, which); fail = true; }
+    }
+    return !named_bar_or(bar_id, kGroup, fail);
+}
+// Bounded wait for a single thread (the MMA issuer).
 __device__ __forceinline__ bool solo_wait(const Ctx &c, int which, uint32_t parity) {
     if (*c.abort_flag) return false;
-    if (!mbar_wait(c.bar(which), parity, kWaitLimit)) {
-        *c.abort_flag = 1;
-        atomicExch(&g_device_error, 1u + (unsigned)which);
+    if (!mbar_wait(c.bar(which), parity, c.limit)) {
+        record_abort(c, which);
         return false;
     }
     return true;
 }
 
-// ---------------------------------------------------------------------------
-// Key side.  Thread (lane quarter qd, half kh, lane l) owns key channel
-// i = 32 qd + l for tokens [32 kh, 32 kh + 32) in the gate prep, and TMEM lane
-// 32 qd + l, columns [32 kh, 32 kh + 32) in the Gram epilogue.
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
-// Gate prep: cumulative decay as running FP32 products (exp of the cumulative
-// log-decay up to rounding); Etil, Qtil into X1, Ktil into KS (rows 0-63) and
-// its transpose into Tensor Memory.  Padding tokens (t >= n): zero b from the
-// TMA bounds fill, zero q, k, alpha forced to 1.  prep_decay forms each
-// thread's product of alpha over its 32 tokens (needs only alpha).  kFull: the
-// chunk has all 64 tokens, so no token needs the padding test.
-template <bool kFull>
-__device__ __forceinline__ void prep_decay(const Ctx &c, int qd, int kh, int lane, int n) {
-    const int i = 32 * qd + lane;
-    const Swz sw((i & 31) * 4u);
-    const uint32_t rbase = (i >> 5) * 16384u + kh * 32 * 128;
-    float pa = 1.f;
+// ---------------------------------------------------------------------------
+// Key side, pass A (thread per key channel i and token half hh; warp w owns
+// channel block w % 4, whose Tensor Memory lanes it may access): decay
+// products from the alpha tile, the chunk length, then in place alpha -> Qtil
+// and b -> Etil, and Ktil into KG.  Tokens past the chunk become padding (no
+// decay, zero rows).  Returns the chunk length n (uniform across the group).
+__device__ __forceinline__ int key_decay(const Ctx &c, int warp, int lane, int t0, int navail, int te,
+                                         ChunkRec &r, bool el) {
+    const int cb = warp & 3, hh = (warp - 1) >> 2;
+    const int i = 32 * cb + lane, tl0 = 32 * hh;
+    const int nv = min(32, max(0, navail - tl0));
+    const Swz sw((i & 31) * 4u);                 // FP32 tiles: byte column of channel i
+    const Swz swh((i & 63) * 2u);                // BF16 tiles
+    const uint32_t fb = (uint32_t)cb * TILE + tl0 * 128;
+    const uint32_t hb = (uint32_t)(i >> 6) * TILE + tl0 * 128;
+    float pr[32];
 #pragma unroll
     for (int tt = 0; tt < 32; ++tt) {
-        const float a = at(c, OFF_KS + rbase + tt * 128 + sw.o[tt & 7]);
-        pa *= (kFull || 32 * kh + tt < n) ? clamp_alpha(a) : 1.f;
+        const float a = at(c, OFF_AT + fb + tt * 128 + sw.o[tt & 7]);
+        pr[tt] = tt < nv ? fmaxf(a, kGammaMin) : 1.f;
     }
-    fptr(c, OFF_PART)[kh * 128 + i] = pa;
+    float run = 1.f;
+#pragma unroll
+    for (int tt = 0; tt < 32; ++tt) {
+        run *= pr[tt];
+        pr[tt] = run;
+    }
+    float *part = fptr(c, OFF_PART);
+    int *nfirst = reinterpret_cast<int *>(c.sm + OFF_MISC + 8);
+    if (hh == 0) part[i] = run;
+    named_bar(kBarK, kGroup);
+    float carry = hh ? part[i] : 1.f;
+    // first local token whose decay since the chunk start is below the floor
+    int first = 32;
+#pragma unroll
+    for (int tt = 31; tt >= 0; --tt)
+        if (carry * pr[tt] < kGammaMin) first = tt;
+    int cut = first < 32 ? tl0 + first : kC;
+    cut = __reduce_min_sync(0xffffffffu, cut);
+    if (lane == 0 && cut < kC) atomicMin(nfirst, cut);
+    named_bar(kBarK, kGroup);
+    const int n = min(navail, *nfirst);
+    if (n < navail) {
+        // Cut chunk: tokens from n on belong to the next chunk (no decay here).
+        float lastv = 1.f;
+#pragma unroll
+        for (int tt = 0; tt < 32; ++tt) {
+            if (tl0 + tt < n) lastv = pr[tt];
+            else pr[tt] = lastv;
+        }
+        if (hh == 0) part[i] = lastv;
+        named_bar(kBarK, kGroup);
+        carry = hh ? part[i] : 1.f;
+    }
+    const unsigned short *kt = reinterpret_cast<const unsigned short *>(c.sm + OFF_KT);
+    const unsigned short *qt = reinterpret_cast<const unsigned short *>(c.sm + OFF_QT);
+#pragma unroll
+    for (int tt = 0; tt < 32; ++tt) {
+        const bool valid = tl0 + tt < n;
+        const float g = carry * pr[tt];
+        const uint32_t o = fb + tt * 128 + sw.o[tt & 7];
+        const uint32_t oh = hb + tt * 128 + swh.o[tt & 7];
+        const float kk = valid ? __uint_as_float((uint32_t)kt[oh >> 1] << 16) : 0.f;
+        const float qq = valid ? __uint_as_float((uint32_t)qt[oh >> 1] << 16) : 0.f;
+        const float bb = at(c, OFF_BT + o);
+        at(c, OFF_BT + o) = to_tf32(bb * kk * g);
+        at(c, OFF_AT + o) = to_tf32(qq * g);
+        at(c, OFF_KG + o) = to_tf32(__fdividef(kk, g));
+    }
+    if (hh == 1) r.gn[i] = carry * pr[31];
+    if (el) {
+        r.t0 = t0;
+        r.n = n;
+        r.last = (t0 + n >= te) ? 1 : 0;
+    }
+    return n;
 }
 
-// Gate prep proper (after prep_decay and a group barrier).
-template <bool kFull>
-__device__ __forceinline__ void prep(const Ctx &c, uint32_t tlane, uint32_t kt_col, int kb, int qd, int kh,
-                                     int lane, int n) {
-    const int i = 32 * qd + lane;
+// Key side, pass B (thread per token t, channel half ch): the rows of Etil
+// (lanes 0-63) or Qtil (lanes 64-127) of 64 channels into the TMEM operand.
+__device__ __forceinline__ void key_rows(const Ctx &c, uint32_t tmem, int warp, int lane) {
+    const int lq = warp & 3, ch = (warp - 1) >> 2;
+    const int t = 32 * (lq & 1) + lane;
+    const uint32_t src = lq < 2 ? OFF_BT : OFF_AT;
+    const uint32_t tl = tmem + TM_EQ + ((uint32_t)(32 * lq) << 16);
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+        const int a = 2 * ch + blk;
+        float x[32];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const float4 g4 = *reinterpret_cast<const float4 *>(c.sm + src + a * TILE + swz128(t, 16 * m));
+            x[4 * m] = g4.x; x[4 * m + 1] = g4.y; x[4 * m + 2] = g4.z; x[4 * m + 3] = g4.w;
+        }
+        tmem_st32_nowait(tl + 32 * a, x);
+    }
+}
+
+// Key side: Ktil^T of the chunk from KG into Tensor Memory (thread per key
+// channel i and token half, lane i), the A operand of the state update.
+__device__ __forceinline__ void key_kt(const Ctx &c, uint32_t tmem, int warp, int lane) {
+    const int cb = warp & 3, hh = (warp - 1) >> 2;
+    const int i = 32 * cb + lane;
     const Swz sw((i & 31) * 4u);
-    const uint32_t rbase = (i >> 5) * 16384u + kh * 32 * 128;
-    const float *part = fptr(c, OFF_PART);
-    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(c.sm + OFF_QK) + (i >> 5) * 2048 + kh * 1024 + (i & 31);
-    const __nv_bfloat16 *ks = qs + 8192;
-    const float p0 = part[i], p1 = part[128 + i];
-    if (kh == 0) fptr(c, OFF_GN)[kb * 128 + i] = p0 * p1;
-    float g = kh ? p0 : 1.f;
-    float r = 1.f / g;
+    const uint32_t fb = OFF_KG + (uint32_t)cb * TILE + hh * 32 * 128;
+    float x[32];
 #pragma unroll
-    for (int grp = 0; grp < 4; ++grp) {
-        float av[8], bv[8], kt[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const uint32_t o = rbase + (8 * grp + u) * 128 + sw.o[u];
-            av[u] = at(c, OFF_KS + o);
-            bv[u] = at(c, OFF_X1 + o);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int tt = 8 * grp + u;
-            const float a = (kFull || 32 * kh + tt < n) ? clamp_alpha(av[u]) : 1.f;
-            g *= a;
-            r *= __fdividef(1.f, a);
-            const float qq = __bfloat162float(qs[tt * 32]), kk = __bfloat162float(ks[tt * 32]);
-            const uint32_t o = rbase + tt * 128 + sw.o[u];
-            at(c, OFF_X1 + o) = to_tf32(bv[u] * kk * g);
-            at(c, OFF_X1 + o + 64 * 128) = to_tf32(qq * g);          // Qtil rows 64-127, same swizzle phase
-            kt[u] = to_tf32(kk * r);
-            at(c, OFF_KS + o) = kt[u];
-        }
-        tmem_st8_nowait(tlane + kt_col + 32 * kh + 8 * grp, kt);
+    for (int tt = 0; tt < 32; ++tt) x[tt] = at(c, fb + tt * 128 + sw.o[tt & 7]);
+    tmem_st32_nowait(tmem + TM_KH + ((uint32_t)(32 * cb) << 16) + 32 * hh, x);
+}
+
+// The chunk's alpha and b tiles (or q and k) by TMA.
+__device__ __forceinline__ void load_ab(const Ctx &c, const Maps &m, int h, int t0) {
+    const uint32_t fb = c.bar(B_FULL_AB);
+    mbar_expect_tx(fb, TX_AB);
+    for (int a = 0; a < 4; ++a) {
+        tma_load_3d(c.sa + OFF_AT + a * TILE, &m.alpha, 32 * a, h, t0, fb);
+        tma_load_3d(c.sa + OFF_BT + a * TILE, &m.b, 32 * a, h, t0, fb);
+    }
+}
+__device__ __forceinline__ void load_qk(const Ctx &c, const Maps &m, int h, int t0) {
+    const uint32_t fb = c.bar(B_FULL_QK);
+    mbar_expect_tx(fb, TX_QK);
+    for (int a = 0; a < 2; ++a) {
+        tma_load_3d(c.sa + OFF_QT + a * TILE, &m.q, 64 * a, h, t0, fb);
+        tma_load_3d(c.sa + OFF_KT + a * TILE, &m.k, 64 * a, h, t0, fb);
     }
 }
 
 // T = (I + A)^{-1} in FP32, in place in AS (A strictly lower, zero above the
-// diagonal), in two parts.  invert_diag (key side): the 32 x 32 diagonal
-// blocks T_AA, T_BB by forward substitution (right-looking: column j of a block
-// per thread, each step's dependency one FMA).  invert_offdiag (state side,
-// which is otherwise waiting for T): T_BA = -T_BB A_BA T_AA.
+// diagonal).  invert_diag: the 32 x 32 diagonal blocks T_AA, T_BB by forward
+// substitution (column j of a block per thread, each step's dependency one
+// FMA).  invert_offdiag: T_BA = -T_BB A_BA T_AA.
 __device__ __forceinline__ void invert_diag(const Ctx &c, int ktid) {
     float *As = fptr(c, OFF_AS);
     if (ktid < 64) {
@@ -248,12 +355,10 @@ __device__ __forceinline__ void invert_diag(const Ctx &c, int ktid) {
         for (int i = 0; i < 32; ++i) As[(base + i) * LDA + base + j] = x[i];
     }
 }
-// gtid: thread index within the 256-thread group that runs this; bar_id: its barrier.
 __device__ __forceinline__ void invert_offdiag(const Ctx &c, int gtid, uint32_t bar_id) {
     float *As = fptr(c, OFF_AS);
     float *Xs = fptr(c, OFF_XS);
-    // Y = A_BA T_AA (32 x 32), 2 x 2 outputs per thread
-    {
+    {   // Y = A_BA T_AA (32 x 32), 2 x 2 outputs per thread
         const int i = 2 * (gtid >> 4), jj = 2 * (gtid & 15);
         float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 8
@@ -267,8 +372,7 @@ __device__ __forceinline__ void invert_offdiag(const Ctx &c, int gtid, uint32_t 
         *reinterpret_cast<float2 *>(Xs + (i + 1) * LDX + jj) = make_float2(y10, y11);
     }
     named_bar(bar_id, kGroup);
-    // T_BA = -T_BB Y
-    {
+    {   // T_BA = -T_BB Y
         const int i = 2 * (gtid >> 4), jj = 2 * (gtid & 15);
         float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 8
@@ -286,12 +390,12 @@ __device__ __forceinline__ void invert_offdiag(const Ctx &c, int gtid, uint32_t 
 
 // Split 32 values into TF32 hi + lo parts and store both into the [j][t] tiles
 // UH / UL at token t, columns 32 sh .. 32 sh + 31.  hi keeps the top 10
-// mantissa bits (a TF32 value exactly), lo = x - hi is exact in FP32 and
-// below one TF32 unit of x; the tensor core reads lo to TF32 by dropping its
-// low bits, so hi + lo carries x to within 2^-20 of |x|.
+// mantissa bits (a TF32 value exactly), lo = x - hi is exact in FP32 and below
+// one TF32 unit of x; the tensor core reads lo to TF32 by dropping its low
+// bits, so hi + lo carries x to within 2^-20 of |x|.
 __device__ __forceinline__ void store_split_jt(const Ctx &c, const float (&x)[32], int t, int sh) {
     const Swz sw((t & 31) * 4u);
-    const uint32_t base = (t >> 5) * 8192u + sh * 32 * 128;
+    const uint32_t base = (t >> 5) * TILE + sh * 32 * 128;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const uint32_t o = base + j * 128 + sw.o[j & 7];
@@ -301,11 +405,13 @@ __device__ __forceinline__ void store_split_jt(const Ctx &c, const float (&x)[32
     }
 }
 
+// Descriptor offset (16-byte units) of K-step kk (8 TF32 = 32 bytes) in a
+// K-major tile of 64-row blocks: 4 K-steps per 128-byte row, then the next block.
+__device__ __forceinline__ uint32_t kstep(int kk) { return ((kk >> 2) * TILE + (kk & 3) * 32) >> 4; }
+
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
-chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
-                const __nv_bfloat16 *__restrict__ vg, const float *S0, __nv_bfloat16 *__restrict__ o, float *S_T,
-                int T, int H) {
+chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     Ctx c;
     // Align by offsetting the __shared__ array itself (not through an integer
@@ -314,12 +420,22 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
     c.sa = smem_u32(c.sm);
     uint32_t *misc = reinterpret_cast<uint32_t *>(c.sm + OFF_MISC);
     c.abort_flag = misc + 1;
+    c.limit = p.wait_limit;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int head = blockIdx.x >> 1, half = blockIdx.x & 1;
-    const int bidx = head / H, h = head % H;
+    const int unit = blockIdx.x >> 1, half = blockIdx.x & 1;   // unit = sequence * H + head
+    const int seq = unit / p.H, h = unit % p.H;
+    int tb, te;
+    if (p.cu_seqlens) {
+        tb = p.cu_seqlens[seq];
+        te = p.cu_seqlens[seq + 1];
+    } else {
+        tb = seq * p.T;
+        te = tb + p.T;
+    }
+    const bool empty = te <= tb;
     const int col0 = half * kDVS;
-    const int nchunks = (T + kC - 1) / kC;
+    const size_t soff = (size_t)unit * kDK * kDV;
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i) mbar_init(c.bar(i), 1);
@@ -339,324 +455,334 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
     const uint32_t tmem = misc[0];
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        // Each lane finally waits (bounded) for the last copy it issued, so that no copy
-        // into shared memory is still in flight when the CTA ends, also after a give-up.
-        if (lane == 0) {            // alpha -> KS rows 0-63, b -> X1 rows 0-63
-            int last = -1;
-            for (int ck = 0; ck < nchunks; ++ck) {
-                if (ck > 0 && !solo_wait(c, B_X1_FREE, (ck - 1) & 1)) break;
-                const uint32_t fb = c.bar(B_FULL_AB);
-                mbar_expect_tx(fb, TX_AB);
-                last = ck;
-                for (int a = 0; a < 4; ++a) {
-                    tma_load_4d(c.sa + OFF_KS + a * 16384, &maps.alpha, 32 * a, h, ck * kC, bidx, fb);
-                    tma_load_4d(c.sa + OFF_X1 + a * 16384, &maps.b, 32 * a, h, ck * kC, bidx, fb);
-                }
-                if (ck + 1 < nchunks) {     // the next chunk's tiles into L2 while this one is processed
-                    for (int a = 0; a < 4; ++a) {
-                        tma_prefetch_4d(&maps.alpha, 32 * a, h, (ck + 1) * kC, bidx);
-                        tma_prefetch_4d(&maps.b, 32 * a, h, (ck + 1) * kC, bidx);
-                    }
-                    for (int a = 0; a < 2; ++a) tma_prefetch_4d(&maps.w, col0 + 32 * a, h, (ck + 1) * kC, bidx);
-                    tma_prefetch_4d(&maps.v, col0, h, (ck + 1) * kC, bidx);
-                }
-            }
-            if (last >= 0) (void)mbar_wait(c.bar(B_FULL_AB), last & 1, kWaitLimit / 8);
-        } else if (lane == 1) {     // q, k -> QK once the gate prep has consumed the previous chunk's
-            int last = -1;
-            for (int ck = 0; ck < nchunks; ++ck) {
-                if (ck > 0 && !solo_wait(c, B_KPREP, (ck - 1) & 1)) break;
-                const uint32_t fb = c.bar(B_FULL_QK);
-                mbar_expect_tx(fb, TX_QK);
-                last = ck;
-                for (int a = 0; a < 4; ++a) {
-                    tma_load_4d(c.sa + OFF_QK + a * 4096, &maps.q, 32 * a, h, ck * kC, bidx, fb);
-                    tma_load_4d(c.sa + OFF_QK + 16384 + a * 4096, &maps.k, 32 * a, h, ck * kC, bidx, fb);
-                }
-                if (ck + 1 < nchunks)
-                    for (int a = 0; a < 4; ++a) {
-                        tma_prefetch_4d(&maps.q, 32 * a, h, (ck + 1) * kC, bidx);
-                        tma_prefetch_4d(&maps.k, 32 * a, h, (ck + 1) * kC, bidx);
-                    }
-            }
-            if (last >= 0) (void)mbar_wait(c.bar(B_FULL_QK), last & 1, kWaitLimit / 8);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint64_t dX1 = sdesc_sw128(c.sa + OFF_X1, 16, 1024);
-            const uint64_t dKK = sdesc_sw128(c.sa + OFF_KS, 16, 1024);           // Ktil rows
-            const uint64_t dKSt = sdesc_sw128(c.sa + OFF_KS + 8192, 16, 1024);   // S rows
+        // Four streams of work, each in chunk order: the Gram of chunk cg, the X
+        // product of chunk cx, U of chunk cu, the state update and output of chunk
+        // cs.  Whichever has its inputs ready is issued, the state chain first.
+        if (lane == 0 && !empty) {
+            const uint64_t dSC = sdesc_sw128(c.sa + OFF_SC, 16, 1024);
+            const uint64_t dKG = sdesc_sw128(c.sa + OFF_KG, 16, 1024);
             const uint64_t dUH = sdesc_sw128(c.sa + OFF_UH, 16, 1024), dUL = sdesc_sw128(c.sa + OFF_UL, 16, 1024);
             const uint32_t id = idesc_tf32(128, 64, 0, 0);
-            for (int ck = 0; ck < nchunks; ++ck) {
-                const uint32_t ph = ck & 1;
-                const uint32_t kt = tmem + TM_KT + 64 * ph, tp = tmem + TM_TP + 64 * ph;
-                // Gram [Etil; Qtil] Ktil^T
-                if (!solo_wait(c, B_KPREP, ph)) break;
-                tc_fence_after();
+            int cg = 0, cx = 0, cu = 0, cs = 0, lastc = 0x7fffffff;
+            long long t_prog = clock64();
+            while (cs <= lastc) {
+                if (cs < cu && mbar_test(c.bar(B_U_READY), cs & 1) && mbar_test(c.bar(B_KH_READY), cs & 1)) {
+                    // S + Ktil^T (U_hi + U_lo) onto the state;  P U_hi onto TM_X (-> O)
+                    const uint32_t tp = tmem + TM_TP + 64 * (cs & 1);
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const uint32_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                    mma_tf32(tmem + TM_G, dX1 + koff, dKK + koff, id, kk > 0);
-                }
-                mma_commit(c.bar(B_G_FULL));
-                // [Etil; Qtil] S
-                if (!solo_wait(c, B_S_READY, ph)) break;
-                tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk) {
+                        mma_tf32_ts(tmem + TM_S, tmem + TM_KH + 8 * kk, dUH + kstep(kk), id, 1);
+                        mma_tf32_ts(tmem + TM_S, tmem + TM_KH + 8 * kk, dUL + kstep(kk), id, 1);
+                    }
+                    mma_commit(c.bar(B_D_FULL));
+                    mma_commit(c.bar(B_KH_FREE));
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const uint32_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                    mma_tf32(tmem + TM_X, dX1 + koff, dKSt + koff, id, kk > 0);
-                }
-                mma_commit(c.bar(B_X_FULL));
-                mma_commit(c.bar(B_X1_FREE));
-                // U = [T; P] (R_hi + R_lo)
-                if (!solo_wait(c, B_R_READY, ph) || !solo_wait(c, B_TP_READY, ph)) break;
-                tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk) mma_tf32_ts(tmem + TM_X, tp + 8 * kk, dUH + kstep(kk), id, 1);
+                    mma_commit(c.bar(B_O_FULL));
+                    mma_commit(c.bar((cs & 1) ? B_TP_FREE1 : B_TP_FREE0));
+                    ++cs;
+                } else if (cu < cx && mbar_test(c.bar(B_R_READY), cu & 1) &&
+                           mbar_test(c.bar((cu & 1) ? B_TP_READY1 : B_TP_READY0), (cu >> 1) & 1)) {
+                    // U = [T; P] (R_hi + R_lo)
+                    const uint32_t tp = tmem + TM_TP + 64 * (cu & 1);
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                    mma_tf32_ts(tmem + TM_U, tp + 8 * kk, dUH + koff, id, kk > 0);
-                    mma_tf32_ts(tmem + TM_U, tp + 8 * kk, dUL + koff, id, 1);
-                }
-                mma_commit(c.bar(B_U_FULL));
-                // S + Ktil^T (U_hi + U_lo) accumulated onto the state;  then P U_hi onto TM_X
-                if (!solo_wait(c, B_U_READY, ph)) break;
-                tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk) {
+                        mma_tf32_ts(tmem + TM_U, tp + 8 * kk, dUH + kstep(kk), id, kk > 0);
+                        mma_tf32_ts(tmem + TM_U, tp + 8 * kk, dUL + kstep(kk), id, 1);
+                    }
+                    mma_commit(c.bar(B_U_FULL));
+                    ++cu;
+                } else if (cx < cg && mbar_test(c.bar(B_S_READY), cx & 1)) {
+                    // [Etil; Qtil] S
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                    mma_tf32_ts(tmem + TM_S, kt + 8 * kk, dUH + koff, id, 1);
-                    mma_tf32_ts(tmem + TM_S, kt + 8 * kk, dUL + koff, id, 1);
-                }
-                mma_commit(c.bar(B_D_FULL));
+                    for (int kk = 0; kk < 16; ++kk) mma_tf32_ts(tmem + TM_X, tmem + TM_EQ + 8 * kk, dSC + kstep(kk), id, kk > 0);
+                    mma_commit(c.bar(B_X_FULL));
+                    ++cx;
+                } else if (cg <= lastc && mbar_test(c.bar(B_KPREP), cg & 1) &&
+                           (cg < 2 || mbar_test(c.bar((cg & 1) ? B_TP_FREE1 : B_TP_FREE0), ((cg - 2) >> 1) & 1))) {
+                    // Gram [Etil; Qtil] Ktil^T into the chunk's [T; P] buffer
+                    tc_fence_after();
+                    if (rec(c, cg).last) lastc = cg;
+                    const uint32_t tp = tmem + TM_TP + 64 * (cg & 1);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                    mma_tf32_ts(tmem + TM_X, tp + 8 * kk, dUH + koff, id, 1);
+                    for (int kk = 0; kk < 16; ++kk) mma_tf32_ts(tp, tmem + TM_EQ + 8 * kk, dKG + kstep(kk), id, kk > 0);
+                    mma_commit(c.bar(B_G_FULL));
+                    ++cg;
+                } else {
+                    if (*c.abort_flag) break;
+                    if (clock64() - t_prog > c.limit) {
+                        record_abort(c, B_DRAIN);
+                        break;
+                    }
+                    continue;
                 }
-                mma_commit(c.bar(B_O_FULL));
-                mma_commit(c.bar(ph ? B_KT_FREE1 : B_KT_FREE0));     // Ktil^T and [T; P] of this parity
+                t_prog = clock64();
             }
             // Every MMA issued above has completed before Tensor Memory is released (bounded).
             mma_commit(c.bar(B_DRAIN));
-            (void)mbar_wait(c.bar(B_DRAIN), 0, kWaitLimit / 8);
+            (void)mbar_wait(c.bar(B_DRAIN), 0, kDrainLimit);
         }
         __syncwarp();
-    } else if (warp < 10) {
+    } else if (warp <= 8) {
         // ------------------------------------------------ key side
-        const int ktid = tid - 64, qd = warp & 3, kh = (warp - 2) >> 2;
-        const int srow = 32 * qd + lane;
-        const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);
+        const int ktid = tid - 32;
         const bool el = ktid == 0;
-        for (int ck = 0; ck < nchunks; ++ck) {
+        const int lq = warp & 3, ch = (warp - 1) >> 2;
+        const int srow = 32 * lq + lane;                       // TMEM lane in the epilogues
+        const uint32_t tlane = tmem + ((uint32_t)(32 * lq) << 16);
+        int t0 = tb;
+        if (el && !empty) {
+            load_ab(c, maps, h, t0);
+            load_qk(c, maps, h, t0);
+        }
+        int pend_ab = empty ? -1 : 0, pend_qk = pend_ab;   // chunk whose loads are in flight, not yet awaited
+        for (int ck = 0; !empty; ++ck) {
             const uint32_t ph = ck & 1;
-            const int t0 = ck * kC, n = min(kC, T - t0);
+            const int navail = min(kC, te - t0);
+            ChunkRec &r = rec(c, ck);
             if (!group_wait(c, B_FULL_AB, ph, el, kBarK)) break;
-            if (n == kC) prep_decay<true>(c, qd, kh, lane, n);
-            else prep_decay<false>(c, qd, kh, lane, n);
+            pend_ab = -1;
             if (!group_wait(c, B_FULL_QK, ph, el, kBarK)) break;
-            if (ck >= 2 && !group_wait(c, ph ? B_KT_FREE1 : B_KT_FREE0, ((ck - 2) >> 1) & 1, el, kBarK)) break;
-            if (n == kC) prep<true>(c, tlane, TM_KT + 64 * ph, ph, qd, kh, lane, n);
-            else prep<false>(c, tlane, TM_KT + 64 * ph, ph, qd, kh, lane, n);
+            pend_qk = -1;
+            if (el) {
+                *reinterpret_cast<volatile int *>(c.sm + OFF_MISC + 8) = kC;
+                const int tn = t0 + kC;
+                if (tn < te) {      // the next chunk's w, v into L2 for the state side
+                    for (int a = 0; a < 2; ++a) tma_prefetch_3d(&maps.w, col0 + 32 * a, h, tn);
+                    tma_prefetch_3d(&maps.v, col0, h, tn);
+                }
+            }
+            const int n = key_decay(c, warp, lane, t0, navail, te, r, el);
+            const bool last = t0 + n >= te;
+            fence_proxy_async_smem();
+            named_bar(kBarK, kGroup);
+            if (el) {
+                mbar_arrive(c.bar(B_RR0 + (ck & 3)));
+                if (!last) {
+                    load_qk(c, maps, h, t0 + n);       // q, k consumed: the next chunk's
+                    pend_qk = ck + 1;
+                }
+            }
+            // [Etil; Qtil] into Tensor Memory once the previous X product has read it
+            if (ck >= 1 && !group_wait(c, B_X_FULL, (ck - 1) & 1, el, kBarK)) break;
+            key_rows(c, tmem, warp, lane);
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarK, kGroup);
-            if (el) mbar_arrive(c.bar(B_KPREP));
-            // Gram epilogue: A (rows 0-63, strictly lower) -> AS; P (rows 64-127) -> [T; P] operand.
-            // AS is free once the state side has copied out the previous chunk's T.
+            if (el) {
+                mbar_arrive(c.bar(B_KPREP));
+                if (!last) {
+                    load_ab(c, maps, h, t0 + n);       // alpha, b consumed: the next chunk's
+                    pend_ab = ck + 1;
+                }
+            }
+            // Gram epilogue: A (rows 0-63, strictly lower) -> AS; P (rows 64-127) masked in place.
             if (!group_wait(c, B_G_FULL, ph, el, kBarK)) break;
-            if (ck >= 1 && !group_wait(c, B_TP_READY, (ck - 1) & 1, el, kBarK)) break;
             tc_fence_after();
             {
+                const uint32_t tp = tlane + TM_TP + 64 * ph + 32 * ch;
                 float g[32];
-                tmem_ld32(tlane + TM_G + 32 * kh, g);
+                tmem_ld32(tp, g);
                 if (srow < 64) {
                     // The diagonal 32 x 32 blocks are only read strictly below their diagonal and are
                     // then overwritten by T_AA, T_BB; A_BA lies wholly below the diagonal.  Only the
                     // block above the diagonal (rows 0-31, columns 32-63) needs its zeros.
-                    float2 *dst = reinterpret_cast<float2 *>(fptr(c, OFF_AS) + srow * LDA + 32 * kh);
-                    const bool upper = srow < 32 && kh == 1;
+                    float2 *dst = reinterpret_cast<float2 *>(fptr(c, OFF_AS) + srow * LDA + 32 * ch);
+                    const bool upper = srow < 32 && ch == 1;
 #pragma unroll
                     for (int jj = 0; jj < 32; jj += 2)
                         dst[jj >> 1] = upper ? make_float2(0.f, 0.f) : make_float2(g[jj], g[jj + 1]);
                 } else {
                     const int t = srow - 64;
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) g[jj] = (32 * kh + jj <= t) ? to_tf32(g[jj]) : 0.f;
-                    tmem_st32_nowait(tlane + TM_TP + 64 * ph + 32 * kh, g);
+                    for (int jj = 0; jj < 32; ++jj) g[jj] = (32 * ch + jj <= t) ? to_tf32(g[jj]) : 0.f;
+                    tmem_st32_nowait(tp, g);
                 }
             }
             named_bar(kBarK, kGroup);
             invert_diag(c, ktid);
+            named_bar(kBarK, kGroup);
+            invert_offdiag(c, ktid, kBarK);
+            if (srow < 64) {        // AS holds exact zeros above the diagonal of T
+                float tv[32];
+                const float *As = fptr(c, OFF_AS) + srow * LDA + 32 * ch;
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) tv[jj] = to_tf32(As[jj]);
+                tmem_st32_nowait(tlane + TM_TP + 64 * ph + 32 * ch, tv);
+            }
             tmem_wait_st();
             tc_fence_before();
             named_bar(kBarK, kGroup);
-            if (el) mbar_arrive(c.bar(B_DIAG_DONE));
+            if (el) mbar_arrive(c.bar(ph ? B_TP_READY1 : B_TP_READY0));
+            // Ktil^T into Tensor Memory once the previous state update has read it
+            if (ck >= 1 && !group_wait(c, B_KH_FREE, (ck - 1) & 1, el, kBarK)) break;
+            tc_fence_after();
+            key_kt(c, tmem, warp, lane);
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar(kBarK, kGroup);
+            if (el) mbar_arrive(c.bar(B_KH_READY));
+            if (last) break;
+            t0 += n;
         }
+        // No copy into shared memory may still be in flight when the CTA ends (bounded).
+        if (el && pend_ab >= 0) (void)mbar_wait(c.bar(B_FULL_AB), pend_ab & 1, kDrainLimit);
+        if (el && pend_qk >= 0) (void)mbar_wait(c.bar(B_FULL_QK), pend_qk & 1, kDrainLimit);
     } else {
         // ------------------------------------------------ state side
-        const int stid = tid - 320, qd = warp & 3, sh = (warp - 10) >> 2;
-        const int srow = 32 * qd + lane;
-        const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);
+        const int stid = tid - 288, lq = warp & 3, sh = (warp - 9) >> 2;
+        const int srow = 32 * lq + lane;
+        const uint32_t tlane = tmem + ((uint32_t)(32 * lq) << 16);
         const uint32_t ts = tlane + TM_S + 32 * sh;        // this thread's state row, 32 columns
         const bool el = stid == 0;
         const Swz ssw((srow & 31) * 4u);
-        const uint32_t sbase = OFF_KS + (srow >> 5) * 16384u + (64 + 32 * sh) * 128;   // S rows of KS
-        {   // S0 -> Tensor Memory and its TF32 copy
-            float S[32];
-            const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 32 * sh;
+        const uint32_t sbase = OFF_SC + (srow >> 5) * TILE + 32 * sh * 128;   // S[i][j] at [j][i]
+        const size_t srow_off = soff + (size_t)srow * kDV + col0 + 32 * sh;
+        if (empty) {
+            if (p.S_T) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                float4 x = S0 ? *reinterpret_cast<const float4 *>(S0 + off + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-                S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(S[j]);
-            tmem_st32_nowait(ts, S);
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar(kBarS, kGroup);
-        if (el) mbar_arrive(c.bar(B_S_READY));
-        bool done_ok = true;
-        for (int ck = 0; ck < nchunks; ++ck) {
-            const uint32_t ph = ck & 1;
-            const int t0 = ck * kC, n = min(kC, T - t0);
-            // w, v of this thread's token (lanes 0-63) and columns, straight into registers;
-            // the loads complete while the MMA below runs.  Padding tokens read as zero.
-            float4 wr[8];
-            uint4 vr[4];
-            if (srow < 64) {
-                if (srow < n) {
-                    const size_t row = (((size_t)bidx * T + t0 + srow) * H + h) * 128 + col0 + 32 * sh;
-                    const float4 *wp = reinterpret_cast<const float4 *>(wg + row);
-                    const uint4 *vp = reinterpret_cast<const uint4 *>(vg + row);
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) wr[m] = __ldg(wp + m);
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) vr[m] = __ldg(vp + m);
-                } else {
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) wr[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) vr[m] = make_uint4(0u, 0u, 0u, 0u);
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 x = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + srow_off + j)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4 *>(p.S_T + srow_off + j) = x;
                 }
             }
-            // R = w*v - Etil S (lanes 0-63) -> R_hi, R_lo
-            if (!group_wait(c, B_X_FULL, ph, el, kBarS)) { done_ok = false; break; }
-            tc_fence_after();
-            if (srow < 64) {
-                float x[32];
-                tmem_ld32(tlane + TM_X + 32 * sh, x);
+        } else {
+            {   // S0 -> Tensor Memory and its TF32 copy
+                float S[32];
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {                  // columns 32 sh + 8 p .. + 7
-                    const uint4 vb = vr[p];
-                    const float4 w0 = wr[2 * p], w1 = wr[2 * p + 1];
-                    float *xp = x + 8 * p;
-                    xp[0] = w0.x * bf_lo(vb.x) - xp[0];
-                    xp[1] = w0.y * bf_hi(vb.x) - xp[1];
-                    xp[2] = w0.z * bf_lo(vb.y) - xp[2];
-                    xp[3] = w0.w * bf_hi(vb.y) - xp[3];
-                    xp[4] = w1.x * bf_lo(vb.z) - xp[4];
-                    xp[5] = w1.y * bf_hi(vb.z) - xp[5];
-                    xp[6] = w1.z * bf_lo(vb.w) - xp[6];
-                    xp[7] = w1.w * bf_hi(vb.w) - xp[7];
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 x = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + srow_off + j)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                    S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
                 }
-                store_split_jt(c, x, srow, sh);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(kBarS, kGroup);
-            if (el) mbar_arrive(c.bar(B_R_READY));
-            // finish T = (I + A)^{-1} and copy it, TF32, into rows 0-63 of the [T; P] operand
-            if (!group_wait(c, B_DIAG_DONE, ph, el, kBarS)) { done_ok = false; break; }
-            tc_fence_after();
-            invert_offdiag(c, stid, kBarS);
-            if (srow < 64) {        // AS holds exact zeros above the diagonal of T
-                float tv[32];
-                const float *As = fptr(c, OFF_AS) + srow * LDA + 32 * sh;
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) tv[jj] = to_tf32(As[jj]);
-                tmem_st32_nowait(tlane + TM_TP + 64 * ph + 32 * sh, tv);
+                for (int j = 0; j < 32; ++j) at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(S[j]);
+                tmem_st32_nowait(ts, S);
+                tmem_wait_st();
             }
-            tmem_wait_st();
-            tc_fence_before();
-            named_bar(kBarS, kGroup);
-            if (el) mbar_arrive(c.bar(B_TP_READY));
-            // U -> U_hi, U_lo
-            if (!group_wait(c, B_U_FULL, ph, el, kBarS)) { done_ok = false; break; }
-            tc_fence_after();
-            if (srow < 64) {
-                float u[32];
-                tmem_ld32(tlane + TM_U + 32 * sh, u);
-                store_split_jt(c, u, srow, sh);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(kBarS, kGroup);
-            if (el) mbar_arrive(c.bar(B_U_READY));
-            // state S <- gamma_n (S + Ktil^T U), in Tensor Memory, and its TF32 copy
-            if (!group_wait(c, B_D_FULL, ph, el, kBarS)) { done_ok = false; break; }
-            tc_fence_after();
-            {
-                float d[32];
-                tmem_ld32(ts, d);
-                const float gn = fptr(c, OFF_GN)[ph * 128 + srow];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    d[j] *= gn;
-                    at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(d[j]);
-                }
-                tmem_st32_nowait(ts, d);
-            }
-            // outputs: lanes 64-127 of TM_X
-            if (!group_wait(c, B_O_FULL, ph, el, kBarS)) { done_ok = false; break; }
-            tc_fence_after();
-            if (srow >= 64) {
-                float v[32];
-                tmem_ld32(tlane + TM_X + 32 * sh, v);
-                const int t = srow - 64;
-                if (t < n) {
-                    __nv_bfloat16 *dst = o + (((size_t)bidx * T + t0 + t) * H + h) * 128 + col0 + 32 * sh;
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        uint4 pk;
-                        __nv_bfloat162 p0 = __floats2bfloat162_rn(v[j], v[j + 1]);
-                        __nv_bfloat162 p1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
-                        __nv_bfloat162 p2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
-                        __nv_bfloat162 p3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
-                        pk.x = *reinterpret_cast<uint32_t *>(&p0);
-                        pk.y = *reinterpret_cast<uint32_t *>(&p1);
-                        pk.z = *reinterpret_cast<uint32_t *>(&p2);
-                        pk.w = *reinterpret_cast<uint32_t *>(&p3);
-                        *reinterpret_cast<uint4 *>(dst + j) = pk;
-                    }
-                }
-            }
-            tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarS, kGroup);
             if (el) mbar_arrive(c.bar(B_S_READY));
-        }
-        if (done_ok && *c.abort_flag == 0 && S_T) {
-            float S[32];
-            tmem_ld32(ts, S);
-            const size_t off = ((size_t)head * kDK + srow) * 128 + col0 + 32 * sh;
+            bool done_ok = true;
+            for (int ck = 0;; ++ck) {
+                const uint32_t ph = ck & 1;
+                if (!group_wait(c, B_RR0 + (ck & 3), (ck >> 2) & 1, el, kBarS)) { done_ok = false; break; }
+                const ChunkRec &r = rec(c, ck);
+                const int t0 = r.t0, n = r.n;
+                const bool last = r.last != 0;
+                // w, v of this thread's token (lanes 0-63) and columns, straight into registers;
+                // the loads complete while the MMA below runs.  Tokens past the chunk read as zero.
+                float z[32];
+                if (srow < 64) {
+                    if (srow < n) {
+                        const size_t row = ((size_t)(t0 + srow) * p.H + h) * kDV + col0 + 32 * sh;
+                        const float4 *wp = reinterpret_cast<const float4 *>(p.w + row);
+                        const uint4 *vp = reinterpret_cast<const uint4 *>(p.v + row);
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4 *>(S_T + off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                        for (int m = 0; m < 4; ++m) {
+                            const uint4 vb = __ldg(vp + m);
+                            const float4 w0 = __ldg(wp + 2 * m), w1 = __ldg(wp + 2 * m + 1);
+                            float *zp = z + 8 * m;
+                            zp[0] = w0.x * bf_lo(vb.x); zp[1] = w0.y * bf_hi(vb.x);
+                            zp[2] = w0.z * bf_lo(vb.y); zp[3] = w0.w * bf_hi(vb.y);
+                            zp[4] = w1.x * bf_lo(vb.z); zp[5] = w1.y * bf_hi(vb.z);
+                            zp[6] = w1.z * bf_lo(vb.w); zp[7] = w1.w * bf_hi(vb.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) z[j] = 0.f;
+                    }
+                }
+                // R = w*v - Etil S (lanes 0-63) -> R_hi, R_lo
+                if (!group_wait(c, B_X_FULL, ph, el, kBarS)) { done_ok = false; break; }
+                tc_fence_after();
+                if (srow < 64) {
+                    float x[32];
+                    tmem_ld32(tlane + TM_X + 32 * sh, x);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) x[j] = z[j] - x[j];
+                    store_split_jt(c, x, srow, sh);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(kBarS, kGroup);
+                if (el) mbar_arrive(c.bar(B_R_READY));
+                // U -> U_hi, U_lo
+                if (!group_wait(c, B_U_FULL, ph, el, kBarS)) { done_ok = false; break; }
+                tc_fence_after();
+                if (srow < 64) {
+                    float u[32];
+                    tmem_ld32(tlane + TM_U + 32 * sh, u);
+                    store_split_jt(c, u, srow, sh);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(kBarS, kGroup);
+                if (el) mbar_arrive(c.bar(B_U_READY));
+                // state S <- gamma_n (S + Ktil^T U), in Tensor Memory, and its TF32 copy
+                if (!group_wait(c, B_D_FULL, ph, el, kBarS)) { done_ok = false; break; }
+                tc_fence_after();
+                {
+                    float d[32];
+                    tmem_ld32(ts, d);
+                    const float gn = r.gn[srow];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        d[j] *= gn;
+                        at(c, sbase + j * 128 + ssw.o[j & 7]) = to_tf32(d[j]);
+                    }
+                    tmem_st32_nowait(ts, d);
+                }
+                // outputs: lanes 64-127 of TM_X
+                if (!group_wait(c, B_O_FULL, ph, el, kBarS)) { done_ok = false; break; }
+                tc_fence_after();
+                if (srow >= 64) {
+                    float v[32];
+                    tmem_ld32(tlane + TM_X + 32 * sh, v);
+                    const int t = srow - 64;
+                    if (t < n) {
+                        __nv_bfloat16 *dst = p.o + ((size_t)(t0 + t) * p.H + h) * kDV + col0 + 32 * sh;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8) {
+                            uint4 pk;
+                            __nv_bfloat162 p0 = __floats2bfloat162_rn(v[j], v[j + 1]);
+                            __nv_bfloat162 p1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
+                            __nv_bfloat162 p2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
+                            __nv_bfloat162 p3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
+                            pk.x = *reinterpret_cast<uint32_t *>(&p0);
+                            pk.y = *reinterpret_cast<uint32_t *>(&p1);
+                            pk.z = *reinterpret_cast<uint32_t *>(&p2);
+                            pk.w = *reinterpret_cast<uint32_t *>(&p3);
+                            *reinterpret_cast<uint4 *>(dst + j) = pk;
+                        }
+                    }
+                }
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(kBarS, kGroup);
+                if (el) mbar_arrive(c.bar(B_S_READY));
+                if (last) break;
+            }
+            if (done_ok && *c.abort_flag == 0 && p.S_T) {
+                float S[32];
+                tmem_ld32(ts, S);
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(p.S_T + srow_off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            }
         }
     }
 
-    // Every role has finished or given up, and the producer and MMA lanes have seen
-    // their last copy and MMA complete: release Tensor Memory.
+    // Every role has finished or given up, and the MMA lane has seen its last MMA
+    // complete: release Tensor Memory.
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -669,35 +795,43 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ wg,
 // ---------------------------------------------------------------------------
 // Host side: tensor maps (driver entry point fetched through the runtime).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 f = fn.load();
+    if (!f) {
+        void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+            fn.store(f);
+        }
     }
-    return fn;
+    return f;
 }
 
-// [B][T][H][d] tensor; box = {box_d, 1, 64, 1}.
-bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, size_t es, int B, int T, int H, int d,
+// Flat [NT][H][d] tensor; box = {box_d, 1, 64}, rows of 128 bytes swizzled as the MMA tiles are.
+bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, size_t es, long long NT, int H, int d,
               int box_d, bool swizzle) {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es, (cuuint64_t)T * H * d * es};
-    cuuint32_t box[4] = {(cuuint32_t)box_d, 1, (cuuint32_t)kC, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, dt, 4, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)NT};
+    cuuint64_t strides[2] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es};
+    cuuint32_t box[3] = {(cuuint32_t)box_d, 1, (cuuint32_t)kC};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+std::atomic<long long> g_wait_limit{4000000000ll};
+std::atomic<unsigned long long> g_attr_set{0};   // bit d: the shared-memory attribute is set on device d
 
 }  // namespace tc
 
 bool chunk_tc_supported(int dk, int dv, gdn2_dtype dt) { return dk == 128 && dv == 128 && dt == GDN2_BF16; }
+
+void set_wait_limit(long long cycles) { tc::g_wait_limit.store(cycles); }
 
 cudaError_t read_device_error(unsigned int *value, bool clear) {
     cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(unsigned int));
@@ -708,26 +842,47 @@ cudaError_t read_device_error(unsigned int *value, bool clear) {
     return e;
 }
 
+// nseq sequences: of T tokens each (cu_seqlens == nullptr), or packed with
+// device offsets cu_seqlens[0..nseq] into T_total = T tokens.
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const float *b,
-                            const float *w, const float *S0, void *o, float *S_T, int B, int T, int H,
-                            cudaStream_t stream) {
+                            const float *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
+                            const int *cu_seqlens, cudaStream_t stream) {
     using namespace tc;
+    const long long NT = cu_seqlens ? (long long)T : (long long)nseq * T;
+    if (NT <= 0 && !cu_seqlens) return cudaSuccess;
     Maps m;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    if (!make_map(&m.q, q, BF, 2, B, T, H, kDK, 32, false) || !make_map(&m.k, k, BF, 2, B, T, H, kDK, 32, false) ||
-        !make_map(&m.v, v, BF, 2, B, T, H, 128, 64, true) ||
-        !make_map(&m.alpha, alpha, F32, 4, B, T, H, kDK, 32, true) ||
-        !make_map(&m.b, b, F32, 4, B, T, H, kDK, 32, true) || !make_map(&m.w, w, F32, 4, B, T, H, 128, 32, true))
+    const long long NTm = NT > 0 ? NT : 1;
+    if (!make_map(&m.q, q, BF, 2, NTm, H, kDK, 64, true) || !make_map(&m.k, k, BF, 2, NTm, H, kDK, 64, true) ||
+        !make_map(&m.v, v, BF, 2, NTm, H, kDV, 64, false) ||
+        !make_map(&m.alpha, alpha, F32, 4, NTm, H, kDK, 32, true) ||
+        !make_map(&m.b, b, F32, 4, NTm, H, kDK, 32, true) || !make_map(&m.w, w, F32, 4, NTm, H, kDV, 32, false))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (!bit || !(g_attr_set.load() & bit)) {
+        e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        if (bit) g_attr_set.fetch_or(bit);
     }
-    const unsigned grid = 2u * (unsigned)B * (unsigned)H;
-    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(m, w, static_cast<const __nv_bfloat16 *>(v), S0,
-                                                            static_cast<__nv_bfloat16 *>(o), S_T, T, H);
+    Params prm;
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.k = static_cast<const __nv_bfloat16 *>(k);
+    prm.v = static_cast<const __nv_bfloat16 *>(v);
+    prm.alpha = alpha;
+    prm.b = b;
+    prm.w = w;
+    prm.S0 = S0;
+    prm.o = static_cast<__nv_bfloat16 *>(o);
+    prm.S_T = S_T;
+    prm.cu_seqlens = cu_seqlens;
+    prm.T = T;
+    prm.H = H;
+    prm.wait_limit = g_wait_limit.load();
+    const unsigned grid = 2u * (unsigned)nseq * (unsigned)H;
+    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(m, prm);
     return cudaGetLastError();
 }
 

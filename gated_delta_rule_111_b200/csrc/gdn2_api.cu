@@ -7,9 +7,10 @@
 
 namespace gdn2 {
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const float *b,
-                            const float *w, const float *S0, void *o, float *S_T, int B, int T, int H,
-                            cudaStream_t stream);
+                            const float *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
+                            const int *cu_seqlens, cudaStream_t stream);
 bool chunk_tc_supported(int dk, int dv, gdn2_dtype dt);
+void set_wait_limit(long long cycles);
 cudaError_t read_device_error(unsigned int *value, bool clear);
 }  // namespace gdn2
 
@@ -67,7 +68,12 @@ const char *gdn2_status_string(gdn2_status s) {
 
 const char *gdn2_last_error(void) { return g_last_error; }
 
-int gdn2_version(void) { return 100; }
+int gdn2_version(void) { return 200; }
+
+gdn2_status gdn2_set_wait_limit(long long cycles) {
+    gdn2::set_wait_limit(cycles > 0 ? cycles : 4000000000ll);
+    return GDN2_OK;
+}
 
 gdn2_status gdn2_device_error(unsigned int *code, int clear) {
     if (!code) return fail(GDN2_ERR_INVALID_ARG, "%s", "null pointer: code");
@@ -115,7 +121,7 @@ gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const fl
 
     cudaError_t err;
     if (gdn2::chunk_tc_supported(d_k, d_v, dt))
-        err = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, s);
+        err = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, nullptr, s);
     else
         err = gdn2::launch_chunk_simt(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, dt, s);
     return cuda_status(err, "gdn2_chunk_fwd launch");

@@ -29,11 +29,14 @@
  *     Calls are asynchronous on that stream and never synchronise the device.
  *   - Supported head sizes: d_k, d_v in {64, 128}.  Other sizes return
  *     GDN2_ERR_UNSUPPORTED.
- *   - Preconditions (documented, not checked on the device): 0 < alpha <= 1
- *     (values below FLT_MIN are treated as FLT_MIN); b and w are not clamped
- *     (the pages ablate an erase gate in [0, 2]).  For the BF16 tensor-core
- *     prefill, the decay accumulated over one 64-token chunk must satisfy
- *     prod(alpha) >= 1e-34 per key channel (sum of -ln(alpha) <= 78).
+ *   - Preconditions (documented, not checked on the device): 0 <= alpha <= 1;
+ *     b and w are not clamped (the pages ablate an erase gate in [0, 2]).
+ *     Every alpha in [0, 1] is supported, however strong the decay: the
+ *     prefill shortens a chunk wherever the decay accumulated inside it would
+ *     leave the FP32 range of its factors.  Values of alpha below 2^-64 are
+ *     computed as 2^-64 (a decayed state row then keeps less than 2^-64 of its
+ *     old value instead of less than that; the difference is below FP32
+ *     rounding of any quantity of the size of the state).
  *   - Errors: argument problems are detected on the host before any launch and
  *     return GDN2_ERR_INVALID_ARG / GDN2_ERR_UNSUPPORTED with nothing enqueued.
  *     A failed launch returns GDN2_ERR_CUDA; gdn2_last_error() describes it.
@@ -120,6 +123,15 @@ const char *gdn2_last_error(void);
  * work, released its resources and returned; outputs of that call are
  * undefined).  clear != 0 resets the flag. */
 gdn2_status gdn2_device_error(unsigned int *code, int clear);
+
+/* Test hook for the kernels' failure handling.  Every wait inside a kernel
+ * gives up after `cycles` SM clock cycles (default 4e9, about 2 s at the B200's
+ * clock), after which the kernel raises the device-side failure flag (see
+ * gdn2_device_error), skips its remaining work, waits for its in-flight
+ * tensor-core operations, releases its Tensor Memory and returns.  A tiny
+ * value makes the next launches fail on purpose; cycles <= 0 restores the
+ * default.  Process-wide; takes effect at the next launch. */
+gdn2_status gdn2_set_wait_limit(long long cycles);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int gdn2_version(void);
