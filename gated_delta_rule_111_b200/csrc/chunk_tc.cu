@@ -91,7 +91,7 @@ constexpr long long kDrainLimit = 4000000000ll; // ~2 s: end-of-kernel waits for
 //   KG  Ktil[s][i] (TF32, 4 channel blocks): B operand of the Gram (K-major)
 //   SC  S[i][j] as [j][i] (TF32, 4 channel blocks): B operand of the X product
 //   UH  R_hi, later U_hi, as [j][t] (2 token blocks);  UL  R_lo, later U_lo
-//   AS  A, then T in place (FP32 [64][66]);  XS block products (FP32 [32][34])
+//   AS  A, then T in place (FP32 [64][68]);  XS block products (FP32 [32][36])
 constexpr uint32_t TILE = 8192;
 constexpr uint32_t OFF_AT = 0;
 constexpr uint32_t OFF_BT = OFF_AT + 4 * TILE;
@@ -101,7 +101,7 @@ constexpr uint32_t OFF_KG = OFF_KT + 2 * TILE;
 constexpr uint32_t OFF_SC = OFF_KG + 4 * TILE;
 constexpr uint32_t OFF_UH = OFF_SC + 4 * TILE;
 constexpr uint32_t OFF_UL = OFF_UH + 2 * TILE;
-constexpr int LDA = 66, LDX = 34;
+constexpr int LDA = 68, LDX = 36;   // padded row strides (float4-aligned)
 constexpr uint32_t OFF_AS = OFF_UL + 2 * TILE;
 constexpr uint32_t OFF_XS = OFF_AS + 64 * LDA * 4;
 // Per-chunk record handed from the key side to the issuer and the state side.
@@ -111,8 +111,8 @@ struct ChunkRec {
 };
 constexpr int kRecSlots = 4;
 constexpr uint32_t OFF_REC = OFF_XS + 32 * LDX * 4;
-constexpr uint32_t OFF_PART = OFF_REC + kRecSlots * sizeof(ChunkRec);   // float[128]
-constexpr uint32_t OFF_BAR = OFF_PART + 512;                             // mbarriers
+constexpr uint32_t OFF_PART = OFF_REC + kRecSlots * sizeof(ChunkRec);   // float[8][128]
+constexpr uint32_t OFF_BAR = OFF_PART + 4096;                            // mbarriers
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;   // [0] tmem base, [1] abort flag, [2] first cut
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
@@ -205,75 +205,92 @@ __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x <<
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------------------
-// Key side, pass A (thread per key channel i and token half hh; warp w owns
-// channel block w % 4, whose Tensor Memory lanes it may access): decay
+// Key side, pass A: thread (cg, tg) owns key channels 4 cg .. 4 cg + 3 of
+// tokens 8 tg .. 8 tg + 7 (a warp covers one group of 8 tokens, a lane four
+// channels, so every access is one 16-byte piece of a swizzled row).  Decay
 // products from the alpha tile, the chunk length, then in place alpha -> Qtil
 // and b -> Etil, and Ktil into KG.  Tokens past the chunk become padding (no
 // decay, zero rows).  Returns the chunk length n (uniform across the group).
-__device__ __forceinline__ int key_decay(const Ctx &c, int warp, int lane, int t0, int navail, int te,
-                                         ChunkRec &r, bool el) {
-    const int cb = warp & 3, hh = (warp - 1) >> 2;
-    const int i = 32 * cb + lane, tl0 = 32 * hh;
-    const int nv = min(32, max(0, navail - tl0));
-    const Swz sw((i & 31) * 4u);                 // FP32 tiles: byte column of channel i
-    const Swz swh((i & 63) * 2u);                // BF16 tiles
-    const uint32_t fb = (uint32_t)cb * TILE + tl0 * 128;
-    const uint32_t hb = (uint32_t)(i >> 6) * TILE + tl0 * 128;
-    float pr[32];
+__device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int navail, int te, ChunkRec &r, bool el) {
+    const int cg = ktid & 31, tg = ktid >> 5, lane = ktid & 31;
+    const int tl0 = 8 * tg;
+    float p[8][4];
 #pragma unroll
-    for (int tt = 0; tt < 32; ++tt) {
-        const float a = at(c, OFF_AT + fb + tt * 128 + sw.o[tt & 7]);
-        pr[tt] = tt < nv ? fmaxf(a, kGammaMin) : 1.f;
+    for (int u = 0; u < 8; ++u) {
+        const float4 a = *reinterpret_cast<const float4 *>(c.sm + OFF_AT + (cg >> 3) * TILE + swz128(tl0 + u, (cg & 7) * 16));
+        const bool v = tl0 + u < navail;
+        p[u][0] = v ? fmaxf(a.x, kGammaMin) : 1.f;
+        p[u][1] = v ? fmaxf(a.y, kGammaMin) : 1.f;
+        p[u][2] = v ? fmaxf(a.z, kGammaMin) : 1.f;
+        p[u][3] = v ? fmaxf(a.w, kGammaMin) : 1.f;
     }
-    float run = 1.f;
 #pragma unroll
-    for (int tt = 0; tt < 32; ++tt) {
-        run *= pr[tt];
-        pr[tt] = run;
-    }
-    float *part = fptr(c, OFF_PART);
+    for (int u = 1; u < 8; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[u][e] *= p[u - 1][e];
+    float *part = fptr(c, OFF_PART);                // [token group][channel]: product over the group
     int *nfirst = reinterpret_cast<int *>(c.sm + OFF_MISC + 8);
-    if (hh == 0) part[i] = run;
+    *reinterpret_cast<float4 *>(part + tg * kDK + 4 * cg) = make_float4(p[7][0], p[7][1], p[7][2], p[7][3]);
     named_bar(kBarK, kGroup);
-    float carry = hh ? part[i] : 1.f;
-    // first local token whose decay since the chunk start is below the floor
-    int first = 32;
+    float carry[4] = {1.f, 1.f, 1.f, 1.f};
+    for (int g = 0; g < tg; ++g) {
+        const float4 q4 = *reinterpret_cast<const float4 *>(part + g * kDK + 4 * cg);
+        carry[0] *= q4.x; carry[1] *= q4.y; carry[2] *= q4.z; carry[3] *= q4.w;
+    }
+    // first token whose decay since the chunk start is below the floor in any of the four channels
+    int first = 8;
 #pragma unroll
-    for (int tt = 31; tt >= 0; --tt)
-        if (carry * pr[tt] < kGammaMin) first = tt;
-    int cut = first < 32 ? tl0 + first : kC;
+    for (int u = 7; u >= 0; --u)
+        if (fminf(fminf(carry[0] * p[u][0], carry[1] * p[u][1]), fminf(carry[2] * p[u][2], carry[3] * p[u][3])) < kGammaMin)
+            first = u;
+    int cut = first < 8 ? tl0 + first : kC;
     cut = __reduce_min_sync(0xffffffffu, cut);
     if (lane == 0 && cut < kC) atomicMin(nfirst, cut);
     named_bar(kBarK, kGroup);
     const int n = min(navail, *nfirst);
     if (n < navail) {
         // Cut chunk: tokens from n on belong to the next chunk (no decay here).
-        float lastv = 1.f;
 #pragma unroll
-        for (int tt = 0; tt < 32; ++tt) {
-            if (tl0 + tt < n) lastv = pr[tt];
-            else pr[tt] = lastv;
-        }
-        if (hh == 0) part[i] = lastv;
+        for (int u = 0; u < 8; ++u)
+            if (tl0 + u >= n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[u][e] = u ? p[u - 1][e] : 1.f;
+        *reinterpret_cast<float4 *>(part + tg * kDK + 4 * cg) = make_float4(p[7][0], p[7][1], p[7][2], p[7][3]);
         named_bar(kBarK, kGroup);
-        carry = hh ? part[i] : 1.f;
-    }
-    const unsigned short *kt = reinterpret_cast<const unsigned short *>(c.sm + OFF_KT);
-    const unsigned short *qt = reinterpret_cast<const unsigned short *>(c.sm + OFF_QT);
 #pragma unroll
-    for (int tt = 0; tt < 32; ++tt) {
-        const bool valid = tl0 + tt < n;
-        const float g = carry * pr[tt];
-        const uint32_t o = fb + tt * 128 + sw.o[tt & 7];
-        const uint32_t oh = hb + tt * 128 + swh.o[tt & 7];
-        const float kk = valid ? __uint_as_float((uint32_t)kt[oh >> 1] << 16) : 0.f;
-        const float qq = valid ? __uint_as_float((uint32_t)qt[oh >> 1] << 16) : 0.f;
-        const float bb = at(c, OFF_BT + o);
-        at(c, OFF_BT + o) = to_tf32(bb * kk * g);
-        at(c, OFF_AT + o) = to_tf32(qq * g);
-        at(c, OFF_KG + o) = to_tf32(__fdividef(kk, g));
+        for (int e = 0; e < 4; ++e) carry[e] = 1.f;
+        for (int g = 0; g < tg; ++g) {
+            const float4 q4 = *reinterpret_cast<const float4 *>(part + g * kDK + 4 * cg);
+            carry[0] *= q4.x; carry[1] *= q4.y; carry[2] *= q4.z; carry[3] *= q4.w;
+        }
     }
-    if (hh == 1) r.gn[i] = carry * pr[31];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int t = tl0 + u;
+        const uint32_t o32 = (cg >> 3) * TILE + swz128(t, (cg & 7) * 16);
+        const uint32_t o16 = (cg >> 4) * TILE + swz128(t, (cg & 15) * 8);
+        const bool valid = t < n;
+        const uint2 kr = valid ? *reinterpret_cast<const uint2 *>(c.sm + OFF_KT + o16) : make_uint2(0u, 0u);
+        const uint2 qr = valid ? *reinterpret_cast<const uint2 *>(c.sm + OFF_QT + o16) : make_uint2(0u, 0u);
+        const float4 b4 = *reinterpret_cast<const float4 *>(c.sm + OFF_BT + o32);
+        const float kk[4] = {bf_lo(kr.x), bf_hi(kr.x), bf_lo(kr.y), bf_hi(kr.y)};
+        const float qq[4] = {bf_lo(qr.x), bf_hi(qr.x), bf_lo(qr.y), bf_hi(qr.y)};
+        const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+        float e4[4], q4[4], k4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float g = carry[e] * p[u][e];
+            e4[e] = to_tf32(bb[e] * kk[e] * g);
+            q4[e] = to_tf32(qq[e] * g);
+            k4[e] = to_tf32(__fdividef(kk[e], g));
+        }
+        *reinterpret_cast<float4 *>(c.sm + OFF_BT + o32) = make_float4(e4[0], e4[1], e4[2], e4[3]);
+        *reinterpret_cast<float4 *>(c.sm + OFF_AT + o32) = make_float4(q4[0], q4[1], q4[2], q4[3]);
+        *reinterpret_cast<float4 *>(c.sm + OFF_KG + o32) = make_float4(k4[0], k4[1], k4[2], k4[3]);
+    }
+    if (tg == 7)
+        *reinterpret_cast<float4 *>(r.gn + 4 * cg) =
+            make_float4(carry[0] * p[7][0], carry[1] * p[7][1], carry[2] * p[7][2], carry[3] * p[7][3]);
     if (el) {
         r.t0 = t0;
         r.n = n;
@@ -333,57 +350,83 @@ __device__ __forceinline__ void load_qk(const Ctx &c, const Maps &m, int h, int 
     }
 }
 
-// T = (I + A)^{-1} in FP32, in place in AS (A strictly lower, zero above the
-// diagonal).  invert_diag: the 32 x 32 diagonal blocks T_AA, T_BB by forward
-// substitution (column j of a block per thread, each step's dependency one
-// FMA).  invert_offdiag: T_BA = -T_BB A_BA T_AA.
-__device__ __forceinline__ void invert_diag(const Ctx &c, int ktid) {
-    float *As = fptr(c, OFF_AS);
-    if (ktid < 64) {
-        const int base = 32 * (ktid >> 5), j = ktid & 31;
-        float x[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = (i == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int l = 0; l < 31; ++l) {
-            const float xl = x[l];
-#pragma unroll
-            for (int i = l + 1; i < 32; ++i) x[i] = fmaf(-As[(base + i) * LDA + base + l], xl, x[i]);
-        }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) As[(base + i) * LDA + base + j] = x[i];
-    }
-}
-__device__ __forceinline__ void invert_offdiag(const Ctx &c, int gtid, uint32_t bar_id) {
+// T = (I + A)^{-1} in FP32, in place in AS, by the 256 key-side threads (A is
+// strictly lower and AS holds exact zeros on and above its diagonal).  Three
+// levels: the four 16 x 16 diagonal blocks by forward substitution (column j of
+// a block per thread, each step's dependency one FMA); then the 16 x 16 blocks
+// below them, T_10 = -T_11 A_10 T_00, in both 32 x 32 halves; then the 32 x 32
+// block T_BA = -T_BB A_BA T_AA.  Products keep a 1 x 4 or 2 x 4 block of outputs
+// per thread in registers (half the group; the other half's warps share the
+// sub-partitions with the state side's epilogues).
+__device__ __forceinline__ void invert_t(const Ctx &c, int ktid, uint32_t bar_id) {
     float *As = fptr(c, OFF_AS);
     float *Xs = fptr(c, OFF_XS);
-    {   // Y = A_BA T_AA (32 x 32), 2 x 2 outputs per thread
-        const int i = 2 * (gtid >> 4), jj = 2 * (gtid & 15);
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) {
-            const float a0 = As[(32 + i) * LDA + l], a1 = As[(33 + i) * LDA + l];
-            const float2 t = *reinterpret_cast<const float2 *>(As + l * LDA + jj);
-            y00 = fmaf(a0, t.x, y00); y01 = fmaf(a0, t.y, y01);
-            y10 = fmaf(a1, t.x, y10); y11 = fmaf(a1, t.y, y11);
+    if (ktid < 64) {                                         // 16 x 16 diagonal blocks
+        const int base = 16 * (ktid >> 4), j = ktid & 15;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int l = 0; l < 15; ++l) {
+            const float xl = x[l];
+#pragma unroll
+            for (int i = l + 1; i < 16; ++i) x[i] = fmaf(-As[(base + i) * LDA + base + l], xl, x[i]);
         }
-        *reinterpret_cast<float2 *>(Xs + i * LDX + jj) = make_float2(y00, y01);
-        *reinterpret_cast<float2 *>(Xs + (i + 1) * LDX + jj) = make_float2(y10, y11);
+        __syncwarp();                                        // the warp's blocks are read before written
+#pragma unroll
+        for (int i = 0; i < 16; ++i) As[(base + i) * LDA + base + j] = x[i];
     }
     named_bar(bar_id, kGroup);
-    {   // T_BA = -T_BB Y
-        const int i = 2 * (gtid >> 4), jj = 2 * (gtid & 15);
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) {
-            const float a0 = As[(32 + i) * LDA + 32 + l], a1 = As[(33 + i) * LDA + 32 + l];
-            const float2 y = *reinterpret_cast<const float2 *>(Xs + l * LDX + jj);
-            y00 = fmaf(a0, y.x, y00); y01 = fmaf(a0, y.y, y01);
-            y10 = fmaf(a1, y.x, y10); y11 = fmaf(a1, y.y, y11);
+    if (ktid < 128) {                                        // Y = A_10 T_00 in both halves (16 x 16 x 16)
+        const int base = 32 * (ktid >> 6), r = (ktid & 63) >> 2, cq = 4 * (ktid & 3);
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = As[(base + 16 + r) * LDA + base + k];
+            const float4 t = *reinterpret_cast<const float4 *>(As + (base + k) * LDA + base + cq);
+            y.x = fmaf(a, t.x, y.x); y.y = fmaf(a, t.y, y.y); y.z = fmaf(a, t.z, y.z); y.w = fmaf(a, t.w, y.w);
         }
-        *reinterpret_cast<float2 *>(As + (32 + i) * LDA + jj) = make_float2(-y00, -y01);
-        *reinterpret_cast<float2 *>(As + (33 + i) * LDA + jj) = make_float2(-y10, -y11);
+        *reinterpret_cast<float4 *>(Xs + (ktid >> 6) * 16 * LDX + r * LDX + cq) = y;
+    }
+    named_bar(bar_id, kGroup);
+    if (ktid < 128) {                                        // T_10 = -T_11 Y
+        const int base = 32 * (ktid >> 6), r = (ktid & 63) >> 2, cq = 4 * (ktid & 3);
+        const float *Y = Xs + (ktid >> 6) * 16 * LDX;
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = As[(base + 16 + r) * LDA + base + 16 + k];
+            const float4 y = *reinterpret_cast<const float4 *>(Y + k * LDX + cq);
+            z.x = fmaf(a, y.x, z.x); z.y = fmaf(a, y.y, z.y); z.z = fmaf(a, y.z, z.z); z.w = fmaf(a, y.w, z.w);
+        }
+        *reinterpret_cast<float4 *>(As + (base + 16 + r) * LDA + base + cq) = make_float4(-z.x, -z.y, -z.z, -z.w);
+    }
+    named_bar(bar_id, kGroup);
+    const int ri = 2 * (ktid >> 3), ci = 4 * (ktid & 7);     // rows ri, ri + 1; columns ci .. ci + 3
+    if (ktid < 128) {                                        // Y = A_BA T_AA (32 x 32 x 32)
+        float4 y0 = make_float4(0.f, 0.f, 0.f, 0.f), y1 = y0;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float a0 = As[(32 + ri) * LDA + k], a1 = As[(33 + ri) * LDA + k];
+            const float4 t = *reinterpret_cast<const float4 *>(As + k * LDA + ci);
+            y0.x = fmaf(a0, t.x, y0.x); y0.y = fmaf(a0, t.y, y0.y); y0.z = fmaf(a0, t.z, y0.z); y0.w = fmaf(a0, t.w, y0.w);
+            y1.x = fmaf(a1, t.x, y1.x); y1.y = fmaf(a1, t.y, y1.y); y1.z = fmaf(a1, t.z, y1.z); y1.w = fmaf(a1, t.w, y1.w);
+        }
+        *reinterpret_cast<float4 *>(Xs + ri * LDX + ci) = y0;
+        *reinterpret_cast<float4 *>(Xs + (ri + 1) * LDX + ci) = y1;
+    }
+    named_bar(bar_id, kGroup);
+    if (ktid < 128) {                                        // T_BA = -T_BB Y
+        float4 z0 = make_float4(0.f, 0.f, 0.f, 0.f), z1 = z0;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float a0 = As[(32 + ri) * LDA + 32 + k], a1 = As[(33 + ri) * LDA + 32 + k];
+            const float4 y = *reinterpret_cast<const float4 *>(Xs + k * LDX + ci);
+            z0.x = fmaf(a0, y.x, z0.x); z0.y = fmaf(a0, y.y, z0.y); z0.z = fmaf(a0, y.z, z0.z); z0.w = fmaf(a0, y.w, z0.w);
+            z1.x = fmaf(a1, y.x, z1.x); z1.y = fmaf(a1, y.y, z1.y); z1.z = fmaf(a1, y.z, z1.z); z1.w = fmaf(a1, y.w, z1.w);
+        }
+        *reinterpret_cast<float4 *>(As + (32 + ri) * LDA + ci) = make_float4(-z0.x, -z0.y, -z0.z, -z0.w);
+        *reinterpret_cast<float4 *>(As + (33 + ri) * LDA + ci) = make_float4(-z1.x, -z1.y, -z1.z, -z1.w);
     }
     named_bar(bar_id, kGroup);
 }
@@ -408,6 +451,81 @@ __device__ __forceinline__ void store_split_jt(const Ctx &c, const float (&x)[32
 // Descriptor offset (16-byte units) of K-step kk (8 TF32 = 32 bytes) in a
 // K-major tile of 64-row blocks: 4 K-steps per 128-byte row, then the next block.
 __device__ __forceinline__ uint32_t kstep(int kk) { return ((kk >> 2) * TILE + (kk & 3) * 32) >> 4; }
+
+// The MMA issuer (one thread).  Four streams of work, each in chunk order:
+// the Gram of chunk cg, the X product of chunk cx, U of chunk cu, the state
+// update and output of chunk cs.  Whichever has its inputs ready is issued,
+// the state chain first.  A separate function keeps its few live values out of
+// the other roles' register allocation.
+__device__ __noinline__ void issuer_role(const Ctx &c, uint32_t tmem) {
+    // B descriptors as (low, high) halves; the K-step offset is added inside each MMA's asm.
+    const uint64_t dSC = sdesc_sw128(c.sa + OFF_SC, 16, 1024), dKG = sdesc_sw128(c.sa + OFF_KG, 16, 1024);
+    const uint64_t dUH = sdesc_sw128(c.sa + OFF_UH, 16, 1024), dUL = sdesc_sw128(c.sa + OFF_UL, 16, 1024);
+    const uint32_t hi = (uint32_t)(dSC >> 32);      // identical for every tile (layout, SBO, version)
+    const uint32_t sc = (uint32_t)dSC, kg = (uint32_t)dKG, uh = (uint32_t)dUH, ul = (uint32_t)dUL;
+    const uint32_t id = idesc_tf32(128, 64, 0, 0);
+    int cg = 0, cx = 0, cu = 0, cs = 0, lastc = 0x7fffffff;
+    long long t_prog = clock64();
+    while (cs <= lastc) {
+        if (cs < cu && mbar_test(c.bar(B_U_READY), cs & 1) && mbar_test(c.bar(B_KH_READY), cs & 1)) {
+            // S + Ktil^T (U_hi + U_lo) onto the state;  P U_hi onto TM_X (-> O)
+            const uint32_t tp = tmem + TM_TP + 64 * (cs & 1);
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_tf32_ts_off(tmem + TM_S, tmem + TM_KH + 8 * kk, uh, hi, kstep(kk), id, 1);
+                mma_tf32_ts_off(tmem + TM_S, tmem + TM_KH + 8 * kk, ul, hi, kstep(kk), id, 1);
+            }
+            mma_commit(c.bar(B_D_FULL));
+            mma_commit(c.bar(B_KH_FREE));
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) mma_tf32_ts_off(tmem + TM_X, tp + 8 * kk, uh, hi, kstep(kk), id, 1);
+            mma_commit(c.bar(B_O_FULL));
+            mma_commit(c.bar((cs & 1) ? B_TP_FREE1 : B_TP_FREE0));
+            ++cs;
+        } else if (cu < cx && mbar_test(c.bar(B_R_READY), cu & 1) &&
+                   mbar_test(c.bar((cu & 1) ? B_TP_READY1 : B_TP_READY0), (cu >> 1) & 1)) {
+            // U = [T; P] (R_hi + R_lo)
+            const uint32_t tp = tmem + TM_TP + 64 * (cu & 1);
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_tf32_ts_off(tmem + TM_U, tp + 8 * kk, uh, hi, kstep(kk), id, kk > 0);
+                mma_tf32_ts_off(tmem + TM_U, tp + 8 * kk, ul, hi, kstep(kk), id, 1);
+            }
+            mma_commit(c.bar(B_U_FULL));
+            ++cu;
+        } else if (cx < cg && mbar_test(c.bar(B_S_READY), cx & 1)) {
+            // [Etil; Qtil] S
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) mma_tf32_ts_off(tmem + TM_X, tmem + TM_EQ + 8 * kk, sc, hi, kstep(kk), id, kk > 0);
+            mma_commit(c.bar(B_X_FULL));
+            ++cx;
+        } else if (cg <= lastc && mbar_test(c.bar(B_KPREP), cg & 1) &&
+                   (cg < 2 || mbar_test(c.bar((cg & 1) ? B_TP_FREE1 : B_TP_FREE0), ((cg - 2) >> 1) & 1))) {
+            // Gram [Etil; Qtil] Ktil^T into the chunk's [T; P] buffer
+            tc_fence_after();
+            if (rec(c, cg).last) lastc = cg;
+            const uint32_t tp = tmem + TM_TP + 64 * (cg & 1);
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) mma_tf32_ts_off(tp, tmem + TM_EQ + 8 * kk, kg, hi, kstep(kk), id, kk > 0);
+            mma_commit(c.bar(B_G_FULL));
+            ++cg;
+        } else {
+            if (*c.abort_flag) break;
+            if (clock64() - t_prog > c.limit) {
+                record_abort(c, B_DRAIN);
+                break;
+            }
+            continue;
+        }
+        t_prog = clock64();
+    }
+    // Every MMA issued above has completed before Tensor Memory is released (bounded).
+    mma_commit(c.bar(B_DRAIN));
+    (void)mbar_wait(c.bar(B_DRAIN), 0, kDrainLimit);
+}
 
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
@@ -456,76 +574,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
 
     if (warp == 0) {
         // ------------------------------------------------ MMA issuer
-        // Four streams of work, each in chunk order: the Gram of chunk cg, the X
-        // product of chunk cx, U of chunk cu, the state update and output of chunk
-        // cs.  Whichever has its inputs ready is issued, the state chain first.
-        if (lane == 0 && !empty) {
-            const uint64_t dSC = sdesc_sw128(c.sa + OFF_SC, 16, 1024);
-            const uint64_t dKG = sdesc_sw128(c.sa + OFF_KG, 16, 1024);
-            const uint64_t dUH = sdesc_sw128(c.sa + OFF_UH, 16, 1024), dUL = sdesc_sw128(c.sa + OFF_UL, 16, 1024);
-            const uint32_t id = idesc_tf32(128, 64, 0, 0);
-            int cg = 0, cx = 0, cu = 0, cs = 0, lastc = 0x7fffffff;
-            long long t_prog = clock64();
-            while (cs <= lastc) {
-                if (cs < cu && mbar_test(c.bar(B_U_READY), cs & 1) && mbar_test(c.bar(B_KH_READY), cs & 1)) {
-                    // S + Ktil^T (U_hi + U_lo) onto the state;  P U_hi onto TM_X (-> O)
-                    const uint32_t tp = tmem + TM_TP + 64 * (cs & 1);
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        mma_tf32_ts(tmem + TM_S, tmem + TM_KH + 8 * kk, dUH + kstep(kk), id, 1);
-                        mma_tf32_ts(tmem + TM_S, tmem + TM_KH + 8 * kk, dUL + kstep(kk), id, 1);
-                    }
-                    mma_commit(c.bar(B_D_FULL));
-                    mma_commit(c.bar(B_KH_FREE));
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) mma_tf32_ts(tmem + TM_X, tp + 8 * kk, dUH + kstep(kk), id, 1);
-                    mma_commit(c.bar(B_O_FULL));
-                    mma_commit(c.bar((cs & 1) ? B_TP_FREE1 : B_TP_FREE0));
-                    ++cs;
-                } else if (cu < cx && mbar_test(c.bar(B_R_READY), cu & 1) &&
-                           mbar_test(c.bar((cu & 1) ? B_TP_READY1 : B_TP_READY0), (cu >> 1) & 1)) {
-                    // U = [T; P] (R_hi + R_lo)
-                    const uint32_t tp = tmem + TM_TP + 64 * (cu & 1);
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        mma_tf32_ts(tmem + TM_U, tp + 8 * kk, dUH + kstep(kk), id, kk > 0);
-                        mma_tf32_ts(tmem + TM_U, tp + 8 * kk, dUL + kstep(kk), id, 1);
-                    }
-                    mma_commit(c.bar(B_U_FULL));
-                    ++cu;
-                } else if (cx < cg && mbar_test(c.bar(B_S_READY), cx & 1)) {
-                    // [Etil; Qtil] S
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 16; ++kk) mma_tf32_ts(tmem + TM_X, tmem + TM_EQ + 8 * kk, dSC + kstep(kk), id, kk > 0);
-                    mma_commit(c.bar(B_X_FULL));
-                    ++cx;
-                } else if (cg <= lastc && mbar_test(c.bar(B_KPREP), cg & 1) &&
-                           (cg < 2 || mbar_test(c.bar((cg & 1) ? B_TP_FREE1 : B_TP_FREE0), ((cg - 2) >> 1) & 1))) {
-                    // Gram [Etil; Qtil] Ktil^T into the chunk's [T; P] buffer
-                    tc_fence_after();
-                    if (rec(c, cg).last) lastc = cg;
-                    const uint32_t tp = tmem + TM_TP + 64 * (cg & 1);
-#pragma unroll
-                    for (int kk = 0; kk < 16; ++kk) mma_tf32_ts(tp, tmem + TM_EQ + 8 * kk, dKG + kstep(kk), id, kk > 0);
-                    mma_commit(c.bar(B_G_FULL));
-                    ++cg;
-                } else {
-                    if (*c.abort_flag) break;
-                    if (clock64() - t_prog > c.limit) {
-                        record_abort(c, B_DRAIN);
-                        break;
-                    }
-                    continue;
-                }
-                t_prog = clock64();
-            }
-            // Every MMA issued above has completed before Tensor Memory is released (bounded).
-            mma_commit(c.bar(B_DRAIN));
-            (void)mbar_wait(c.bar(B_DRAIN), 0, kDrainLimit);
-        }
+        if (lane == 0 && !empty) issuer_role(c, tmem);
         __syncwarp();
     } else if (warp <= 8) {
         // ------------------------------------------------ key side
@@ -556,7 +605,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                     tma_prefetch_3d(&maps.v, col0, h, tn);
                 }
             }
-            const int n = key_decay(c, warp, lane, t0, navail, te, r, el);
+            const int n = key_decay(c, ktid, t0, navail, te, r, el);
             const bool last = t0 + n >= te;
             fence_proxy_async_smem();
             named_bar(kBarK, kGroup);
@@ -588,15 +637,14 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                 const uint32_t tp = tlane + TM_TP + 64 * ph + 32 * ch;
                 float g[32];
                 tmem_ld32(tp, g);
-                if (srow < 64) {
-                    // The diagonal 32 x 32 blocks are only read strictly below their diagonal and are
-                    // then overwritten by T_AA, T_BB; A_BA lies wholly below the diagonal.  Only the
-                    // block above the diagonal (rows 0-31, columns 32-63) needs its zeros.
-                    float2 *dst = reinterpret_cast<float2 *>(fptr(c, OFF_AS) + srow * LDA + 32 * ch);
-                    const bool upper = srow < 32 && ch == 1;
+                if (srow < 64) {      // A strictly lower; exact zeros on and above the diagonal
+                    float4 *dst = reinterpret_cast<float4 *>(fptr(c, OFF_AS) + srow * LDA + 32 * ch);
 #pragma unroll
-                    for (int jj = 0; jj < 32; jj += 2)
-                        dst[jj >> 1] = upper ? make_float2(0.f, 0.f) : make_float2(g[jj], g[jj + 1]);
+                    for (int jj = 0; jj < 32; jj += 4) {
+                        const int s0 = 32 * ch + jj;
+                        dst[jj >> 2] = make_float4(s0 < srow ? g[jj] : 0.f, s0 + 1 < srow ? g[jj + 1] : 0.f,
+                                                   s0 + 2 < srow ? g[jj + 2] : 0.f, s0 + 3 < srow ? g[jj + 3] : 0.f);
+                    }
                 } else {
                     const int t = srow - 64;
 #pragma unroll
@@ -605,10 +653,8 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                 }
             }
             named_bar(kBarK, kGroup);
-            invert_diag(c, ktid);
-            named_bar(kBarK, kGroup);
-            invert_offdiag(c, ktid, kBarK);
-            if (srow < 64) {        // AS holds exact zeros above the diagonal of T
+            invert_t(c, ktid, kBarK);
+            if (srow < 64) {        // AS holds exact zeros above the diagonal of T (TF32 copy)
                 float tv[32];
                 const float *As = fptr(c, OFF_AS) + srow * LDA + 32 * ch;
 #pragma unroll
