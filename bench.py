@@ -56,25 +56,39 @@ def prefill_bytes(B, T, H, dk, dv):
 
 
 def prefill_mma_flops(B, T, H, dk=128, dv=128, C=64):
-    """Tensor-core FLOPs one tensor-core prefill launch executes (TF32 MMAs as issued:
-    per CTA = (batch, head, d_v/2 columns) and chunk: Gram [Etil;Qtil]Ktil^T 2C x C x dk,
-    [Etil;Qtil]S 2C x dv/2 x dk, U = [T;P](R_hi + R_lo) 2 x 2C x dv/2 x C, state update
-    Ktil^T(U_hi + U_lo) 2 x dk x dv/2 x C, P U_hi 2C x dv/2 x C)."""
+    """Tensor-core FLOPs one tensor-core prefill launch issues (TF32 MMAs, M = 128, N = 64,
+    as issued per CTA = (batch, head, d_v/2 columns) and chunk: Gram [Etil;Qtil]Ktil^T
+    2C x C x dk, [Etil;Qtil]S 2C x dv/2 x dk, U = [T;P](R_hi + R_lo) 2 x 2C x dv/2 x C,
+    state update Ktil^T(U_hi + U_lo) 2 x dk x dv/2 x C, output [T;P] U_hi 2C x dv/2 x C)."""
     n = dv // 2
     macs = 2 * C * C * dk + 2 * C * n * dk + 2 * (2 * C * n * C) + 2 * (dk * n * C) + 2 * C * n * C
     chunks = -(-T // C)
     return 2 * macs * chunks * 2 * B * H
 
 
+def prefill_algorithmic_flops(B, T, H, dk=128, dv=128, C=64):
+    """FLOPs of the chunkwise method itself, counting each triangle once: per chunk of C
+    tokens and head, A and P (C^2 dk together), [Etil;Qtil] S (2 C dk dv), T R and P U
+    (C(C+1)/2 dv each), Ktil^T U (C dk dv) and the triangular inversion (C^3 / 6) --
+    about 1.33e5 FLOP per token and head at d = 128, 3.5e10 per launch of the 4K workload."""
+    macs = C * C * dk + 2 * C * dk * dv + C * (C + 1) * dv + C * dk * dv + C ** 3 / 6
+    return 2 * macs * (T / C) * B * H
+
+
 TF32_PER_BF16 = 1.1 / 2.25       # nominal dense TF32 / BF16 tensor rates on B200
 
 
-def measured_tensor_peak():
+def measured_bf16_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
-            return float(json.load(f)["bf16_tflops"]) * TF32_PER_BF16, "measured bf16 burst x nominal tf32/bf16"
-    return 1590.0 * TF32_PER_BF16, "fallback bf16 x nominal tf32/bf16"
+            return float(json.load(f)["bf16_tflops"]), "measured bf16 dense burst (cuBLAS)"
+    return 1590.0, "fallback bf16 dense burst"
+
+
+def measured_tensor_peak():
+    bf, src = measured_bf16_peak()
+    return bf * TF32_PER_BF16, src + " x nominal tf32/bf16"
 
 
 def decode_bytes(B, H, dk, dv):
@@ -157,6 +171,44 @@ def oracle_tokens_per_s(budget_s=12.0, max_heads=None):
     desc = (f"oracle FP64 on {heads} heads x {Ts} tokens (d=128) of the prefill workload"
             f"{f', repeated {reps}x' if reps > 1 else ''}, {dt:.1f} s")
     return value, threads, desc, dt
+
+
+def oracle_decode_state_gbs(budget_s=4.0):
+    """The FP64 oracle's decode step on a bounded sample of the decode workload: as many
+    of its (batch, head) states as fill ``budget_s`` of repeated steps, reported in the
+    decode metric's unit (GB of FP32 state read and written per second)."""
+    import oracle
+    D = DECODE
+    threads = oracle.num_threads()
+    heads = max(threads, 16)
+    x = gi.decode_inputs(1, 1, heads, D["dk"], D["dv"], dtype="bf16", seed=3, s0_std=0.02)
+    S = x["S0"].astype(np.float64)
+    args = [x[n][0] for n in ("q", "k", "v", "alpha", "b", "w")]
+    reps, dt = 0, 0.0
+    t0 = time.perf_counter()
+    while reps == 0 or dt < budget_s:
+        _, S = oracle.gdn2_step(*args, S)
+        reps += 1
+        dt = time.perf_counter() - t0
+    gbs = state_bytes(1, heads, D["dk"], D["dv"]) * reps / dt / 1e9
+    return gbs, threads, f"oracle FP64 decode step on {heads} heads (d=128), {reps} steps, {dt:.1f} s"
+
+
+def oracle_long_tokens_per_s(budget_s=4.0):
+    """The FP64 oracle on a bounded sample of the long ragged workload (its 16 heads over
+    the first tokens, with S0), in tokens of H heads per second."""
+    import oracle
+    L = LONG
+    threads = oracle.num_threads()
+    Ts = 256
+    x = gi.chunk_inputs(1, Ts, L["H"], L["dk"], L["dv"], dtype="bf16", seed=0, s0_std=0.02)
+    reps, dt = 0, 0.0
+    t0 = time.perf_counter()
+    while reps == 0 or dt < budget_s:
+        oracle.gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], x["S0"])
+        reps += 1
+        dt = time.perf_counter() - t0
+    return Ts * reps / dt, threads, f"oracle FP64 on the 16 heads x {Ts} tokens, {reps}x, {dt:.1f} s"
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -372,6 +424,16 @@ def run_long(args, torch, dist, g, world, rank, dev, stream):
     return ms
 
 
+def bench_config(world):
+    """The workload description both arms print (the reference arm times the same workload)."""
+    B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
+    return {"workload": "GDN-2 chunkwise prefill B=4 T=4096 H=16 d_k=d_v=128 chunk=64, S0=0",
+            "global_batch": B * world, "seq_len": T, "heads": H, "d_k": dk, "d_v": dv,
+            "dtypes": "q/k/v/o bf16, alpha/b/w fp32, state fp32, fp32 accumulation",
+            "l2": "inputs (675 MB per call) larger than the 126 MB L2; no flush",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 def _num(x):
     return None if x != x else x      # NaN (workload not run) -> null
 
@@ -391,41 +453,51 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=fl
     traffic = load_traffic()
     tflops = prefill_mma_flops(B, T, H, dk, dv) / (ms_step / 1e3) / 1e12
     tpeak, tsrc = measured_tensor_peak()
+    algo_flops = prefill_algorithmic_flops(B, T, H, dk, dv)
+    atflops = algo_flops / (ms_step / 1e3) / 1e12
+    bpeak, bsrc = measured_bf16_peak()
 
-    cpu = None
+    cpu = dec_cpu = long_cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc, _ = oracle_tokens_per_s(budget_s=args.cpu_budget)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        v, cores, desc = oracle_decode_state_gbs()
+        dec_cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+        v, cores, desc = oracle_long_tokens_per_s()
+        long_cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": _num(value), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": _num(ms_step), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; recipe in gdn2_inputs.py)",
-            "config": {"workload": "GDN-2 chunkwise prefill B=4 T=4096 H=16 d_k=d_v=128 chunk=64, S0=0",
-                       "global_batch": B * world, "seq_len": T, "heads": H, "d_k": dk, "d_v": dv,
-                       "dtypes": "q/k/v/o bf16, alpha/b/w fp32, state fp32, fp32 accumulation",
-                       "l2": "inputs (675 MB per call) larger than the 126 MB L2; no flush",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "config": bench_config(world),
             "e2e": {"value": _num(job_tokens_per_s(B, T, world, e2e_ms)), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": _num(e2e_ms)},
             "roofline": {"bound": "hbm", "achieved": _num(pre_gbs), "peak": hbm, "unit": "GB/s",
                          "frac": _num(pre_gbs / hbm), "traffic": traffic.get("gdn2_chunk"),
                          "kernel": "gdn2 chunkwise prefill", "algorithmic_bytes_per_launch": pre_bytes,
                          "peak_source": f"{hbm_src} HBM copy bandwidth", "frac_of_8TBps": _num(pre_gbs / 8000.0)},
-            "tensor_secondary": {"achieved": _num(tflops), "peak": tpeak, "unit": "TFLOP/s", "dtype": "tf32",
-                                 "frac": _num(tflops / tpeak), "flops_per_launch": prefill_mma_flops(B, T, H, dk, dv),
-                                 "peak_source": tsrc},
+            "tensor": {"achieved": _num(atflops), "peak": bpeak, "unit": "TFLOP/s", "frac": _num(atflops / bpeak),
+                       "flops_per_launch": algo_flops, "peak_source": bsrc,
+                       "note": "algorithmic FLOPs of the chunkwise method over the measured launch time, "
+                               "against the dense BF16 peak"},
+            "tensor_issued_tf32": {"achieved": _num(tflops), "peak": tpeak, "unit": "TFLOP/s",
+                                   "frac": _num(tflops / tpeak), "flops_per_launch": prefill_mma_flops(B, T, H, dk, dv),
+                                   "peak_source": tsrc,
+                                   "note": "TF32 MMA FLOPs as issued (split operands and the per-CTA key side counted)"},
             "decode": {"metric": "GDN-2 decode state GB/s @B256 H16 d128", "value": _num(st_gbs), "unit": "GB/s",
                        "us_per_step": _num(dec_ms * 1e3), "steps": steps_d * reps,
                        "roofline": {"bound": "hbm", "achieved": _num(dec_gbs), "peak": hbm, "unit": "GB/s",
                                     "frac": _num(dec_gbs / hbm), "traffic": traffic.get("gdn2_decode"),
                                     "algorithmic_bytes_per_launch": dec_bytes,
-                                    "frac_of_8TBps": _num(dec_gbs / 8000.0)}},
+                                    "frac_of_8TBps": _num(dec_gbs / 8000.0)},
+                       "cpu_baseline": dec_cpu},
             "long_ragged": {"workload": "B=1 T=65573 H=16 d_k=d_v=128, S0 != 0 (ragged last chunk)",
                             "ms_per_call": _num(long_ms),
                             "tokens_per_s": _num(LONG["B"] * LONG["T"] * world / (long_ms / 1e3)),
-                            "note": "latency bound: 32 CTAs walk 1,025 chunks each; reported, no target"},
+                            "note": "latency bound: 32 CTAs walk 1,025 chunks each; reported, no target",
+                            "cpu_baseline": long_cpu},
             "gpu_launches": args.steps,
             "clocks": clk.summary() if clk is not None else None,
             "cpu_baseline": cpu,
@@ -474,8 +546,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": statistics.median(secs) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": "GDN-2 chunkwise prefill B=4 T=4096 H=16 d_k=d_v=128 chunk=64, S0=0",
-                       "global_batch": PREFILL["B"], "seq_len": PREFILL["T"]},
+            "config": bench_config(world),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": descs[-1]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -62,10 +62,31 @@ def test_job_value_scales_with_ranks(capsys):
     assert four["n_gpus"] == 4 and four["config"]["global_batch"] == 4 * bench.PREFILL["B"]
 
 
-def test_tensor_secondary(capsys):
+def test_tensor_issued_tf32(capsys):
     d = _line(capsys, ms=0.5)
-    t = d["tensor_secondary"]
-    # 4.72 M MACs per CTA and chunk; 128 CTAs x 64 chunks for B=4, T=4096, H=16
+    t = d["tensor_issued_tf32"]
+    # 72 TF32 MMAs of M128 N64 K8 = 4.72 M MACs per CTA and chunk; 128 CTAs x 64 chunks
     assert t["flops_per_launch"] == 2 * 4_718_592 * 64 * 128
     assert t["achieved"] == pytest.approx(t["flops_per_launch"] / 0.5e-3 / 1e12)
-    assert t["frac"] == pytest.approx(t["achieved"] / t["peak"]) and t["dtype"] == "tf32"
+    assert t["frac"] == pytest.approx(t["achieved"] / t["peak"])
+
+
+def test_tensor_algorithmic_against_bf16_peak(capsys):
+    """Tensor-pipe utilisation: the method's own FLOPs (each triangle counted once) over
+    the launch time, against the dense BF16 peak."""
+    d = _line(capsys, ms=0.5)
+    t = d["tensor"]
+    C, dk, dv = 64, 128, 128
+    per_chunk_macs = C * C * dk + 2 * C * dk * dv + C * (C + 1) * dv + C * dk * dv + C ** 3 / 6
+    assert per_chunk_macs == pytest.approx(4_246_186.67, rel=1e-9)
+    P = bench.PREFILL
+    assert t["flops_per_launch"] == pytest.approx(2 * per_chunk_macs * (P["T"] / C) * P["B"] * P["H"])
+    assert 3.4e10 < t["flops_per_launch"] < 3.6e10
+    assert t["achieved"] == pytest.approx(t["flops_per_launch"] / 0.5e-3 / 1e12)
+    assert t["frac"] == pytest.approx(t["achieved"] / t["peak"])
+    assert "bf16" in t["peak_source"]
+
+
+def test_reference_arm_prints_the_same_config():
+    assert bench.bench_config(1)["workload"] == bench.bench_config(2)["workload"]
+    assert set(bench.bench_config(1)) >= {"workload", "global_batch", "seq_len", "heads", "d_k", "d_v", "dtypes"}
