@@ -7,6 +7,8 @@ device these functions raise.
 
 Functions (same names as the C ABI):
   gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, ...)  -> (o, S_T)   chunkwise prefill
+  gdn2_chunk_fwd_varlen(q, k, v, alpha, b, w, cu_seqlens, S0=None, ...)
+                                                      -> (o, S_T)   packed variable-length batch
   gdn2_recurrent_step(q, k, v, alpha, b, w, S, ...)   -> o          in-place decode step
 """
 from __future__ import annotations
@@ -19,7 +21,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_recurrent_step", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_recurrent_step", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
            "load_library", "exported_symbols",
            "GDN2_OK", "GDN2_ERR_INVALID_ARG", "GDN2_ERR_UNSUPPORTED", "GDN2_ERR_CUDA", "Gdn2Error"]
 
@@ -52,6 +54,8 @@ def load_library(rebuild_if_stale: bool = True) -> ctypes.CDLL:
     vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
     lib.gdn2_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp]
     lib.gdn2_chunk_fwd.restype = i
+    lib.gdn2_chunk_fwd_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, i, fp, vp, fp, i, i, i, i, i, vp]
+    lib.gdn2_chunk_fwd_varlen.restype = i
     lib.gdn2_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn2_recurrent_step.restype = i
     lib.gdn2_status_string.argtypes = [i]
@@ -151,6 +155,43 @@ def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, *, o=None, S_T=None, output_fi
     with torch.cuda.device(dev):
         _check(lib.gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
                                   _ptr(S_T), B, T, H, dk, dv, code, _stream(stream, dev)))
+    return o, S_T
+
+
+def gdn2_chunk_fwd_varlen(q, k, v, alpha, b, w, cu_seqlens, S0=None, *, o=None, S_T=None,
+                          output_final_state=True, stream=None):
+    """Chunkwise prefill of a packed batch.  q,k [T,H,dk], v [T,H,dv] (bf16 or fp32); alpha,b
+    [T,H,dk], w [T,H,dv] fp32; cu_seqlens int32 [N+1] on the same device (sequence n is rows
+    cu_seqlens[n] .. cu_seqlens[n+1]-1); S0 [N,H,dk,dv] fp32 or None.  Returns (o [T,H,dv],
+    S_T [N,H,dk,dv] or None)."""
+    lib = load_library()
+    if q.device.type != "cuda":
+        raise ValueError("gdn2_chunk_fwd_varlen needs CUDA tensors (there is no CPU implementation)")
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("q", q, dk), ("k", k, dk), ("v", v, dv)):
+        _need(t, name, dt, (T, H, d), dev)
+    for name, t, d in (("alpha", alpha, dk), ("b", b, dk), ("w", w, dv)):
+        _need(t, name, torch.float32, (T, H, d), dev)
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens: expected a 1-D tensor of N + 1 offsets")
+    N = cu_seqlens.numel() - 1
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=dt, device=dev)
+    else:
+        _need(o, "o", dt, (T, H, dv), dev)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    elif S_T is not None:
+        _need(S_T, "S_T", torch.float32, (N, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        _check(lib.gdn2_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(cu_seqlens),
+                                         N, _ptr(S0), _ptr(o), _ptr(S_T), T, H, dk, dv, code, _stream(stream, dev)))
     return o, S_T
 
 

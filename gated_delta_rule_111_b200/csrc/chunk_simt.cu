@@ -20,8 +20,10 @@
 // factor can overflow for any alpha in (0, 1].  U holds the per-token
 // corrections u_t = z_t - (diag(alpha_t) S_{t-1})^T e_t of the token recurrence.
 //
-// Grid: one CTA per (batch*head, 32-column slice of d_v); the value columns of
-// the recurrence evolve independently given the key-side quantities.
+// Grid: one CTA per (sequence*head, 32-column slice of d_v); the value columns
+// of the recurrence evolve independently given the key-side quantities.  A
+// sequence is either row block s of B sequences of T tokens, or, for packed
+// variable-length batches, tokens cu_seqlens[s] .. cu_seqlens[s+1] - 1.
 #include "common.cuh"
 
 namespace gdn2 {
@@ -45,7 +47,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 chunk_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                   const float *__restrict__ alpha, const float *__restrict__ bgate,
                   const float *__restrict__ wgate, const float *S0, TIn *__restrict__ o, float *S_T,
-                  int T, int H, int dv) {
+                  const int *cu_seqlens, int T, int H, int dv) {
     using SM = SimtSmem<DK>;
     constexpr int LD = SM::LD, LDC = SM::LDC;
     extern __shared__ float smem[];
@@ -60,8 +62,15 @@ chunk_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
     float *Sst = U + kC * kDVS;         // [DK][kDVS] state slice
     float *gl = Sst + DK * kDVS;        // [DK] g at the chunk's last token
 
-    const int head = blockIdx.x;        // b * H + h
-    const int bidx = head / H, h = head % H;
+    const int head = blockIdx.x;        // sequence * H + h
+    const int seq = head / H, h = head % H;
+    // Tokens [tb, te) of the flat token index (seq * T + t, or packed offsets).
+    int tb = seq * T, te = tb + T;
+    if (cu_seqlens) {
+        tb = min(max(cu_seqlens[seq], 0), T);
+        te = min(max(cu_seqlens[seq + 1], tb), T);
+    }
+    const int len = te - tb;
     const int col0 = blockIdx.y * kDVS;
     const int tid = threadIdx.x;
 
@@ -71,15 +80,15 @@ chunk_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
         Sst[idx] = S0 ? S0[state_off + (size_t)i * dv + col0 + j] : 0.f;
     }
 
-    for (int c0 = 0; c0 < T; c0 += kC) {
-        const int n = min(kC, T - c0);
+    for (int c0 = 0; c0 < len; c0 += kC) {
+        const int n = min(kC, len - c0);
         __syncthreads();
         // 1. Load the chunk; padding tokens act as k = q = e = z = 0, alpha = 1.
         for (int idx = tid; idx < kC * DK; idx += kThreads) {
             const int t = idx / DK, i = idx % DK;
             float g = 0.f, kk = 0.f, ee = 0.f, qq = 0.f;
             if (t < n) {
-                const size_t off = ((size_t)(bidx * T + c0 + t) * H + h) * DK + i;
+                const size_t off = ((size_t)(tb + c0 + t) * H + h) * DK + i;
                 g = logf(clamp_alpha(__ldg(alpha + off)));
                 kk = Elem<TIn>::load(k + off);
                 ee = __ldg(bgate + off) * kk;
@@ -91,7 +100,7 @@ chunk_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
             const int t = idx / kDVS, j = idx % kDVS;
             float zz = 0.f;
             if (t < n) {
-                const size_t off = ((size_t)(bidx * T + c0 + t) * H + h) * dv + col0 + j;
+                const size_t off = ((size_t)(tb + c0 + t) * H + h) * dv + col0 + j;
                 zz = __ldg(wgate + off) * Elem<TIn>::load(v + off);
             }
             Z[idx] = zz;
@@ -158,7 +167,7 @@ chunk_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
             float acc = 0.f;
             for (int i = 0; i < DK; ++i) acc = fmaf(qt[i], Sst[i * kDVS + j], acc);
             for (int s = 0; s <= t; ++s) acc = fmaf(pt[s], U[s * kDVS + j], acc);
-            const size_t off = ((size_t)(bidx * T + c0 + t) * H + h) * dv + col0 + j;
+            const size_t off = ((size_t)(tb + c0 + t) * H + h) * dv + col0 + j;
             Elem<TIn>::store(o + off, acc);
         }
         __syncthreads();
@@ -182,7 +191,7 @@ chunk_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
 template <typename TIn, int DK>
 cudaError_t launch_typed(const void *q, const void *k, const void *v, const float *alpha, const float *b,
                          const float *w, const float *S0, void *o, float *S_T, int B, int T, int H, int dv,
-                         cudaStream_t stream) {
+                         const int *cu_seqlens, cudaStream_t stream) {
     auto kern = chunk_simt_kernel<TIn, DK>;
     const size_t smem = SimtSmem<DK>::bytes;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -190,7 +199,7 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
     dim3 grid((unsigned)B * (unsigned)H, (unsigned)(dv / kDVS));
     kern<<<grid, kThreads, smem, stream>>>(static_cast<const TIn *>(q), static_cast<const TIn *>(k),
                                            static_cast<const TIn *>(v), alpha, b, w, S0,
-                                           static_cast<TIn *>(o), S_T, T, H, dv);
+                                           static_cast<TIn *>(o), S_T, cu_seqlens, T, H, dv);
     return cudaGetLastError();
 }
 
@@ -198,13 +207,15 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
 
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *alpha,
                               const float *b, const float *w, const float *S0, void *o, float *S_T,
-                              int B, int T, int H, int dk, int dv, gdn2_dtype dt, cudaStream_t stream) {
+                              int B, int T, int H, int dk, int dv, gdn2_dtype dt, const int *cu_seqlens,
+                              cudaStream_t stream) {
     if (dt == GDN2_BF16) {
-        if (dk == 128) return launch_typed<__nv_bfloat16, 128>(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, dv, stream);
-        return launch_typed<__nv_bfloat16, 64>(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, dv, stream);
+        if (dk == 128)
+            return launch_typed<__nv_bfloat16, 128>(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, dv, cu_seqlens, stream);
+        return launch_typed<__nv_bfloat16, 64>(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, dv, cu_seqlens, stream);
     }
-    if (dk == 128) return launch_typed<float, 128>(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, dv, stream);
-    return launch_typed<float, 64>(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, dv, stream);
+    if (dk == 128) return launch_typed<float, 128>(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, dv, cu_seqlens, stream);
+    return launch_typed<float, 64>(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, dv, cu_seqlens, stream);
 }
 
 }  // namespace gdn2

@@ -544,9 +544,9 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
     const int unit = blockIdx.x >> 1, half = blockIdx.x & 1;   // unit = sequence * H + head
     const int seq = unit / p.H, h = unit % p.H;
     int tb, te;
-    if (p.cu_seqlens) {
-        tb = p.cu_seqlens[seq];
-        te = p.cu_seqlens[seq + 1];
+    if (p.cu_seqlens) {         // packed offsets, clamped to the T tokens there are
+        tb = min(max(p.cu_seqlens[seq], 0), p.T);
+        te = min(max(p.cu_seqlens[seq + 1], tb), p.T);
     } else {
         tb = seq * p.T;
         te = tb + p.T;

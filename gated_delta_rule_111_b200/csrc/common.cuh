@@ -32,8 +32,11 @@ cudaError_t launch_recurrent_step(const void *q, const void *k, const void *v, c
                                   const float *b, const float *w, float *S, void *o, int B, int H,
                                   int dk, int dv, gdn2_dtype dt, cudaStream_t stream);
 
+// B sequences of T tokens (cu_seqlens == nullptr), or B packed sequences with device
+// offsets cu_seqlens[0..B] into T tokens in all.
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *alpha,
                               const float *b, const float *w, const float *S0, void *o, float *S_T,
-                              int B, int T, int H, int dk, int dv, gdn2_dtype dt, cudaStream_t stream);
+                              int B, int T, int H, int dk, int dv, gdn2_dtype dt, const int *cu_seqlens,
+                              cudaStream_t stream);
 
 }  // namespace gdn2

@@ -80,22 +80,29 @@ gdn2_status gdn2_device_error(unsigned int *code, int clear) {
     return cuda_status(gdn2::read_device_error(code, clear != 0), "gdn2_device_error");
 }
 
-gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *b,
-                           const float *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
-                           int d_v, gdn2_dtype dt, void *stream) {
+// Shared host-side checks and dispatch of the two prefill entry points.  nseq
+// sequences of T tokens each (cu == nullptr), or nseq packed sequences whose
+// device offsets cu[0..nseq] index T tokens in all.
+static gdn2_status chunk_fwd_common(const void *q, const void *k, const void *v, const float *alpha,
+                                    const float *b, const float *w, const int *cu, const float *S0, void *o,
+                                    float *S_T, int nseq, int T, int H, int d_k, int d_v, gdn2_dtype dt,
+                                    void *stream) {
     g_last_error[0] = 0;
-    gdn2_status st = check_common(B, H, d_k, d_v, dt);
+    gdn2_status st = check_common(nseq, H, d_k, d_v, dt);
     if (st != GDN2_OK) return st;
     if (T < 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "negative T");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (B == 0 || H == 0) return GDN2_OK;
+    if (nseq == 0 || H == 0) return GDN2_OK;
     const size_t es = dt == GDN2_BF16 ? 2 : 4;
-    const size_t state_bytes = (size_t)B * H * d_k * d_v * sizeof(float);
+    const size_t state_bytes = (size_t)nseq * H * d_k * d_v * sizeof(float);
     if (S0 && (st = check_ptr(S0, "S0")) != GDN2_OK) return st;
     if (S_T && (st = check_ptr(S_T, "S_T")) != GDN2_OK) return st;
     if (S0 && S_T && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes))
         return fail(GDN2_ERR_INVALID_ARG, "%s", "S_T partially overlaps S0 (only exact aliasing is allowed)");
-    if (T == 0) {
+    if (cu) {
+        if (reinterpret_cast<uintptr_t>(cu) & 3u) return fail(GDN2_ERR_INVALID_ARG, "%s", "cu_seqlens not 4-byte aligned");
+    }
+    if (T == 0) {          // every sequence is empty: S_T = S0
         if (!S_T || S_T == S0) return GDN2_OK;
         cudaError_t err = S0 ? cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, s)
                              : cudaMemsetAsync(S_T, 0, state_bytes, s);
@@ -106,7 +113,7 @@ gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const fl
     for (int i = 0; i < 6; ++i)
         if ((st = check_ptr(ins[i], names[i])) != GDN2_OK) return st;
     if ((st = check_ptr(o, "o")) != GDN2_OK) return st;
-    const size_t tok = (size_t)B * T * H;
+    const size_t tok = (size_t)(cu ? 1 : nseq) * T * H;
     const size_t in_bytes[6] = {tok * d_k * es, tok * d_k * es, tok * d_v * es,
                                 tok * d_k * 4,  tok * d_k * 4,  tok * d_v * 4};
     const size_t o_bytes = tok * d_v * es;
@@ -118,13 +125,33 @@ gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const fl
         for (int i = 0; i < 6; ++i)
             if (overlaps(S_T, state_bytes, ins[i], in_bytes[i]))
                 return fail(GDN2_ERR_INVALID_ARG, "S_T overlaps %s", names[i]);
+    if (cu) {
+        const size_t cu_bytes = (size_t)(nseq + 1) * sizeof(int);
+        if (overlaps(o, o_bytes, cu, cu_bytes) || overlaps(S_T, state_bytes, cu, cu_bytes))
+            return fail(GDN2_ERR_INVALID_ARG, "%s", "an output overlaps cu_seqlens");
+    }
 
     cudaError_t err;
     if (gdn2::chunk_tc_supported(d_k, d_v, dt))
-        err = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, nullptr, s);
+        err = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, nseq, T, H, cu, s);
     else
-        err = gdn2::launch_chunk_simt(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, dt, s);
+        err = gdn2::launch_chunk_simt(q, k, v, alpha, b, w, S0, o, S_T, nseq, T, H, d_k, d_v, dt, cu, s);
     return cuda_status(err, "gdn2_chunk_fwd launch");
+}
+
+gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *b,
+                           const float *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
+                           int d_v, gdn2_dtype dt, void *stream) {
+    return chunk_fwd_common(q, k, v, alpha, b, w, nullptr, S0, o, S_T, B, T, H, d_k, d_v, dt, stream);
+}
+
+gdn2_status gdn2_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *alpha, const float *b,
+                                  const float *w, const int32_t *cu_seqlens, int N, const float *S0, void *o,
+                                  float *S_T, int T_total, int H, int d_k, int d_v, gdn2_dtype dt, void *stream) {
+    g_last_error[0] = 0;
+    if (!cu_seqlens && N > 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "null pointer: cu_seqlens");
+    return chunk_fwd_common(q, k, v, alpha, b, w, reinterpret_cast<const int *>(cu_seqlens), S0, o, S_T, N, T_total,
+                            H, d_k, d_v, dt, stream);
 }
 
 gdn2_status gdn2_recurrent_step(const void *q, const void *k, const void *v, const float *alpha,

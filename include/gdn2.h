@@ -91,6 +91,35 @@ gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v,
                            gdn2_dtype dt, void *stream);
 
 /*
+ * Chunkwise prefill of a packed batch of N variable-length sequences (the same
+ * recurrence per sequence; chunking restarts at every sequence start).
+ *
+ *   q, k      [T_total][H][d_k]  dt          read (sequence n is rows cu_seqlens[n]
+ *   v         [T_total][H][d_v]  dt          .. cu_seqlens[n+1] - 1 of every tensor)
+ *   alpha, b  [T_total][H][d_k]  float       read
+ *   w         [T_total][H][d_v]  float       read
+ *   cu_seqlens [N + 1] int32     DEVICE      read: 0 = cu[0] <= cu[1] <= ... <= cu[N] =
+ *                                            T_total.  Not checked on the host (it lives
+ *                                            on the device); the kernels clamp every
+ *                                            offset into [0, T_total], so a bad table
+ *                                            never reads or writes outside the buffers.
+ *   S0        [N][H][d_k][d_v]   float       read; NULL means zero initial states
+ *   o         [T_total][H][d_v]  dt          written
+ *   S_T       [N][H][d_k][d_v]   float       written (state after each sequence's last
+ *                                            token; S0 for an empty sequence); may be
+ *                                            NULL, and may alias S0
+ *
+ * Equivalent to one gdn2_chunk_fwd per sequence, in one launch (and bit for bit
+ * identical to those calls).  N = 0 or H = 0 is a no-op.
+ */
+gdn2_status gdn2_chunk_fwd_varlen(const void *q, const void *k, const void *v,
+                                  const float *alpha, const float *b, const float *w,
+                                  const int32_t *cu_seqlens, int N,
+                                  const float *S0, void *o, float *S_T,
+                                  int T_total, int H, int d_k, int d_v,
+                                  gdn2_dtype dt, void *stream);
+
+/*
  * Fused single-token decode step (the recurrent mode; the same mathematics with
  * T = 1, updating the state in place).
  *
@@ -124,8 +153,8 @@ const char *gdn2_last_error(void);
  * undefined).  clear != 0 resets the flag. */
 gdn2_status gdn2_device_error(unsigned int *code, int clear);
 
-/* Test hook for the kernels' failure handling.  Every wait inside a kernel
- * gives up after `cycles` SM clock cycles (default 4e9, about 2 s at the B200's
+/* Test hook for the kernels' failure handling.  Every wait inside the
+ * tensor-core prefill kernel gives up after `cycles` SM clock cycles (default 4e9, about 2 s at the B200's
  * clock), after which the kernel raises the device-side failure flag (see
  * gdn2_device_error), skips its remaining work, waits for its in-flight
  * tensor-core operations, releases its Tensor Memory and returns.  A tiny

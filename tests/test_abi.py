@@ -127,3 +127,25 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "LIB", str(tmp_path / "libgdn2.so"))
     with pytest.raises(ImportError, match="libgdn2.so not found"):
         g.load_library(rebuild_if_stale=False)
+
+
+def _varlen(lib, cu=A16 * 8192, N=3, T=10, H=1, dk=128, dv=128, dt=BF16, o=A16 * 64):
+    P = ctypes.c_void_p
+    return lib.gdn2_chunk_fwd_varlen(P(A16), P(A16), P(A16), P(A16), P(A16), P(A16), P(cu), N, None, P(o), None,
+                                     T, H, dk, dv, dt, None)
+
+
+def test_varlen_host_checks(lib):
+    assert _varlen(lib, cu=None) == g.GDN2_ERR_INVALID_ARG
+    assert b"cu_seqlens" in lib.gdn2_last_error()
+    assert _varlen(lib, cu=A16 * 8192 + 2) == g.GDN2_ERR_INVALID_ARG
+    assert _varlen(lib, N=-1) == g.GDN2_ERR_INVALID_ARG
+    assert _varlen(lib, dk=96) == g.GDN2_ERR_UNSUPPORTED
+    assert _varlen(lib, N=0, cu=None) == g.GDN2_OK          # nothing to do, before any CUDA call
+    assert _varlen(lib, o=A16) == g.GDN2_ERR_INVALID_ARG    # o overlaps the inputs
+
+
+def test_varlen_binding_validates_offsets_tensor():
+    x = torch.zeros(8, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdn2_chunk_fwd_varlen(x, x, x, x, x, x, torch.zeros(3, dtype=torch.int32))
