@@ -48,6 +48,7 @@ def _bind(path):
     lib.oracle_kda.argtypes = [i] * 5 + [dp] * 8
     lib.oracle_gdn.argtypes = [i] * 5 + [dp] * 8
     lib.oracle_b0_sum.argtypes = [i] * 5 + [dp] * 7
+    lib.oracle_gdn2_bwd.argtypes = [i] * 5 + [dp] * 16
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
 
@@ -151,3 +152,23 @@ def b0_sum(q, k, v, alpha, w, S0=None, *, lib=None):
     _load(lib).oracle_b0_sum(B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(w),
                           _ptr(S0), _ptr(o))
     return o
+
+
+def gdn2_bwd(q, k, v, alpha, b, w, S0=None, dO=None, dST=None, *, lib=None):
+    """Gradients of L = sum(dO * o) + sum(dST * S_T) for the recurrence of :func:`gdn2`,
+    by reverse mode through the same token loop (the gate-aware backward pass the
+    "Token processing and parallel training" section calls for: channel-wise decay
+    and separate erase / write gates each get their own gradient).  dO [B,T,H,dv]
+    (None = zeros), dST [B,H,dk,dv] (None = zeros).  Returns a dict of float64
+    arrays dq, dk, dv, dalpha, db, dw, dS0.  Keeps every forward state: T x dk x dv
+    doubles per head, so meant for test-sized inputs."""
+    q, k, v, alpha, b, w, S0, dO, dST = map(_f64, (q, k, v, alpha, b, w, S0, dO, dST))
+    B, T, H, dk, dv = _dims(q, v)
+    if dO is None:
+        dO = np.zeros((B, T, H, dv))
+    out = {n: np.empty_like(x) for n, x in (("dq", q), ("dk", k), ("dv", v), ("dalpha", alpha), ("db", b), ("dw", w))}
+    out["dS0"] = np.empty((B, H, dk, dv))
+    _load(lib).oracle_gdn2_bwd(B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
+                               _ptr(S0), _ptr(dO), _ptr(dST), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                               _ptr(out["dalpha"]), _ptr(out["db"]), _ptr(out["dw"]), _ptr(out["dS0"]))
+    return out

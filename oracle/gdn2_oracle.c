@@ -23,6 +23,7 @@
  *   oracle_kda       Kimi Delta Attention, written in transition-matrix form
  *   oracle_gdn       Gated DeltaNet (scalar decay), written in transition-matrix form
  *   oracle_b0_sum    closed-form decayed causal linear attention (the b = 0 case)
+ *   oracle_gdn2_bwd  gradient of oracle_gdn2 (reverse mode through its token loop)
  */
 #include <math.h>
 #include <stdlib.h>
@@ -237,5 +238,119 @@ void oracle_b0_sum(int B, int T, int H, int dk, int dv,
                 }
             }
             free(coef);
+        }
+}
+
+/*
+ * Gradient of the GDN-2 recurrence (reverse mode through the token loop of
+ * oracle_gdn2, in the same notation).  Given the upstream gradients dO of the
+ * outputs and dST of the final state (NULL = zero), returns the gradients of
+ * L = sum(dO * o) + sum(dST * S_T) with respect to q, k, v, alpha, b, w and S0
+ * (dS0 may be NULL).  The backward pass over one token t, with G the gradient
+ * with respect to S_t:
+ *   G     += q_t dO_t^T                    o_t = S_t^T q_t
+ *   dq_t   = S_t dO_t
+ *   dk_t   = G u,    du = G^T k_t          S_t = Sbar + k_t u^T,  u = z - r
+ *   dw_t   = du * v_t,  dv_t = du * w_t    z = w_t * v_t
+ *   dSbar  = G - e du^T,  de = -Sbar du    r = Sbar^T e
+ *   db_t   = de * k_t,   dk_t += de * b_t  e = b_t * k_t
+ *   dalpha_t[i] = sum_j S_{t-1}[i][j] dSbar[i][j];  G <- diag(alpha_t) dSbar
+ * The forward states S_0 .. S_{T-1} are kept (T x dk x dv doubles per head).
+ */
+void oracle_gdn2_bwd(int B, int T, int H, int dk, int dv,
+                     const double *q, const double *k, const double *v,
+                     const double *alpha, const double *bgate, const double *wgate,
+                     const double *S0, const double *dO, const double *dST,
+                     double *dq, double *dk_, double *dv_, double *dalpha, double *db, double *dw,
+                     double *dS0) {
+    const size_t D2 = (size_t)dk * dv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            double *Sst = (double *)malloc(sizeof(double) * D2 * (size_t)(T + 1));   /* S_0 .. S_T */
+            double *G = (double *)malloc(sizeof(double) * D2);
+            double *Sb = (double *)malloc(sizeof(double) * D2);
+            double *e = (double *)malloc(sizeof(double) * dk);
+            double *z = (double *)malloc(sizeof(double) * dv);
+            double *u = (double *)malloc(sizeof(double) * dv);
+            double *du = (double *)malloc(sizeof(double) * dv);
+            double *de = (double *)malloc(sizeof(double) * dk);
+            load_state(Sst, S0, b, h, H, dk, dv);
+            /* forward, keeping every state */
+            for (int t = 0; t < T; ++t) {
+                const double *Sp = Sst + D2 * t;
+                double *Sn = Sst + D2 * (t + 1);
+                for (int i = 0; i < dk; ++i) {
+                    const double a = VEC(alpha, b, t, h, i, T, H, dk);
+                    for (int j = 0; j < dv; ++j) Sn[(size_t)i * dv + j] = a * Sp[(size_t)i * dv + j];
+                    e[i] = VEC(bgate, b, t, h, i, T, H, dk) * VEC(k, b, t, h, i, T, H, dk);
+                }
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dk; ++i) acc += Sn[(size_t)i * dv + j] * e[i];
+                    u[j] = VEC(wgate, b, t, h, j, T, H, dv) * VEC(v, b, t, h, j, T, H, dv) - acc;
+                }
+                for (int i = 0; i < dk; ++i) {
+                    const double ki = VEC(k, b, t, h, i, T, H, dk);
+                    for (int j = 0; j < dv; ++j) Sn[(size_t)i * dv + j] += ki * u[j];
+                }
+            }
+            /* backward */
+            if (dST) memcpy(G, STATE(dST, b, h, H, dk, dv), sizeof(double) * D2);
+            else memset(G, 0, sizeof(double) * D2);
+            for (int t = T - 1; t >= 0; --t) {
+                const double *Sp = Sst + D2 * t, *St = Sst + D2 * (t + 1);
+                for (int i = 0; i < dk; ++i) {
+                    const double qi = VEC(q, b, t, h, i, T, H, dk);
+                    for (int j = 0; j < dv; ++j) G[(size_t)i * dv + j] += qi * VEC(dO, b, t, h, j, T, H, dv);
+                }
+                for (int i = 0; i < dk; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) acc += St[(size_t)i * dv + j] * VEC(dO, b, t, h, j, T, H, dv);
+                    VEC(dq, b, t, h, i, T, H, dk) = acc;
+                }
+                /* recompute Sbar, e, z, u of this token */
+                for (int i = 0; i < dk; ++i) {
+                    const double a = VEC(alpha, b, t, h, i, T, H, dk);
+                    for (int j = 0; j < dv; ++j) Sb[(size_t)i * dv + j] = a * Sp[(size_t)i * dv + j];
+                    e[i] = VEC(bgate, b, t, h, i, T, H, dk) * VEC(k, b, t, h, i, T, H, dk);
+                }
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dk; ++i) acc += Sb[(size_t)i * dv + j] * e[i];
+                    z[j] = VEC(wgate, b, t, h, j, T, H, dv) * VEC(v, b, t, h, j, T, H, dv);
+                    u[j] = z[j] - acc;
+                }
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dk; ++i) acc += G[(size_t)i * dv + j] * VEC(k, b, t, h, i, T, H, dk);
+                    du[j] = acc;
+                    VEC(dw, b, t, h, j, T, H, dv) = acc * VEC(v, b, t, h, j, T, H, dv);
+                    VEC(dv_, b, t, h, j, T, H, dv) = acc * VEC(wgate, b, t, h, j, T, H, dv);
+                }
+                for (int i = 0; i < dk; ++i) {
+                    double gu = 0.0, sd = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        gu += G[(size_t)i * dv + j] * u[j];
+                        sd += Sb[(size_t)i * dv + j] * du[j];
+                    }
+                    de[i] = -sd;
+                    const double ki = VEC(k, b, t, h, i, T, H, dk), bi = VEC(bgate, b, t, h, i, T, H, dk);
+                    VEC(db, b, t, h, i, T, H, dk) = de[i] * ki;
+                    VEC(dk_, b, t, h, i, T, H, dk) = gu + de[i] * bi;
+                }
+                for (int i = 0; i < dk; ++i) {
+                    const double a = VEC(alpha, b, t, h, i, T, H, dk);
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        const double dsb = G[(size_t)i * dv + j] - e[i] * du[j];
+                        acc += Sp[(size_t)i * dv + j] * dsb;
+                        G[(size_t)i * dv + j] = a * dsb;
+                    }
+                    VEC(dalpha, b, t, h, i, T, H, dk) = acc;
+                }
+            }
+            if (dS0) memcpy(STATE(dS0, b, h, H, dk, dv), G, sizeof(double) * D2);
+            free(Sst); free(G); free(Sb); free(e); free(z); free(u); free(du); free(de);
         }
 }
