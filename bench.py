@@ -7,7 +7,8 @@ Prints one JSON line (rank 0).  Headline: chunkwise prefill tokens/s on the
 state, S0 = 0).  One timed step = one gdn2_chunk_fwd call on that batch (one
 kernel launch).  The decode step (batch 256, H=16, d=128, FP32 state, 64
 consecutive in-place steps) is timed in the same run and reported under
-"decode" as state GB/s.
+"decode" as state GB/s; the chunkwise backward (gdn2_chunk_bwd: gradients of
+every input of the prefill workload) under "backward" as tokens/s.
 
 * value      device time, inputs resident in HBM, CUDA events on the launching
              stream, max over ranks; inputs (675 MB) exceed the 126 MB L2.
@@ -89,6 +90,14 @@ def measured_bf16_peak():
 def measured_tensor_peak():
     bf, src = measured_bf16_peak()
     return bf * TF32_PER_BF16, src + " x nominal tf32/bf16"
+
+
+def backward_bytes(B, T, H, dk, dv):
+    """Algorithmic HBM bytes of one backward call: q,k,v,dO bf16 and alpha,b,w fp32 read;
+    dq,dk,dv bf16 and dalpha,db,dw fp32 written (4,864 B per token-head); the FP32 dS0
+    written.  The workspace (chunk-boundary states, T, P, U, dR) is not counted."""
+    per = 2 * (2 * dk + dv) + 4 * (2 * dk + dv) + 2 * dv + 2 * (2 * dk + dv) + 4 * (2 * dk + dv)
+    return B * T * H * per + B * H * dk * dv * 4
 
 
 def decode_bytes(B, H, dk, dv):
@@ -211,6 +220,25 @@ def oracle_long_tokens_per_s(budget_s=4.0):
     return Ts * reps / dt, threads, f"oracle FP64 on the 16 heads x {Ts} tokens, {reps}x, {dt:.1f} s"
 
 
+def oracle_backward_tokens_per_s(budget_s=4.0, Ts=256):
+    """The FP64 oracle gradient on a bounded sample of the prefill workload (its 16 heads
+    over the first ``Ts`` tokens, with upstream gradients dO and dST), in tokens of H heads
+    per second."""
+    import oracle
+    P = PREFILL
+    threads = oracle.num_threads()
+    x = gi.chunk_inputs(1, Ts, P["H"], P["dk"], P["dv"], dtype="bf16", seed=0)
+    rng = np.random.default_rng(1)
+    dO = gi.round_to_bf16(rng.standard_normal((1, Ts, P["H"], P["dv"])).astype(np.float32))
+    reps, dt = 0, 0.0
+    t0 = time.perf_counter()
+    while reps == 0 or dt < budget_s:
+        oracle.gdn2_bwd(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], None, dO)
+        reps += 1
+        dt = time.perf_counter() - t0
+    return Ts * reps / dt, threads, f"oracle FP64 gradient on the 16 heads x {Ts} tokens, {reps}x, {dt:.1f} s"
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -295,7 +323,10 @@ def run_ours(args):
     long_ms = float("nan")
     if args.workload in ("all", "long"):
         long_ms = run_long(args, torch, dist, g, world, rank, dev, stream)
-    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms)
+    bwd_ms = float("nan")
+    if args.workload in ("all", "backward"):
+        bwd_ms = run_backward(args, torch, dist, g, world, rank, dev, stream)
+    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms, bwd_ms)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -424,6 +455,41 @@ def run_long(args, torch, dist, g, world, rank, dev, stream):
     return ms
 
 
+def run_backward(args, torch, dist, g, world, rank, dev, stream):
+    """The chunkwise backward (gdn2_chunk_bwd) on the prefill workload with a BF16 upstream
+    gradient dO and dST = 0, workspace preallocated; returns ms per call (three launches)."""
+    B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
+    x = gi.chunk_inputs(**PREFILL, seed=rank)
+    d = device_inputs(torch, x, dev)
+    del x
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(100 + rank)
+    dO = torch.randn((B, T, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    ws = torch.empty(g.gdn2_chunk_bwd_workspace_size(B, T, H, dk, dv), dtype=torch.uint8, device=dev)
+    out = {"dq": torch.empty_like(d["q"]), "dk": torch.empty_like(d["k"]), "dv": torch.empty_like(d["v"]),
+           "dalpha": torch.empty_like(d["alpha"]), "db": torch.empty_like(d["b"]), "dw": torch.empty_like(d["w"]),
+           "dS0": torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)}
+
+    def call():
+        g.gdn2_chunk_bwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], None, dO, None, workspace=ws,
+                         out=out, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    sync_ranks(torch, dist, world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(3, min(args.steps, 10))
+    ev0.record(stream)
+    for _ in range(reps):
+        call()
+    ev1.record(stream)
+    sync_ranks(torch, dist, world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / reps, torch, dist, world, dev)
+    del d, dO, ws, out
+    torch.cuda.empty_cache()
+    return ms
+
+
 def bench_config(world):
     """The workload description both arms print (the reference arm times the same workload)."""
     B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
@@ -438,7 +504,7 @@ def _num(x):
     return None if x != x else x      # NaN (workload not run) -> null
 
 
-def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=float("nan")):
+def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=float("nan"), bwd_ms=float("nan")):
     B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
     Bd, Hd = DECODE["B"], DECODE["H"]
     steps_d = DECODE["steps"]
@@ -457,7 +523,9 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=fl
     atflops = algo_flops / (ms_step / 1e3) / 1e12
     bpeak, bsrc = measured_bf16_peak()
 
-    cpu = dec_cpu = long_cpu = None
+    bwd_bytes = backward_bytes(B, T, H, dk, dv)
+    bwd_gbs = bwd_bytes / (bwd_ms / 1e3) / 1e9
+    cpu = dec_cpu = long_cpu = bwd_cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc, _ = oracle_tokens_per_s(budget_s=args.cpu_budget)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
@@ -465,6 +533,9 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=fl
         dec_cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
         v, cores, desc = oracle_long_tokens_per_s()
         long_cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+        if bwd_ms == bwd_ms:
+            v, cores, desc = oracle_backward_tokens_per_s()
+            bwd_cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:
         line = {
@@ -498,6 +569,16 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=fl
                             "tokens_per_s": _num(LONG["B"] * LONG["T"] * world / (long_ms / 1e3)),
                             "note": "latency bound: 32 CTAs walk 1,025 chunks each; reported, no target",
                             "cpu_baseline": long_cpu},
+            "backward": {"metric": "GDN-2 chunk bwd tokens/s @H16 d128 T4K", "unit": "tokens/s",
+                         "value": _num(job_tokens_per_s(B, T, world, bwd_ms)), "ms_per_call": _num(bwd_ms),
+                         "workload": "gradients of every input of the prefill workload (BF16 dO, dST = 0)",
+                         "launches_per_call": 3,
+                         "roofline": {"bound": "hbm", "achieved": _num(bwd_gbs), "peak": hbm, "unit": "GB/s",
+                                      "frac": _num(bwd_gbs / hbm), "traffic": traffic.get("gdn2_chunk_bwd"),
+                                      "algorithmic_bytes_per_launch": bwd_bytes,
+                                      "note": "whole call (prep + state + grad launches) against the "
+                                              "algorithmic bytes; workspace traffic not counted"},
+                         "cpu_baseline": bwd_cpu},
             "gpu_launches": args.steps,
             "clocks": clk.summary() if clk is not None else None,
             "cpu_baseline": cpu,
@@ -561,7 +642,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["all", "prefill", "decode", "long"], default="all",
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "long", "backward"], default="all",
                     help="run only one workload's measurement (for profiling one kernel)")
     args = ap.parse_args()
     if args.impl == "ours":

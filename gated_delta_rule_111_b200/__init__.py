@@ -10,6 +10,8 @@ Functions (same names as the C ABI):
   gdn2_chunk_fwd_varlen(q, k, v, alpha, b, w, cu_seqlens, S0=None, ...)
                                                       -> (o, S_T)   packed variable-length batch
   gdn2_recurrent_step(q, k, v, alpha, b, w, S, ...)   -> o          in-place decode step
+  gdn2_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dST, ...) -> dict    gradients of every input
+  gdn2_chunk_bwd_workspace_size(B, T, H, dk, dv)      -> bytes      workspace of gdn2_chunk_bwd
 """
 from __future__ import annotations
 
@@ -21,7 +23,8 @@ import torch
 
 from . import build as _build
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_recurrent_step", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_recurrent_step", "gdn2_chunk_bwd",
+           "gdn2_chunk_bwd_workspace_size", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
            "load_library", "exported_symbols",
            "GDN2_OK", "GDN2_ERR_INVALID_ARG", "GDN2_ERR_UNSUPPORTED", "GDN2_ERR_CUDA", "Gdn2Error"]
 
@@ -58,6 +61,12 @@ def load_library(rebuild_if_stale: bool = True) -> ctypes.CDLL:
     lib.gdn2_chunk_fwd_varlen.restype = i
     lib.gdn2_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn2_recurrent_step.restype = i
+    sz = ctypes.c_size_t
+    lib.gdn2_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, fp, vp, sz,
+                                   i, i, i, i, i, i, vp]
+    lib.gdn2_chunk_bwd.restype = i
+    lib.gdn2_chunk_bwd_workspace_size.argtypes = [i, i, i, i, i]
+    lib.gdn2_chunk_bwd_workspace_size.restype = sz
     lib.gdn2_status_string.argtypes = [i]
     lib.gdn2_status_string.restype = ctypes.c_char_p
     lib.gdn2_last_error.argtypes = []
@@ -218,3 +227,56 @@ def gdn2_recurrent_step(q, k, v, alpha, b, w, S, *, o=None, stream=None):
         _check(lib.gdn2_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
                                        B, H, dk, dv, code, _stream(stream, dev)))
     return o
+
+
+def gdn2_chunk_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int) -> int:
+    """Bytes of device workspace gdn2_chunk_bwd needs (0 for unsupported head sizes)."""
+    return int(load_library().gdn2_chunk_bwd_workspace_size(B, T, H, dk, dv))
+
+
+def gdn2_chunk_bwd(q, k, v, alpha, b, w, S0=None, dO=None, dST=None, *, workspace=None, out=None,
+                   stream=None):
+    """Gradients of a loss through gdn2_chunk_fwd.  Inputs as for gdn2_chunk_fwd; dO [B,T,H,dv] in
+    q's dtype (None = zero), dST [B,H,dk,dv] fp32 or None.  Returns a dict with dq, dk, dv (q's
+    dtype), dalpha, db, dw, dS0 (fp32).  ``workspace`` (uint8 CUDA tensor of at least
+    gdn2_chunk_bwd_workspace_size bytes) and ``out`` (a dict of preallocated gradients) are
+    optional; missing buffers are allocated here."""
+    lib = load_library()
+    if q.device.type != "cuda":
+        raise ValueError("gdn2_chunk_bwd needs CUDA tensors (there is no CPU implementation)")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("q", q, dk), ("k", k, dk), ("v", v, dv)):
+        _need(t, name, dt, (B, T, H, d), dev)
+    for name, t, d in (("alpha", alpha, dk), ("b", b, dk), ("w", w, dv)):
+        _need(t, name, torch.float32, (B, T, H, d), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    if dO is None:
+        dO = torch.zeros((B, T, H, dv), dtype=dt, device=dev)
+    _need(dO, "dO", dt, (B, T, H, dv), dev)
+    if dST is not None:
+        _need(dST, "dST", torch.float32, (B, H, dk, dv), dev)
+    shapes = {"dq": ((B, T, H, dk), dt), "dk": ((B, T, H, dk), dt), "dv": ((B, T, H, dv), dt),
+              "dalpha": ((B, T, H, dk), torch.float32), "db": ((B, T, H, dk), torch.float32),
+              "dw": ((B, T, H, dv), torch.float32), "dS0": ((B, H, dk, dv), torch.float32)}
+    g = dict(out or {})
+    for name, (shape, dtype) in shapes.items():
+        if g.get(name) is None:
+            g[name] = torch.empty(shape, dtype=dtype, device=dev)
+        else:
+            _need(g[name], name, dtype, shape, dev)
+    need = gdn2_chunk_bwd_workspace_size(B, T, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    elif workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError("workspace: expected a contiguous tensor on the inputs' device")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(lib.gdn2_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
+                                  _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dalpha"]),
+                                  _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), _ptr(workspace), ws_bytes,
+                                  B, T, H, dk, dv, code, _stream(stream, dev)))
+    return g

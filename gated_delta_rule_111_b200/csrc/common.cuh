@@ -39,4 +39,12 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
                               int B, int T, int H, int dk, int dv, gdn2_dtype dt, const int *cu_seqlens,
                               cudaStream_t stream);
 
+// Chunkwise backward: prep, state and gradient launches.  workspace holds
+// chunk_bwd_workspace_floats(B, T, H, dk, dv) floats.
+size_t chunk_bwd_workspace_floats(int B, int T, int H, int dk, int dv);
+cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const float *b,
+                             const float *w, const float *S0, const void *dO, const float *dST, void *dq, void *dk,
+                             void *dv, float *dalpha, float *db, float *dw, float *dS0, float *workspace, int B,
+                             int T, int H, int d_k, int d_v, gdn2_dtype dt, cudaStream_t stream);
+
 }  // namespace gdn2

@@ -154,6 +154,63 @@ gdn2_status gdn2_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
                             H, d_k, d_v, dt, stream);
 }
 
+size_t gdn2_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v) {
+    if (B < 0 || T < 0 || H < 0 || (d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128)) return 0;
+    return gdn2::chunk_bwd_workspace_floats(B, T, H, d_k, d_v) * sizeof(float);
+}
+
+gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const float *b,
+                           const float *w, const float *S0, const void *dO, const float *dST, void *dq, void *dk,
+                           void *dv, float *dalpha, float *db, float *dw, float *dS0, void *workspace,
+                           size_t workspace_bytes, int B, int T, int H, int d_k, int d_v, gdn2_dtype dt,
+                           void *stream) {
+    g_last_error[0] = 0;
+    gdn2_status st = check_common(B, H, d_k, d_v, dt);
+    if (st != GDN2_OK) return st;
+    if (T < 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "negative T");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = (size_t)B * H * d_k * d_v * sizeof(float);
+    if (dS0 && (st = check_ptr(dS0, "dS0")) != GDN2_OK) return st;
+    if (dST && (st = check_ptr(dST, "dST")) != GDN2_OK) return st;
+    if (B == 0 || H == 0) return GDN2_OK;
+    if (dS0 && overlaps(dS0, state_bytes, dST, state_bytes))
+        return fail(GDN2_ERR_INVALID_ARG, "%s", "dS0 overlaps dST");
+    if (T == 0) {          // no tokens: dS0 = dST
+        if (!dS0) return GDN2_OK;
+        cudaError_t err = dST ? cudaMemcpyAsync(dS0, dST, state_bytes, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(dS0, 0, state_bytes, s);
+        return cuda_status(err, "T = 0 gradient copy");
+    }
+    const size_t es = dt == GDN2_BF16 ? 2 : 4;
+    const size_t tok = (size_t)B * T * H;
+    const void *ins[9] = {q, k, v, alpha, b, w, dO, S0, dST};
+    const char *in_names[9] = {"q", "k", "v", "alpha", "b", "w", "dO", "S0", "dST"};
+    const size_t in_bytes[9] = {tok * d_k * es, tok * d_k * es, tok * d_v * es, tok * d_k * 4, tok * d_k * 4,
+                                tok * d_v * 4,  tok * d_v * es, state_bytes,    state_bytes};
+    for (int i = 0; i < 7; ++i)
+        if ((st = check_ptr(ins[i], in_names[i])) != GDN2_OK) return st;
+    if (S0 && (st = check_ptr(S0, "S0")) != GDN2_OK) return st;
+    void *outs[8] = {dq, dk, dv, dalpha, db, dw, dS0, workspace};
+    const char *out_names[8] = {"dq", "dk", "dv", "dalpha", "db", "dw", "dS0", "workspace"};
+    const size_t need = gdn2::chunk_bwd_workspace_floats(B, T, H, d_k, d_v) * sizeof(float);
+    const size_t out_bytes[8] = {tok * d_k * es, tok * d_k * es, tok * d_v * es, tok * d_k * 4,
+                                 tok * d_k * 4,  tok * d_v * 4,  state_bytes,    need};
+    for (int i = 0; i < 8; ++i)
+        if (i != 6 && (st = check_ptr(outs[i], out_names[i])) != GDN2_OK) return st;
+    if (workspace_bytes < need) return fail(GDN2_ERR_INVALID_ARG, "%s", "workspace smaller than gdn2_chunk_bwd_workspace_size");
+    for (int o = 0; o < 8; ++o) {
+        for (int i = 0; i < 9; ++i)
+            if (overlaps(outs[o], out_bytes[o], ins[i], in_bytes[i]))
+                return fail(GDN2_ERR_INVALID_ARG, "%s overlaps an input", out_names[o]);
+        for (int o2 = o + 1; o2 < 8; ++o2)
+            if (overlaps(outs[o], out_bytes[o], outs[o2], out_bytes[o2]))
+                return fail(GDN2_ERR_INVALID_ARG, "%s overlaps another output or the workspace", out_names[o]);
+    }
+    cudaError_t err = gdn2::launch_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dST, dq, dk, dv, dalpha, db, dw, dS0,
+                                             static_cast<float *>(workspace), B, T, H, d_k, d_v, dt, s);
+    return cuda_status(err, "gdn2_chunk_bwd launch");
+}
+
 gdn2_status gdn2_recurrent_step(const void *q, const void *k, const void *v, const float *alpha,
                                 const float *b, const float *w, float *S, void *o, int B, int H, int d_k,
                                 int d_v, gdn2_dtype dt, void *stream) {

@@ -45,6 +45,7 @@
 #ifndef GDN2_H_
 #define GDN2_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -118,6 +119,46 @@ gdn2_status gdn2_chunk_fwd_varlen(const void *q, const void *k, const void *v,
                                   const float *S0, void *o, float *S_T,
                                   int T_total, int H, int d_k, int d_v,
                                   gdn2_dtype dt, void *stream);
+
+/*
+ * Chunkwise backward ("Token processing and parallel training": training goes
+ * through the chunkwise form, so its gradient carries the channel-wise decay and
+ * the separate erase and write gates through every per-block factor).  Computes
+ * the gradient of a scalar loss with respect to every input of gdn2_chunk_fwd,
+ * given the loss's gradients with respect to its outputs.  FP32 arithmetic on
+ * CUDA cores; the decay factors are exponentials of differences of cumulative
+ * log-decays, so no factor leaves the FP32 range for any alpha in (0, 1].
+ *
+ *   q, k, v, alpha, b, w, S0   as in gdn2_chunk_fwd (B sequences of T tokens)   read
+ *   dO        [B][T][H][d_v]  dt            read (dLoss/do)
+ *   dST       [B][H][d_k][d_v] float        read (dLoss/dS_T); NULL means zero
+ *   dq, dk    [B][T][H][d_k]  dt            written
+ *   dv        [B][T][H][d_v]  dt            written
+ *   dalpha, db [B][T][H][d_k] float         written
+ *   dw        [B][T][H][d_v]  float         written
+ *   dS0       [B][H][d_k][d_v] float        written; may be NULL
+ *   workspace device buffer of at least gdn2_chunk_bwd_workspace_size(...)
+ *             bytes, 16-byte aligned, owned by the caller; its contents on
+ *             entry do not matter and are overwritten.
+ *
+ * The forward pass is recomputed inside (the states at chunk boundaries go to
+ * the workspace), so nothing from gdn2_chunk_fwd needs to be kept.  alpha is
+ * differentiated at max(alpha, 2^-64), the value the prefill computes with;
+ * dalpha divides by that value.  Supported: d_k, d_v in {64, 128}, BF16 or FP32.
+ * T = 0, B = 0 or H = 0: nothing is read; dS0 = dST (zero if dST is NULL).
+ * No output may overlap an input, another output or the workspace.
+ */
+gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v,
+                           const float *alpha, const float *b, const float *w,
+                           const float *S0, const void *dO, const float *dST,
+                           void *dq, void *dk, void *dv,
+                           float *dalpha, float *db, float *dw, float *dS0,
+                           void *workspace, size_t workspace_bytes,
+                           int B, int T, int H, int d_k, int d_v,
+                           gdn2_dtype dt, void *stream);
+
+/* Bytes of workspace gdn2_chunk_bwd needs for these sizes (0 if unsupported). */
+size_t gdn2_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
 
 /*
  * Fused single-token decode step (the recurrent mode; the same mathematics with

@@ -149,3 +149,34 @@ def test_varlen_binding_validates_offsets_tensor():
     x = torch.zeros(8, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         g.gdn2_chunk_fwd_varlen(x, x, x, x, x, x, torch.zeros(3, dtype=torch.int32))
+
+
+def _bwd(lib, ws=A16 * 4096, ws_bytes=1 << 40, B=1, T=10, H=1, dk=128, dv=128, dt=BF16, dq=A16 * 64,
+         S0=None, dST=None, dS0=None):
+    # inputs at A16..A16*8, outputs spaced far apart so that only the named overlaps exist
+    q, k, v, a, b, w, dO = (A16 * (1 + i) for i in range(7))
+    outs = [dq, A16 * 128, A16 * 192, A16 * 256, A16 * 320, A16 * 384]
+    return lib.gdn2_chunk_bwd(q, k, v, a, b, w, S0, dO, dST, *outs, dS0, ws, ws_bytes, B, T, H, dk, dv, dt, None)
+
+
+def test_backward_host_checks(lib):
+    assert _bwd(lib, dk=96) == g.GDN2_ERR_UNSUPPORTED
+    assert _bwd(lib, dt=7) == g.GDN2_ERR_UNSUPPORTED
+    assert _bwd(lib, T=-1) == g.GDN2_ERR_INVALID_ARG
+    assert _bwd(lib, B=0) == g.GDN2_OK and _bwd(lib, H=0) == g.GDN2_OK
+    need = lib.gdn2_chunk_bwd_workspace_size(1, 10, 1, 128, 128)
+    assert need == 4 * (2 * 128 * 128 + 2 * 64 * 64 + 2 * 10 * 128)
+    assert _bwd(lib, ws_bytes=need - 4) == g.GDN2_ERR_INVALID_ARG
+    assert b"workspace" in lib.gdn2_last_error()
+    assert _bwd(lib, ws=None) == g.GDN2_ERR_INVALID_ARG
+    assert _bwd(lib, dq=A16 + 8) == g.GDN2_ERR_INVALID_ARG          # misaligned
+    assert _bwd(lib, dq=A16 * 2) == g.GDN2_ERR_INVALID_ARG          # dq overlaps k
+    assert b"overlaps" in lib.gdn2_last_error()
+    assert _bwd(lib, ws=A16 * 128) == g.GDN2_ERR_INVALID_ARG        # workspace overlaps dk
+    assert lib.gdn2_chunk_bwd_workspace_size(1, 10, 1, 96, 128) == 0
+
+
+def test_backward_binding_refuses_cpu_tensors():
+    x = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdn2_chunk_bwd(x, x, x, x, x, x)

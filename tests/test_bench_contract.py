@@ -29,7 +29,7 @@ def test_keys_and_types(capsys):
     d = _line(capsys)
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
               "scaling", "vs_baseline", "dtype", "data", "config", "e2e", "roofline", "gpu_launches", "clocks",
-              "cpu_baseline", "decode", "long_ragged"):
+              "cpu_baseline", "decode", "long_ragged", "backward"):
         assert k in d, k
     assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["vs_baseline"] is None
     assert d["steps"] == 20 and d["warmup"] == 5 and d["n_gpus"] == 1 and d["gpu_launches"] == 20
@@ -90,3 +90,15 @@ def test_tensor_algorithmic_against_bf16_peak(capsys):
 def test_reference_arm_prints_the_same_config():
     assert bench.bench_config(1)["workload"] == bench.bench_config(2)["workload"]
     assert set(bench.bench_config(1)) >= {"workload", "global_batch", "seq_len", "heads", "d_k", "d_v", "dtypes"}
+
+
+def test_backward_entry(capsys):
+    args = argparse.Namespace(steps=20, warmup=5, no_cpu_baseline=True, cpu_budget=1.0)
+    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), float("nan"), 2.0)
+    d = json.loads(capsys.readouterr().out.strip())
+    bw = d["backward"]
+    P = bench.PREFILL
+    assert bw["value"] == pytest.approx(P["B"] * P["T"] / 2.0e-3)
+    # 4,864 B per token-head (q,k,v,dO bf16 + alpha,b,w fp32 in; dq,dk,dv bf16 + dalpha,db,dw fp32 out)
+    assert bench.backward_bytes(1, 1, 1, 128, 128) == 4864 + 128 * 128 * 4
+    assert bw["roofline"]["achieved"] == pytest.approx(bench.backward_bytes(4, 4096, 16, 128, 128) / 2.0e-3 / 1e9)
