@@ -12,6 +12,7 @@ Functions (same names as the C ABI):
   gdn2_recurrent_step(q, k, v, alpha, b, w, S, ...)   -> o          in-place decode step
   gdn2_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dST, ...) -> dict    gradients of every input
   gdn2_chunk_bwd_workspace_size(B, T, H, dk, dv)      -> bytes      workspace of gdn2_chunk_bwd
+  gdn2_chunk_bwd_noalloc(..., out)                    -> dict       the same, workspace inside the library
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ import torch
 from . import build as _build
 
 __all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_recurrent_step", "gdn2_chunk_bwd",
-           "gdn2_chunk_bwd_workspace_size", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
+           "gdn2_chunk_bwd_workspace_size", "gdn2_chunk_bwd_noalloc", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
            "load_library", "exported_symbols",
            "GDN2_OK", "GDN2_ERR_INVALID_ARG", "GDN2_ERR_UNSUPPORTED", "GDN2_ERR_CUDA", "Gdn2Error"]
 
@@ -65,6 +66,9 @@ def load_library(rebuild_if_stale: bool = True) -> ctypes.CDLL:
     lib.gdn2_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, fp, vp, sz,
                                    i, i, i, i, i, i, vp]
     lib.gdn2_chunk_bwd.restype = i
+    lib.gdn2_chunk_bwd_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, fp,
+                                           i, i, i, i, i, i, vp]
+    lib.gdn2_chunk_bwd_noalloc.restype = i
     lib.gdn2_chunk_bwd_workspace_size.argtypes = [i, i, i, i, i]
     lib.gdn2_chunk_bwd_workspace_size.restype = sz
     lib.gdn2_status_string.argtypes = [i]
@@ -280,3 +284,36 @@ def gdn2_chunk_bwd(q, k, v, alpha, b, w, S0=None, dO=None, dST=None, *, workspac
                                   _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), _ptr(workspace), ws_bytes,
                                   B, T, H, dk, dv, code, _stream(stream, dev)))
     return g
+
+
+def gdn2_chunk_bwd_noalloc(q, k, v, alpha, b, w, S0, dO, dST, out, *, stream=None):
+    """gdn2_chunk_bwd with the library's fixed 32 MiB device workspace (no allocation in
+    the call).  ``out`` is a dict of preallocated gradient tensors dq, dk, dv, dalpha, db,
+    dw, dS0 (dS0 may be None); dO must be given.  Returns ``out``."""
+    lib = load_library()
+    if q.device.type != "cuda":
+        raise ValueError("gdn2_chunk_bwd_noalloc needs CUDA tensors (there is no CPU implementation)")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("q", q, dk), ("k", k, dk), ("v", v, dv), ("dO", dO, dv)):
+        _need(t, name, dt, (B, T, H, d), dev)
+    for name, t, d in (("alpha", alpha, dk), ("b", b, dk), ("w", w, dv)):
+        _need(t, name, torch.float32, (B, T, H, d), dev)
+    for name, t in (("S0", S0), ("dST", dST)):
+        if t is not None:
+            _need(t, name, torch.float32, (B, H, dk, dv), dev)
+    shapes = {"dq": ((B, T, H, dk), dt), "dk": ((B, T, H, dk), dt), "dv": ((B, T, H, dv), dt),
+              "dalpha": ((B, T, H, dk), torch.float32), "db": ((B, T, H, dk), torch.float32),
+              "dw": ((B, T, H, dv), torch.float32), "dS0": ((B, H, dk, dv), torch.float32)}
+    for name, (shape, dtype) in shapes.items():
+        if name == "dS0" and out.get(name) is None:
+            continue
+        _need(out[name], name, dtype, shape, dev)
+    with torch.cuda.device(dev):
+        _check(lib.gdn2_chunk_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0),
+                                          _ptr(dO), _ptr(dST), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                          _ptr(out["dalpha"]), _ptr(out["db"]), _ptr(out["dw"]), _ptr(out.get("dS0")),
+                                          B, T, H, dk, dv, code, _stream(stream, dev)))
+    return out

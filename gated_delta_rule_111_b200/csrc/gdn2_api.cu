@@ -54,6 +54,12 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 }  // namespace
 
+namespace gdn2 {
+// The message gdn2_last_error() returns on this thread, for entry points defined
+// in other files of the library.
+void set_last_error(const char *message) { snprintf(g_last_error, sizeof(g_last_error), "%s", message); }
+}  // namespace gdn2
+
 extern "C" {
 
 const char *gdn2_status_string(gdn2_status s) {

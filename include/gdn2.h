@@ -161,6 +161,31 @@ gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v,
 size_t gdn2_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
 
 /*
+ * gdn2_chunk_bwd for callers that cannot allocate device memory (no counterpart
+ * in the paper: an interface for code that runs inside another runtime's memory
+ * manager or a fixed memory budget, or on a host path where cudaMalloc/cudaFree
+ * would synchronise the device).  Same arguments and results as gdn2_chunk_bwd
+ * without the workspace, which is a fixed 32 MiB array in the library's own
+ * device memory, reserved on every GPU that loads the library until the process
+ * exits.  Allocates nothing.
+ *
+ * Sizes whose gdn2_chunk_bwd_workspace_size exceeds 32 MiB are rejected with
+ * GDN2_ERR_INVALID_ARG (gdn2_last_error says so).  The first call on a device
+ * looks up the array's device address there (cudaGetSymbolAddress); make that
+ * first call before any stream capture on that device.  Every call shares the
+ * array: calls whose kernels may overlap on the GPU (other streams, other host
+ * threads, without ordering) race on it.  Nothing in it needs clearing between
+ * calls.
+ */
+gdn2_status gdn2_chunk_bwd_noalloc(const void *q, const void *k, const void *v,
+                                   const float *alpha, const float *b, const float *w,
+                                   const float *S0, const void *dO, const float *dST,
+                                   void *dq, void *dk, void *dv,
+                                   float *dalpha, float *db, float *dw, float *dS0,
+                                   int B, int T, int H, int d_k, int d_v,
+                                   gdn2_dtype dt, void *stream);
+
+/*
  * Fused single-token decode step (the recurrent mode; the same mathematics with
  * T = 1, updating the state in place).
  *
