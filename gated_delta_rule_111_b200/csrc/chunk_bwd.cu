@@ -27,13 +27,20 @@
 // log-decays are kept base 2 and as compensated (hi, lo) pairs, so a difference
 // g_t - g_s keeps its own precision however large |g| has grown in the chunk.
 //
-// Three launches on the caller's stream:
+// Four launches on the caller's stream.  Everything that does not depend on the
+// carried state is computed for all chunks in parallel first, so the serial part
+// is two matrix products per chunk and direction:
 //   prep   grid (chunk, sequence x head): A and P from differences of logs, T by
-//          column-parallel forward substitution; T and P to the workspace.
+//          column-parallel forward substitution; Etil, Khat, Qtil and 2^(g_n).
+//   prep2  grid (chunk, sequence x head): T Etil, T^T Khat, T Z, T^T P^T dO and
+//          Qtil^T dO, so that per chunk
+//            U  = (T Z) - (T Etil) S,              S'  = diag(2^g_n) S + Khat^T U,
+//            dR = (T^T P^T dO) + (T^T Khat) dS',   dS  = diag(2^g_n) dS' + Qtil^T dO - Etil^T dR.
 //   state  grid (sequence x head, 32-column slice of d_v), serial over chunks: the
-//          forward recurrence again (every chunk's start state and U to the
-//          workspace), then the dS recurrence backwards (dR and every chunk's dS'
-//          to the workspace, dS0 out).  Each CTA carries only its value columns.
+//          forward sweep (every chunk's start state and U to the workspace), then
+//          the backward sweep (every chunk's dS' and dR, and dS0).  The next
+//          chunk's operand tiles stream into a second shared-memory buffer
+//          (cp.async) while the current chunk computes.
 //   grad   grid (chunk, sequence x head), independent CTAs: the contractions over
 //          the value columns and the per-token gradients.
 #include "common.cuh"
@@ -95,13 +102,48 @@ __device__ void comp_cumsum(float *hi, float *lo, int ld) {
     __syncthreads();
 }
 
+// 16-byte asynchronous global -> shared copies (completion by wait_group: no spin loop).
+__device__ __forceinline__ void cp_async16(float *dst, const float *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// rows x cols floats (cols a multiple of 4; both row strides multiples of 4 floats).
+__device__ __forceinline__ void copy_tile_async(float *dst, int dst_ld, const float *src, size_t src_ld, int rows,
+                                                int cols) {
+    const int per = cols >> 2;
+    for (int idx = threadIdx.x; idx < rows * per; idx += kThreads) {
+        const int r = idx / per, c4 = (idx - r * per) << 2;
+        cp_async16(dst + r * dst_ld + c4, src + r * src_ld + c4);
+    }
+}
+
+// Per-chunk key block of the workspace (FP32, rows padded by 4 floats):
+//   Et, Kh, Qt, TEt = T Et, TKh = T^T Kh    [64][DK + 4] each
+//   TZ = T Z, TPdO = T^T P^T dO              [64][DV + 4] each
+//   QdO = Qt^T dO                            [DK][DV + 4]
+//   gnf = 2^(g_n)                            [DK]
+template <int DK, int DV>
+struct Kb {
+    static constexpr int LK = DK + 4, LV = DV + 4;
+    static constexpr size_t ET = 0, KH = ET + kC * LK, QT = KH + kC * LK, TET = QT + kC * LK, TKH = TET + kC * LK,
+                            TZ = TKH + kC * LK, TPDO = TZ + kC * LV, QDO = TPDO + kC * LV, GNF = QDO + DK * LV,
+                            floats = GNF + DK;
+    static_assert(floats % 4 == 0, "16-byte aligned blocks");
+};
+
 // Workspace views (FP32).  nch = ceil(T / 64), units = B * H.
 //   Sc  [units][nch][dk][dv]   state at the start of every chunk
 //   dSc [units][nch][dk][dv]   gradient of every chunk's end state
 //   TP  [units][nch][2][64][64]  T = (I + A)^{-1}, then P
 //   U, dR [B][T][H][dv]        per token, laid out like o
+//   KB  [units][nch][Kb::floats]  the key block above
 struct Ws {
-    float *Sc, *dSc, *TP, *U, *dR;
+    float *Sc, *dSc, *TP, *U, *dR, *KB;
 };
 
 // acc[r][c] += sum_k A(m, k) B(k, n) on shared-memory operands, with A(m, k) at
@@ -147,10 +189,11 @@ struct PrepSmem {
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
-template <typename TIn, int DK>
+template <typename TIn, int DK, int DV>
 __global__ void __launch_bounds__(kThreads)
 bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const float *__restrict__ alpha,
-                const float *__restrict__ bgate, float *TP, int T, int H) {
+                const float *__restrict__ bgate, float *TP, float *KB, int T, int H) {
+    using L = Kb<DK, DV>;
     constexpr int LB = PrepSmem<DK>::LB;
     extern __shared__ float smem[];
     float *cg = smem, *cl = cg + kC * LB, *ck = cl + kC * LB, *ce = ck + kC * LB, *cq = ce + kC * LB;
@@ -158,6 +201,7 @@ bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const floa
     const int c = blockIdx.x, unit = blockIdx.y, seq = unit / H, h = unit % H, tid = threadIdx.x;
     const int nch = gridDim.x, c0 = c * kC, n = min(kC, T - c0);
     const size_t tok0 = (size_t)seq * T + c0;
+    float *kb = KB + ((size_t)unit * nch + c) * L::floats;
 
     // thread owns (t = tid/64 + 4r, s = tid%64), r = 0..15
     float a[16], p[16];
@@ -180,6 +224,17 @@ bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const floa
         }
         __syncthreads();
         comp_cumsum<32>(cg, cl, LB);
+        // Etil = e 2^g, Khat = k 2^(g_n - g), Qtil = q 2^g, 2^(g_n) for this channel block
+        for (int idx = tid; idx < kC * 32; idx += kThreads) {
+            const int t = idx >> 5, i = idx & 31;
+            const float gh = cg[t * LB + i], gl = cl[t * LB + i];
+            const float f = ex2(gh + gl);
+            const float kh = ck[t * LB + i] * ex2(gdiff(cg[(kC - 1) * LB + i], cl[(kC - 1) * LB + i], gh, gl));
+            kb[L::ET + t * L::LK + ib + i] = ce[t * LB + i] * f;
+            kb[L::KH + t * L::LK + ib + i] = kh;
+            kb[L::QT + t * L::LK + ib + i] = cq[t * LB + i] * f;
+            if (t == kC - 1) kb[L::GNF + ib + i] = f;
+        }
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             const int t = tb + 4 * r;
@@ -227,211 +282,221 @@ bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const floa
 }
 
 // ---------------------------------------------------------------------------
-// state: the two serial sweeps for one (sequence, head, column slice).
-template <int DK>
-struct StateSmem {
-    static constexpr int LD = DK + 1;
-    static constexpr size_t floats =
-        3 * (size_t)kC * LD + 2 * (size_t)kC * LDT + 3 * (size_t)kC * LDZ + 2 * (size_t)DK * LDZ + 2 * DK;
+// prep2: the products with T and with dO that do not involve the carried state.
+template <int DV>
+struct Prep2Smem {
+    static constexpr int LDV = DV + 1, LB = 33;
+    static constexpr size_t floats = 2 * (size_t)kC * LDT + 3 * (size_t)kC * LDV + 3 * (size_t)kC * LB;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
-// Loads the key side of chunk [c0, c0 + n): G = cumulative log2 alpha (hi in Qt,
-// lo in Et), then Et = b k 2^G, Kh = k 2^(g_n - G), and (with_q) Qt = q 2^G;
-// gl = (hi, lo) of g_n.  Padding rows are zero and hold G at its last value.
-template <typename TIn, int DK>
-__device__ void state_key_side(const TIn *q, const TIn *k, const float *alpha, const float *bgate, size_t tok0,
-                               int n, int H, int h, float *Et, float *Kh, float *Qt, float *gl, bool with_q) {
-    constexpr int LD = DK + 1;
-    const int tid = threadIdx.x;
-    for (int idx = tid; idx < kC * DK; idx += kThreads) {
-        const int t = idx / DK, i = idx % DK;
-        Qt[t * LD + i] = (t < n) ? log2_alpha(alpha + ((tok0 + t) * H + h) * DK + i) : 0.f;
+template <typename TIn, int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_prep2_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, const TIn *__restrict__ dO,
+                 const float *TP, float *KB, int T, int H) {
+    using L = Kb<DK, DV>;
+    constexpr int LDV = Prep2Smem<DV>::LDV, LB = Prep2Smem<DV>::LB;
+    using MV = Mm<kC, DV, 4, DV / 16>;      // 64 x DV outputs
+    using MB = Mm<kC, 32, 4, 2>;            // 64 x 32 outputs
+    using MQ = Mm<32, DV, 2, DV / 16>;      // 32 x DV outputs
+    extern __shared__ float smem[];
+    float *Tm = smem, *Pm = Tm + kC * LDT;
+    float *sO = Pm + kC * LDT, *sZ = sO + kC * LDV, *sW = sZ + kC * LDV;
+    float *b1 = sW + kC * LDV, *b2 = b1 + kC * LB, *b3 = b2 + kC * LB;
+    const int c = blockIdx.x, unit = blockIdx.y, seq = unit / H, h = unit % H, tid = threadIdx.x;
+    const int nch = gridDim.x, c0 = c * kC, n = min(kC, T - c0);
+    const size_t tok0 = (size_t)seq * T + c0;
+    const size_t chunk = (size_t)unit * nch + c;
+    float *kb = KB + chunk * L::floats;
+
+    const float *tp = TP + chunk * 2 * kC * kC;
+    for (int idx = tid; idx < kC * kC; idx += kThreads) {
+        Tm[(idx >> 6) * LDT + (idx & 63)] = tp[idx];
+        Pm[(idx >> 6) * LDT + (idx & 63)] = tp[kC * kC + idx];
     }
-    __syncthreads();
-    comp_cumsum<DK>(Qt, Et, LD);
-    for (int idx = tid; idx < DK; idx += kThreads) {
-        gl[idx] = Qt[(kC - 1) * LD + idx];
-        gl[DK + idx] = Et[(kC - 1) * LD + idx];
-    }
-    __syncthreads();
-    for (int idx = tid; idx < kC * DK; idx += kThreads) {
-        const int t = idx / DK, i = idx % DK;
-        const float gh = Qt[t * LD + i], glo = Et[t * LD + i];
-        float kk = 0.f, bb = 0.f, qq = 0.f;
+    for (int idx = tid; idx < kC * DV; idx += kThreads) {
+        const int t = idx / DV, j = idx % DV;
+        float o = 0.f, z = 0.f;
         if (t < n) {
-            const size_t off = ((tok0 + t) * H + h) * DK + i;
-            kk = Elem<TIn>::load(k + off);
-            bb = __ldg(bgate + off);
-            if (with_q) qq = Elem<TIn>::load(q + off);
+            const size_t off = ((tok0 + t) * H + h) * DV + j;
+            o = Elem<TIn>::load(dO + off);
+            z = __ldg(wgate + off) * Elem<TIn>::load(v + off);
         }
-        const float f = ex2(gh + glo);
-        Et[t * LD + i] = bb * kk * f;
-        Kh[t * LD + i] = kk * ex2(gdiff(gl[i], gl[DK + i], gh, glo));
-        if (with_q) Qt[t * LD + i] = qq * f;
+        sO[t * LDV + j] = o;
+        sZ[t * LDV + j] = z;
+    }
+    __syncthreads();
+    {   // W = P^T dO
+        float acc[4][DV / 16];
+        MV::zero(acc);
+        MV::run(acc, Pm, 1, LDT, sO, LDV, 1, kC);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int cc = 0; cc < DV / 16; ++cc) sW[(MV::mg() + r * 16) * LDV + MV::ng() + cc * 16] = acc[r][cc];
+    }
+    __syncthreads();
+    {   // TPdO = T^T W, TZ = T Z
+        float a1[4][DV / 16], a2[4][DV / 16];
+        MV::zero(a1);
+        MV::zero(a2);
+        MV::run(a1, Tm, 1, LDT, sW, LDV, 1, kC);
+        MV::run(a2, Tm, LDT, 1, sZ, LDV, 1, kC);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int cc = 0; cc < DV / 16; ++cc) {
+                const int t = MV::mg() + r * 16, j = MV::ng() + cc * 16;
+                kb[L::TPDO + t * L::LV + j] = a1[r][cc];
+                kb[L::TZ + t * L::LV + j] = a2[r][cc];
+            }
+    }
+    for (int ib = 0; ib < DK; ib += 32) {
+        __syncthreads();
+        for (int idx = tid; idx < kC * 32; idx += kThreads) {
+            const int t = idx >> 5, i = idx & 31;
+            b1[t * LB + i] = kb[L::ET + t * L::LK + ib + i];
+            b2[t * LB + i] = kb[L::KH + t * L::LK + ib + i];
+            b3[t * LB + i] = kb[L::QT + t * L::LK + ib + i];
+        }
+        __syncthreads();
+        {   // TEt = T Et, TKh = T^T Kh on this channel block
+            float a1[4][2], a2[4][2];
+            MB::zero(a1);
+            MB::zero(a2);
+            MB::run(a1, Tm, LDT, 1, b1, LB, 1, kC);
+            MB::run(a2, Tm, 1, LDT, b2, LB, 1, kC);
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int t = MB::mg() + r * 16, i = MB::ng() + cc * 16;
+                    kb[L::TET + t * L::LK + ib + i] = a1[r][cc];
+                    kb[L::TKH + t * L::LK + ib + i] = a2[r][cc];
+                }
+        }
+        {   // QdO rows of this channel block = Qt^T dO
+            float a3[2][DV / 16];
+            MQ::zero(a3);
+            MQ::run(a3, b3, 1, LB, sO, LDV, 1, kC);
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int cc = 0; cc < DV / 16; ++cc)
+                    kb[L::QDO + (size_t)(ib + MQ::mg() + r * 16) * L::LV + MQ::ng() + cc * 16] = a3[r][cc];
+        }
     }
 }
 
-template <typename TIn, int DK>
+// ---------------------------------------------------------------------------
+// state: the two serial sweeps for one (sequence, head, column slice).
+template <int DK>
+struct StateSmem {
+    static constexpr int LK = DK + 4, LZ = kCS + 4;
+    // one operand buffer: X1 [64][LK], X2 [64][LK], Zs [64][LZ], Qs [DK][LZ], gnf [DK]
+    static constexpr size_t buf = 2 * (size_t)kC * LK + (size_t)kC * LZ + (size_t)DK * LZ + DK;
+    static constexpr size_t floats = 2 * buf + (size_t)DK * LZ + (size_t)kC * LZ;
+    static constexpr size_t bytes = floats * sizeof(float);
+};
+
+template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_state_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
-                 const float *__restrict__ alpha, const float *__restrict__ bgate, const float *__restrict__ wgate,
-                 const float *S0, const TIn *__restrict__ dO, const float *dST, float *dS0, Ws ws, int T, int H,
-                 int dv) {
-    constexpr int LD = DK + 1;
+bwd_state_kernel(const float *S0, const float *dST, float *dS0, Ws ws, int T, int H) {
+    using L = Kb<DK, DV>;
+    using SM = StateSmem<DK>;
+    constexpr int LK = SM::LK, LZ = SM::LZ;
     using M64 = Mm<kC, kCS, 4, 2>;          // 64 x 32 outputs
     using MDK = Mm<DK, kCS, DK / 16, 2>;    // DK x 32 outputs
-    extern __shared__ float smem[];
-    float *Et = smem, *Kh = Et + kC * LD, *Qt = Kh + kC * LD;
-    float *Tm = Qt + kC * LD, *Pm = Tm + kC * LDT;
-    float *Z = Pm + kC * LDT, *U = Z + kC * LDZ, *W = U + kC * LDZ;
-    float *Sst = W + kC * LDZ, *dS = Sst + DK * LDZ, *gl = dS + DK * LDZ;     // gl: [2][DK]
+    extern __shared__ __align__(16) float smem[];
+    float *St = smem + 2 * SM::buf, *Us = St + DK * LZ;
 
     const int unit = blockIdx.x, seq = unit / H, h = unit % H;
     const int col0 = blockIdx.y * kCS, tid = threadIdx.x;
     const size_t tokb = (size_t)seq * T;
-    const int nch = (T + kC - 1) / kC;
-    const size_t soff = (size_t)unit * DK * dv;
+    const int nch = (T + kC - 1) / kC, steps = 2 * nch;
+    const size_t soff = (size_t)unit * DK * DV;
     const int m64 = M64::mg(), n64 = M64::ng(), mdk = MDK::mg(), ndk = MDK::ng();
+
+    // step k < nch: forward over chunk k; step k >= nch: backward over chunk 2 nch - 1 - k
+    auto issue = [&](int kstep) {
+        float *b = smem + (kstep & 1) * SM::buf;
+        float *X1 = b, *X2 = X1 + kC * LK, *Zs = X2 + kC * LK, *Qs = Zs + kC * LZ, *gnf = Qs + DK * LZ;
+        const bool fwd = kstep < nch;
+        const int c = fwd ? kstep : steps - 1 - kstep;
+        const float *kb = ws.KB + ((size_t)unit * nch + c) * L::floats;
+        copy_tile_async(X1, LK, kb + (fwd ? L::TET : L::TKH), L::LK, kC, DK);
+        copy_tile_async(X2, LK, kb + (fwd ? L::KH : L::ET), L::LK, kC, DK);
+        copy_tile_async(Zs, LZ, kb + (fwd ? L::TZ : L::TPDO) + col0, L::LV, kC, kCS);
+        if (!fwd) copy_tile_async(Qs, LZ, kb + L::QDO + col0, L::LV, DK, kCS);
+        copy_tile_async(gnf, DK, kb + L::GNF, DK, 1, DK);
+        cp_async_commit();
+    };
 
     for (int idx = tid; idx < DK * kCS; idx += kThreads) {
         const int i = idx / kCS, j = idx % kCS;
-        Sst[i * LDZ + j] = S0 ? S0[soff + (size_t)i * dv + col0 + j] : 0.f;
+        St[i * LZ + j] = S0 ? S0[soff + (size_t)i * DV + col0 + j] : 0.f;
     }
-    // ---------------- forward sweep: chunk start states and U
-    for (int c = 0; c < nch; ++c) {
-        const int c0 = c * kC, n = min(kC, T - c0);
+    issue(0);
+    for (int kstep = 0; kstep < steps; ++kstep) {
+        if (kstep + 1 < steps) {
+            issue(kstep + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        const bool fwd = kstep < nch;
+        const int c = fwd ? kstep : steps - 1 - kstep;
+        const int n = min(kC, T - c * kC);
         const size_t chunk = (size_t)unit * nch + c;
+        if (kstep == nch) {             // the backward sweep starts from dST
+            for (int idx = tid; idx < DK * kCS; idx += kThreads) {
+                const int i = idx / kCS, j = idx % kCS;
+                St[i * LZ + j] = dST ? dST[soff + (size_t)i * DV + col0 + j] : 0.f;
+            }
+        }
         __syncthreads();
+        const float *b = smem + (kstep & 1) * SM::buf;
+        const float *X1 = b, *X2 = X1 + kC * LK, *Zs = X2 + kC * LK, *Qs = Zs + kC * LZ, *gnf = Qs + DK * LZ;
+        float *save = (fwd ? ws.Sc : ws.dSc) + chunk * DK * DV + col0;
         for (int idx = tid; idx < DK * kCS; idx += kThreads) {
             const int i = idx / kCS, j = idx % kCS;
-            ws.Sc[chunk * DK * dv + (size_t)i * dv + col0 + j] = Sst[i * LDZ + j];
+            save[(size_t)i * DV + j] = St[i * LZ + j];
         }
-        state_key_side<TIn, DK>(q, k, alpha, bgate, tokb + c0, n, H, h, Et, Kh, Qt, gl, false);
-        const float *tp = ws.TP + chunk * 2 * kC * kC;
-        for (int idx = tid; idx < kC * kC; idx += kThreads) Tm[(idx >> 6) * LDT + (idx & 63)] = tp[idx];
-        for (int idx = tid; idx < kC * kCS; idx += kThreads) {
-            const int t = idx / kCS, j = idx % kCS;
-            float zz = 0.f;
-            if (t < n) {
-                const size_t off = ((tokb + c0 + t) * H + h) * dv + col0 + j;
-                zz = __ldg(wgate + off) * Elem<TIn>::load(v + off);
-            }
-            Z[t * LDZ + j] = zz;
-        }
-        __syncthreads();
-        {   // W = Z - Et S
+        {   // forward: U = TZ - TEt S;  backward: dR = TPdO + TKh dS
             float acc[4][2];
             M64::zero(acc);
-            M64::run(acc, Et, LD, 1, Sst, LDZ, 1, DK);
+            M64::run(acc, X1, LK, 1, St, LZ, 1, DK);
+            float *out = fwd ? ws.U : ws.dR;
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int t = m64 + r * 16, j = n64 + cc * 16;
-                    W[t * LDZ + j] = Z[t * LDZ + j] - acc[r][cc];
+                    const float u = fwd ? Zs[t * LZ + j] - acc[r][cc] : Zs[t * LZ + j] + acc[r][cc];
+                    Us[t * LZ + j] = u;
+                    if (t < n) out[((tokb + c * kC + t) * H + h) * DV + col0 + j] = u;
                 }
         }
         __syncthreads();
-        {   // U = T W
-            float acc[4][2];
-            M64::zero(acc);
-            M64::run(acc, Tm, LDT, 1, W, LDZ, 1, kC);
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int t = m64 + r * 16, j = n64 + cc * 16;
-                    U[t * LDZ + j] = acc[r][cc];
-                    if (t < n) ws.U[((tokb + c0 + t) * H + h) * dv + col0 + j] = acc[r][cc];
-                }
-        }
-        __syncthreads();
-        {   // S <- diag(exp g_n) S + Kh^T U
+        {   // forward: S = gnf S + Kh^T U;  backward: dS = gnf dS + QdO - Et^T dR
             float acc[DK / 16][2];
             MDK::zero(acc);
-            MDK::run(acc, Kh, 1, LD, U, LDZ, 1, kC);
+            MDK::run(acc, X2, 1, LK, Us, LZ, 1, kC);
 #pragma unroll
             for (int r = 0; r < DK / 16; ++r)
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int i = mdk + r * 16, j = ndk + cc * 16;
-                    Sst[i * LDZ + j] = fmaf(ex2(gl[i] + gl[DK + i]), Sst[i * LDZ + j], acc[r][cc]);
+                    const float carried = gnf[i] * St[i * LZ + j];
+                    St[i * LZ + j] = fwd ? carried + acc[r][cc] : carried + Qs[i * LZ + j] - acc[r][cc];
                 }
         }
+        __syncthreads();                // buffer kstep & 1 is refilled by the next issue()
     }
-    // ---------------- backward sweep: the dS recurrence
-    __syncthreads();
-    for (int idx = tid; idx < DK * kCS; idx += kThreads) {
-        const int i = idx / kCS, j = idx % kCS;
-        dS[i * LDZ + j] = dST ? dST[soff + (size_t)i * dv + col0 + j] : 0.f;
-    }
-    for (int c = nch - 1; c >= 0; --c) {
-        const int c0 = c * kC, n = min(kC, T - c0);
-        const size_t chunk = (size_t)unit * nch + c;
-        __syncthreads();
-        for (int idx = tid; idx < DK * kCS; idx += kThreads) {
-            const int i = idx / kCS, j = idx % kCS;
-            ws.dSc[chunk * DK * dv + (size_t)i * dv + col0 + j] = dS[i * LDZ + j];
-        }
-        state_key_side<TIn, DK>(q, k, alpha, bgate, tokb + c0, n, H, h, Et, Kh, Qt, gl, true);
-        const float *tp = ws.TP + chunk * 2 * kC * kC;
-        for (int idx = tid; idx < kC * kC; idx += kThreads) {
-            Tm[(idx >> 6) * LDT + (idx & 63)] = tp[idx];
-            Pm[(idx >> 6) * LDT + (idx & 63)] = tp[kC * kC + idx];
-        }
-        for (int idx = tid; idx < kC * kCS; idx += kThreads) {
-            const int t = idx / kCS, j = idx % kCS;
-            float d = 0.f;
-            if (t < n) d = Elem<TIn>::load(dO + ((tokb + c0 + t) * H + h) * dv + col0 + j);
-            Z[t * LDZ + j] = d;
-        }
-        __syncthreads();
-        {   // dU = P^T dO + Kh dS
-            float acc[4][2];
-            M64::zero(acc);
-            M64::run(acc, Pm, 1, LDT, Z, LDZ, 1, kC);
-            M64::run(acc, Kh, LD, 1, dS, LDZ, 1, DK);
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) W[(m64 + r * 16) * LDZ + n64 + cc * 16] = acc[r][cc];
-        }
-        __syncthreads();
-        {   // dR = T^T dU
-            float acc[4][2];
-            M64::zero(acc);
-            M64::run(acc, Tm, 1, LDT, W, LDZ, 1, kC);
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int t = m64 + r * 16, j = n64 + cc * 16;
-                    U[t * LDZ + j] = acc[r][cc];
-                    if (t < n) ws.dR[((tokb + c0 + t) * H + h) * dv + col0 + j] = acc[r][cc];
-                }
-        }
-        __syncthreads();
-        {   // dS <- diag(exp g_n) dS + Qt^T dO - Et^T dR
-            float acc[DK / 16][2], neg[DK / 16][2];
-            MDK::zero(acc);
-            MDK::zero(neg);
-            MDK::run(acc, Qt, 1, LD, Z, LDZ, 1, kC);
-            MDK::run(neg, Et, 1, LD, U, LDZ, 1, kC);
-#pragma unroll
-            for (int r = 0; r < DK / 16; ++r)
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int i = mdk + r * 16, j = ndk + cc * 16;
-                    dS[i * LDZ + j] = fmaf(ex2(gl[i] + gl[DK + i]), dS[i * LDZ + j], acc[r][cc] - neg[r][cc]);
-                }
-        }
-    }
-    __syncthreads();
     if (dS0) {
         for (int idx = tid; idx < DK * kCS; idx += kThreads) {
             const int i = idx / kCS, j = idx % kCS;
-            dS0[soff + (size_t)i * dv + col0 + j] = dS[i * LDZ + j];
+            dS0[soff + (size_t)i * DV + col0 + j] = St[i * LZ + j];
         }
     }
 }
@@ -611,17 +676,22 @@ cudaError_t launch_bwd_typed(const void *q_, const void *k_, const void *v_, con
     const TIn *q = static_cast<const TIn *>(q_), *k = static_cast<const TIn *>(k_),
               *v = static_cast<const TIn *>(v_), *dO = static_cast<const TIn *>(dO_);
     const int nch = (T + kC - 1) / kC, units = B * H;
-    auto kp = bwd_prep_kernel<TIn, DK>;
-    auto ks = bwd_state_kernel<TIn, DK>;
+    auto kp = bwd_prep_kernel<TIn, DK, DV>;
+    auto kp2 = bwd_prep2_kernel<TIn, DK, DV>;
+    auto ks = bwd_state_kernel<DK, DV>;
     auto kg = bwd_grad_kernel<TIn, DK, DV>;
     cudaError_t err;
     if ((err = set_smem(kp, PrepSmem<DK>::bytes)) != cudaSuccess) return err;
+    if ((err = set_smem(kp2, Prep2Smem<DV>::bytes)) != cudaSuccess) return err;
     if ((err = set_smem(ks, StateSmem<DK>::bytes)) != cudaSuccess) return err;
     if ((err = set_smem(kg, GradSmem<DV>::bytes)) != cudaSuccess) return err;
-    kp<<<dim3((unsigned)nch, (unsigned)units), kThreads, PrepSmem<DK>::bytes, stream>>>(q, k, alpha, b, ws.TP, T, H);
+    const dim3 grid_c((unsigned)nch, (unsigned)units);
+    kp<<<grid_c, kThreads, PrepSmem<DK>::bytes, stream>>>(q, k, alpha, b, ws.TP, ws.KB, T, H);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    ks<<<dim3((unsigned)units, (unsigned)(DV / kCS)), kThreads, StateSmem<DK>::bytes, stream>>>(
-        q, k, v, alpha, b, w, S0, dO, dST, dS0, ws, T, H, DV);
+    kp2<<<grid_c, kThreads, Prep2Smem<DV>::bytes, stream>>>(v, w, dO, ws.TP, ws.KB, T, H);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    ks<<<dim3((unsigned)units, (unsigned)(DV / kCS)), kThreads, StateSmem<DK>::bytes, stream>>>(S0, dST, dS0, ws, T,
+                                                                                                 H);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     kg<<<dim3((unsigned)nch, (unsigned)units), kThreads, GradSmem<DV>::bytes, stream>>>(
         q, k, v, alpha, b, w, dO, ws, static_cast<TIn *>(dq), static_cast<TIn *>(dk), static_cast<TIn *>(dv), dalpha,
@@ -648,9 +718,15 @@ cudaError_t launch_bwd_dt(const void *q, const void *k, const void *v, const flo
 
 }  // namespace
 
+static size_t kb_floats(int dk, int dv) {
+    if (dk == 128) return dv == 128 ? Kb<128, 128>::floats : Kb<128, 64>::floats;
+    return dv == 128 ? Kb<64, 128>::floats : Kb<64, 64>::floats;
+}
+
 size_t chunk_bwd_workspace_floats(int B, int T, int H, int dk, int dv) {
     const size_t nch = (size_t)(T + kC - 1) / kC, units = (size_t)B * H;
-    return 2 * units * nch * dk * dv + units * nch * 2 * kC * kC + 2 * (size_t)B * T * H * dv;
+    return 2 * units * nch * dk * dv + units * nch * 2 * kC * kC + 2 * (size_t)B * T * H * dv +
+           units * nch * kb_floats(dk, dv);
 }
 
 cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const float *b,
@@ -664,6 +740,7 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
     ws.TP = ws.dSc + units * nch * d_k * d_v;
     ws.U = ws.TP + units * nch * 2 * kC * kC;
     ws.dR = ws.U + (size_t)B * T * H * d_v;
+    ws.KB = ws.dR + (size_t)B * T * H * d_v;
     if (dt == GDN2_BF16)
         return launch_bwd_dt<__nv_bfloat16>(q, k, v, alpha, b, w, S0, dO, dST, dq, dk, dv, dalpha, db, dw, dS0, ws, B,
                                             T, H, d_k, d_v, stream);

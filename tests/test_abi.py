@@ -165,7 +165,10 @@ def test_backward_host_checks(lib):
     assert _bwd(lib, T=-1) == g.GDN2_ERR_INVALID_ARG
     assert _bwd(lib, B=0) == g.GDN2_OK and _bwd(lib, H=0) == g.GDN2_OK
     need = lib.gdn2_chunk_bwd_workspace_size(1, 10, 1, 128, 128)
-    assert need == 4 * (2 * 128 * 128 + 2 * 64 * 64 + 2 * 10 * 128)
+    # chunk states and gradients, T and P, U and dR per token, and the key block
+    # (five [64][132] tiles, two [64][132], one [128][132], 128 decay factors)
+    key_block = 5 * 64 * 132 + 2 * 64 * 132 + 128 * 132 + 128
+    assert need == 4 * (2 * 128 * 128 + 2 * 64 * 64 + 2 * 10 * 128 + key_block)
     assert _bwd(lib, ws_bytes=need - 4) == g.GDN2_ERR_INVALID_ARG
     assert b"workspace" in lib.gdn2_last_error()
     assert _bwd(lib, ws=None) == g.GDN2_ERR_INVALID_ARG
