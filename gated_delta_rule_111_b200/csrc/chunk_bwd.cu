@@ -146,37 +146,79 @@ struct Ws {
     float *Sc, *dSc, *TP, *U, *dR, *KB;
 };
 
-// acc[r][c] += sum_k A(m, k) B(k, n) on shared-memory operands, with A(m, k) at
-// A[m*sam + k*sak] and B(k, n) at B[k*sbk + n*sbn].  Thread tid owns the outputs
-// m = mg + r*MG, n = ng + c*NG (interleaved, so a warp's loads fall in distinct
-// banks for the strides used here).
-template <int M, int N, int TM, int TN>
-struct Mm {
-    static constexpr int NG = N / TN, MG = M / TM;
-    static_assert(MG * NG == kThreads, "one output micro-tile per thread");
-    __device__ static int mg() { return threadIdx.x / NG; }
-    __device__ static int ng() { return threadIdx.x % NG; }
-    __device__ static void zero(float (&acc)[TM][TN]) {
+// ---------------------------------------------------------------------------
+// Products on shared-memory operands with the warp-level tensor-core MMA
+// (mma.sync m16n8k8, TF32 inputs, FP32 accumulation), three products per step:
+// each operand is split into a TF32 high part and a TF32 remainder, and
+// a_lo b_hi + a_hi b_lo + a_hi b_hi keeps FP32-level accuracy (the dropped
+// a_lo b_lo term is below 2^-22 of the product).
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    const float rest = x - __uint_as_float(hi);
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(rest));
+}
+
+__device__ __forceinline__ void mma_16x8x8(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// One warp's (16 WM) x (8 WN) block of C += A B, A(m, k) at A[m*sam + k*sak] and
+// B(k, n) at B[k*sbk + n*sbn], rows from m0 and columns from n0; K a multiple of 8.
+// Fragment layout of m16n8k8 (lane = 4 g + tg): A rows g, g + 8 and columns tg,
+// tg + 4; B rows tg, tg + 4 and column g; C rows g, g + 8 and columns 2 tg, 2 tg + 1.
+// Shared-memory banks: a row-major operand (unit column step) wants a row stride
+// of 4 mod 32 floats, a transposed one (unit row step) 8 mod 32.
+template <int WM, int WN>
+struct Wt {
+    float c[WM][WN][4];
+    __device__ __forceinline__ void zero() {
 #pragma unroll
-        for (int r = 0; r < TM; ++r)
+        for (int a = 0; a < WM; ++a)
 #pragma unroll
-            for (int c = 0; c < TN; ++c) acc[r][c] = 0.f;
+            for (int b = 0; b < WN; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) c[a][b][i] = 0.f;
     }
-    __device__ static void run(float (&acc)[TM][TN], const float *A, int sam, int sak, const float *B, int sbk,
-                               int sbn, int K) {
-        const int m0 = mg(), n0 = ng();
-#pragma unroll 4
-        for (int kk = 0; kk < K; ++kk) {
-            float a[TM], b[TN];
+    __device__ __forceinline__ void run(const float *A, int sam, int sak, const float *B, int sbk, int sbn, int K,
+                                        int m0, int n0) {
+        const int lane = threadIdx.x & 31, g = lane >> 2, tg = lane & 3;
+#pragma unroll 2
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            uint32_t ah[WM][4], al[WM][4], bh[WN][2], bl[WN][2];
 #pragma unroll
-            for (int r = 0; r < TM; ++r) a[r] = A[(m0 + r * MG) * sam + kk * sak];
+            for (int a = 0; a < WM; ++a) {
+                const float *p = A + (m0 + a * 16 + g) * sam + (k0 + tg) * sak;
+                split_tf32(p[0], ah[a][0], al[a][0]);
+                split_tf32(p[8 * sam], ah[a][1], al[a][1]);
+                split_tf32(p[4 * sak], ah[a][2], al[a][2]);
+                split_tf32(p[8 * sam + 4 * sak], ah[a][3], al[a][3]);
+            }
 #pragma unroll
-            for (int c = 0; c < TN; ++c) b[c] = B[kk * sbk + (n0 + c * NG) * sbn];
+            for (int b = 0; b < WN; ++b) {
+                const float *p = B + (k0 + tg) * sbk + (n0 + b * 8 + g) * sbn;
+                split_tf32(p[0], bh[b][0], bl[b][0]);
+                split_tf32(p[4 * sbk], bh[b][1], bl[b][1]);
+            }
 #pragma unroll
-            for (int r = 0; r < TM; ++r)
+            for (int a = 0; a < WM; ++a)
 #pragma unroll
-                for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+                for (int b = 0; b < WN; ++b) {
+                    mma_16x8x8(c[a][b], al[a], bh[b]);
+                    mma_16x8x8(c[a][b], ah[a], bl[b]);
+                    mma_16x8x8(c[a][b], ah[a], bh[b]);
+                }
         }
+    }
+    // Row and column of accumulator entry c[a][b][i].
+    __device__ __forceinline__ static int row(int m0, int a, int i) {
+        return m0 + a * 16 + ((threadIdx.x & 31) >> 2) + (i >> 1) * 8;
+    }
+    __device__ __forceinline__ static int col(int n0, int b, int i) {
+        return n0 + b * 8 + 2 * (threadIdx.x & 3) + (i & 1);
     }
 };
 
@@ -285,8 +327,8 @@ bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const floa
 // prep2: the products with T and with dO that do not involve the carried state.
 template <int DV>
 struct Prep2Smem {
-    static constexpr int LDV = DV + 1, LB = 33;
-    static constexpr size_t floats = 2 * (size_t)kC * LDT + 3 * (size_t)kC * LDV + 3 * (size_t)kC * LB;
+    static constexpr int LT = kC + 8, LDV = DV + 8, LB = 40;
+    static constexpr size_t floats = 2 * (size_t)kC * LT + 3 * (size_t)kC * LDV + 3 * (size_t)kC * LB;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
@@ -295,13 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_prep2_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, const TIn *__restrict__ dO,
                  const float *TP, float *KB, int T, int H) {
     using L = Kb<DK, DV>;
-    constexpr int LDV = Prep2Smem<DV>::LDV, LB = Prep2Smem<DV>::LB;
-    using MV = Mm<kC, DV, 4, DV / 16>;      // 64 x DV outputs
-    using MB = Mm<kC, 32, 4, 2>;            // 64 x 32 outputs
-    using MQ = Mm<32, DV, 2, DV / 16>;      // 32 x DV outputs
+    constexpr int LT = Prep2Smem<DV>::LT, LDV = Prep2Smem<DV>::LDV, LB = Prep2Smem<DV>::LB;
+    constexpr int VN = DV / 32;             // n8 blocks per warp over DV / 4 columns
     extern __shared__ float smem[];
-    float *Tm = smem, *Pm = Tm + kC * LDT;
-    float *sO = Pm + kC * LDT, *sZ = sO + kC * LDV, *sW = sZ + kC * LDV;
+    const int warp = threadIdx.x >> 5;
+    float *Tm = smem, *Pm = Tm + kC * LT;
+    float *sO = Pm + kC * LT, *sZ = sO + kC * LDV, *sW = sZ + kC * LDV;
     float *b1 = sW + kC * LDV, *b2 = b1 + kC * LB, *b3 = b2 + kC * LB;
     const int c = blockIdx.x, unit = blockIdx.y, seq = unit / H, h = unit % H, tid = threadIdx.x;
     const int nch = gridDim.x, c0 = c * kC, n = min(kC, T - c0);
@@ -311,8 +352,8 @@ bwd_prep2_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, con
 
     const float *tp = TP + chunk * 2 * kC * kC;
     for (int idx = tid; idx < kC * kC; idx += kThreads) {
-        Tm[(idx >> 6) * LDT + (idx & 63)] = tp[idx];
-        Pm[(idx >> 6) * LDT + (idx & 63)] = tp[kC * kC + idx];
+        Tm[(idx >> 6) * LT + (idx & 63)] = tp[idx];
+        Pm[(idx >> 6) * LT + (idx & 63)] = tp[kC * kC + idx];
     }
     for (int idx = tid; idx < kC * DV; idx += kThreads) {
         const int t = idx / DV, j = idx % DV;
@@ -326,30 +367,35 @@ bwd_prep2_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, con
         sZ[t * LDV + j] = z;
     }
     __syncthreads();
+    const int vm0 = (warp >> 2) * 32, vn0 = (warp & 3) * (DV / 4);   // 64 x DV outputs: 32 x DV/4 per warp
     {   // W = P^T dO
-        float acc[4][DV / 16];
-        MV::zero(acc);
-        MV::run(acc, Pm, 1, LDT, sO, LDV, 1, kC);
+        Wt<2, VN> w;
+        w.zero();
+        w.run(Pm, 1, LT, sO, LDV, 1, kC, vm0, vn0);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int cc = 0; cc < DV / 16; ++cc) sW[(MV::mg() + r * 16) * LDV + MV::ng() + cc * 16] = acc[r][cc];
+            for (int b = 0; b < VN; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sW[w.row(vm0, a, i) * LDV + w.col(vn0, b, i)] = w.c[a][b][i];
     }
     __syncthreads();
     {   // TPdO = T^T W, TZ = T Z
-        float a1[4][DV / 16], a2[4][DV / 16];
-        MV::zero(a1);
-        MV::zero(a2);
-        MV::run(a1, Tm, 1, LDT, sW, LDV, 1, kC);
-        MV::run(a2, Tm, LDT, 1, sZ, LDV, 1, kC);
+        Wt<2, VN> w1, w2;
+        w1.zero();
+        w2.zero();
+        w1.run(Tm, 1, LT, sW, LDV, 1, kC, vm0, vn0);
+        w2.run(Tm, LT, 1, sZ, LDV, 1, kC, vm0, vn0);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int cc = 0; cc < DV / 16; ++cc) {
-                const int t = MV::mg() + r * 16, j = MV::ng() + cc * 16;
-                kb[L::TPDO + t * L::LV + j] = a1[r][cc];
-                kb[L::TZ + t * L::LV + j] = a2[r][cc];
-            }
+            for (int b = 0; b < VN; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = w1.row(vm0, a, i), j = w1.col(vn0, b, i);
+                    kb[L::TPDO + t * L::LV + j] = w1.c[a][b][i];
+                    kb[L::TZ + t * L::LV + j] = w2.c[a][b][i];
+                }
     }
     for (int ib = 0; ib < DK; ib += 32) {
         __syncthreads();
@@ -360,30 +406,32 @@ bwd_prep2_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, con
             b3[t * LB + i] = kb[L::QT + t * L::LK + ib + i];
         }
         __syncthreads();
-        {   // TEt = T Et, TKh = T^T Kh on this channel block
-            float a1[4][2], a2[4][2];
-            MB::zero(a1);
-            MB::zero(a2);
-            MB::run(a1, Tm, LDT, 1, b1, LB, 1, kC);
-            MB::run(a2, Tm, 1, LDT, b2, LB, 1, kC);
+        {   // TEt = T Et, TKh = T^T Kh on this channel block (64 x 32: 16 x 16 per warp)
+            const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;
+            Wt<1, 2> w1, w2;
+            w1.zero();
+            w2.zero();
+            w1.run(Tm, LT, 1, b1, LB, 1, kC, m0, n0);
+            w2.run(Tm, 1, LT, b2, LB, 1, kC, m0, n0);
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int t = MB::mg() + r * 16, i = MB::ng() + cc * 16;
-                    kb[L::TET + t * L::LK + ib + i] = a1[r][cc];
-                    kb[L::TKH + t * L::LK + ib + i] = a2[r][cc];
+                for (int i = 0; i < 4; ++i) {
+                    const int t = w1.row(m0, 0, i), ic = w1.col(n0, b, i);
+                    kb[L::TET + t * L::LK + ib + ic] = w1.c[0][b][i];
+                    kb[L::TKH + t * L::LK + ib + ic] = w2.c[0][b][i];
                 }
         }
-        {   // QdO rows of this channel block = Qt^T dO
-            float a3[2][DV / 16];
-            MQ::zero(a3);
-            MQ::run(a3, b3, 1, LB, sO, LDV, 1, kC);
+        {   // QdO rows of this channel block = Qt^T dO (32 x DV: 16 x DV/4 per warp)
+            const int m0 = (warp >> 2) * 16, n0 = (warp & 3) * (DV / 4);
+            Wt<1, VN> w3;
+            w3.zero();
+            w3.run(b3, 1, LB, sO, LDV, 1, kC, m0, n0);
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
+            for (int b = 0; b < VN; ++b)
 #pragma unroll
-                for (int cc = 0; cc < DV / 16; ++cc)
-                    kb[L::QDO + (size_t)(ib + MQ::mg() + r * 16) * L::LV + MQ::ng() + cc * 16] = a3[r][cc];
+                for (int i = 0; i < 4; ++i)
+                    kb[L::QDO + (size_t)(ib + w3.row(m0, 0, i)) * L::LV + w3.col(n0, b, i)] = w3.c[0][b][i];
         }
     }
 }
@@ -392,9 +440,10 @@ bwd_prep2_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, con
 // state: the two serial sweeps for one (sequence, head, column slice).
 template <int DK>
 struct StateSmem {
-    static constexpr int LK = DK + 4, LZ = kCS + 4;
-    // one operand buffer: X1 [64][LK], X2 [64][LK], Zs [64][LZ], Qs [DK][LZ], gnf [DK]
-    static constexpr size_t buf = 2 * (size_t)kC * LK + (size_t)kC * LZ + (size_t)DK * LZ + DK;
+    // X1 is read row-major, X2 transposed: row strides 4 and 8 mod 32 floats
+    static constexpr int LK = DK + 4, LK2 = DK + 8, LZ = kCS + 8;
+    // one operand buffer: X1 [64][LK], X2 [64][LK2], Zs [64][LZ], Qs [DK][LZ], gnf [DK]
+    static constexpr size_t buf = (size_t)kC * LK + (size_t)kC * LK2 + (size_t)kC * LZ + (size_t)DK * LZ + DK;
     static constexpr size_t floats = 2 * buf + (size_t)DK * LZ + (size_t)kC * LZ;
     static constexpr size_t bytes = floats * sizeof(float);
 };
@@ -404,10 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_state_kernel(const float *S0, const float *dST, float *dS0, Ws ws, int T, int H) {
     using L = Kb<DK, DV>;
     using SM = StateSmem<DK>;
-    constexpr int LK = SM::LK, LZ = SM::LZ;
-    using M64 = Mm<kC, kCS, 4, 2>;          // 64 x 32 outputs
-    using MDK = Mm<DK, kCS, DK / 16, 2>;    // DK x 32 outputs
+    constexpr int LK = SM::LK, LK2 = SM::LK2, LZ = SM::LZ;
+    constexpr int SN = DK == 128 ? 4 : 2;   // DK x 32 outputs: 16 x (8 SN) per warp
     extern __shared__ __align__(16) float smem[];
+    const int warp = threadIdx.x >> 5;
+    const int um0 = (warp >> 1) * 16, un0 = (warp & 1) * 16;                          // 64 x 32 outputs
+    const int sm0 = DK == 128 ? warp * 16 : (warp >> 1) * 16, sn0 = DK == 128 ? 0 : (warp & 1) * 16;
     float *St = smem + 2 * SM::buf, *Us = St + DK * LZ;
 
     const int unit = blockIdx.x, seq = unit / H, h = unit % H;
@@ -415,17 +466,16 @@ bwd_state_kernel(const float *S0, const float *dST, float *dS0, Ws ws, int T, in
     const size_t tokb = (size_t)seq * T;
     const int nch = (T + kC - 1) / kC, steps = 2 * nch;
     const size_t soff = (size_t)unit * DK * DV;
-    const int m64 = M64::mg(), n64 = M64::ng(), mdk = MDK::mg(), ndk = MDK::ng();
 
     // step k < nch: forward over chunk k; step k >= nch: backward over chunk 2 nch - 1 - k
     auto issue = [&](int kstep) {
         float *b = smem + (kstep & 1) * SM::buf;
-        float *X1 = b, *X2 = X1 + kC * LK, *Zs = X2 + kC * LK, *Qs = Zs + kC * LZ, *gnf = Qs + DK * LZ;
+        float *X1 = b, *X2 = X1 + kC * LK, *Zs = X2 + kC * LK2, *Qs = Zs + kC * LZ, *gnf = Qs + DK * LZ;
         const bool fwd = kstep < nch;
         const int c = fwd ? kstep : steps - 1 - kstep;
         const float *kb = ws.KB + ((size_t)unit * nch + c) * L::floats;
         copy_tile_async(X1, LK, kb + (fwd ? L::TET : L::TKH), L::LK, kC, DK);
-        copy_tile_async(X2, LK, kb + (fwd ? L::KH : L::ET), L::LK, kC, DK);
+        copy_tile_async(X2, LK2, kb + (fwd ? L::KH : L::ET), L::LK, kC, DK);
         copy_tile_async(Zs, LZ, kb + (fwd ? L::TZ : L::TPDO) + col0, L::LV, kC, kCS);
         if (!fwd) copy_tile_async(Qs, LZ, kb + L::QDO + col0, L::LV, DK, kCS);
         copy_tile_async(gnf, DK, kb + L::GNF, DK, 1, DK);
@@ -456,39 +506,39 @@ bwd_state_kernel(const float *S0, const float *dST, float *dS0, Ws ws, int T, in
         }
         __syncthreads();
         const float *b = smem + (kstep & 1) * SM::buf;
-        const float *X1 = b, *X2 = X1 + kC * LK, *Zs = X2 + kC * LK, *Qs = Zs + kC * LZ, *gnf = Qs + DK * LZ;
+        const float *X1 = b, *X2 = X1 + kC * LK, *Zs = X2 + kC * LK2, *Qs = Zs + kC * LZ, *gnf = Qs + DK * LZ;
         float *save = (fwd ? ws.Sc : ws.dSc) + chunk * DK * DV + col0;
         for (int idx = tid; idx < DK * kCS; idx += kThreads) {
             const int i = idx / kCS, j = idx % kCS;
             save[(size_t)i * DV + j] = St[i * LZ + j];
         }
         {   // forward: U = TZ - TEt S;  backward: dR = TPdO + TKh dS
-            float acc[4][2];
-            M64::zero(acc);
-            M64::run(acc, X1, LK, 1, St, LZ, 1, DK);
+            Wt<1, 2> w;
+            w.zero();
+            w.run(X1, LK, 1, St, LZ, 1, DK, um0, un0);
             float *out = fwd ? ws.U : ws.dR;
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int t = m64 + r * 16, j = n64 + cc * 16;
-                    const float u = fwd ? Zs[t * LZ + j] - acc[r][cc] : Zs[t * LZ + j] + acc[r][cc];
+                for (int i = 0; i < 4; ++i) {
+                    const int t = w.row(um0, 0, i), j = w.col(un0, b, i);
+                    const float u = fwd ? Zs[t * LZ + j] - w.c[0][b][i] : Zs[t * LZ + j] + w.c[0][b][i];
                     Us[t * LZ + j] = u;
                     if (t < n) out[((tokb + c * kC + t) * H + h) * DV + col0 + j] = u;
                 }
         }
         __syncthreads();
         {   // forward: S = gnf S + Kh^T U;  backward: dS = gnf dS + QdO - Et^T dR
-            float acc[DK / 16][2];
-            MDK::zero(acc);
-            MDK::run(acc, X2, 1, LK, Us, LZ, 1, kC);
+            Wt<1, SN> w;
+            w.zero();
+            w.run(X2, 1, LK2, Us, LZ, 1, kC, sm0, sn0);
 #pragma unroll
-            for (int r = 0; r < DK / 16; ++r)
+            for (int b = 0; b < SN; ++b)
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int i = mdk + r * 16, j = ndk + cc * 16;
-                    const float carried = gnf[i] * St[i * LZ + j];
-                    St[i * LZ + j] = fwd ? carried + acc[r][cc] : carried + Qs[i * LZ + j] - acc[r][cc];
+                for (int i = 0; i < 4; ++i) {
+                    const int r = w.row(sm0, 0, i), j = w.col(sn0, b, i);
+                    const float carried = gnf[r] * St[r * LZ + j];
+                    St[r * LZ + j] = fwd ? carried + w.c[0][b][i] : carried + Qs[r * LZ + j] - w.c[0][b][i];
                 }
         }
         __syncthreads();                // buffer kstep & 1 is refilled by the next issue()
@@ -505,7 +555,7 @@ bwd_state_kernel(const float *S0, const float *dST, float *dS0, Ws ws, int T, in
 // grad: per-token gradients of one chunk.  Key channels in blocks of 32.
 template <int DV>
 struct GradSmem {
-    static constexpr int LDV = DV + 1, LB = 33;
+    static constexpr int LDV = DV + 4, LB = 33;
     static constexpr size_t floats = 3 * (size_t)kC * LDV + 2 * (size_t)kC * LDT + 2 * 32 * (size_t)LDV +
                                      7 * (size_t)kC * LB + 32;
     static_assert(2 * 32 * LDV >= kC * LB, "the lo tile fits where S and dS' were");
@@ -519,9 +569,8 @@ bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
                 const TIn *__restrict__ dO, Ws ws, TIn *dq, TIn *dk, TIn *dvv, float *dalpha, float *db,
                 float *dw, int T, int H) {
     constexpr int LDV = GradSmem<DV>::LDV, LB = GradSmem<DV>::LB;
-    using MP = Mm<kC, kC, 4, 4>;     // 64 x 64 outputs
-    using MX = Mm<kC, 32, 4, 2>;     // 64 x 32 outputs
     extern __shared__ float smem[];
+    const int warp = threadIdx.x >> 5;
     float *sO = smem, *sU = sO + kC * LDV, *sR = sU + kC * LDV;
     float *dP = sR + kC * LDV, *dA = dP + kC * LDT;
     float *sS = dA + kC * LDT, *sD = sS + 32 * LDV;
@@ -549,20 +598,23 @@ bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
         sO[t * LDV + j] = o; sU[t * LDV + j] = u; sR[t * LDV + j] = r;
     }
     __syncthreads();
-    {   // dP = dO U^T (s <= t), dA = -dR U^T (s < t)
-        float ap[4][4], aa[4][4];
-        MP::zero(ap);
-        MP::zero(aa);
-        MP::run(ap, sO, LDV, 1, sU, 1, LDV, DV);
-        MP::run(aa, sR, LDV, 1, sU, 1, LDV, DV);
+    {   // dP = dO U^T (s <= t), dA = -dR U^T (s < t); 64 x 64, 32 x 16 per warp
+        const int m0 = (warp >> 2) * 32, n0 = (warp & 3) * 16;
+        Wt<2, 2> wp, wa;
+        wp.zero();
+        wa.zero();
+        wp.run(sO, LDV, 1, sU, 1, LDV, DV, m0, n0);
+        wa.run(sR, LDV, 1, sU, 1, LDV, DV, m0, n0);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const int t = MP::mg() + r * 16, s = MP::ng() + cc * 16;
-                dP[t * LDT + s] = (s <= t) ? ap[r][cc] : 0.f;
-                dA[t * LDT + s] = (s < t) ? -aa[r][cc] : 0.f;
-            }
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = wp.row(m0, a, i), s = wp.col(n0, b, i);
+                    dP[t * LDT + s] = (s <= t) ? wp.c[a][b][i] : 0.f;
+                    dA[t * LDT + s] = (s < t) ? -wa.c[a][b][i] : 0.f;
+                }
     }
     for (int ib = 0; ib < DK; ib += 32) {
         __syncthreads();
@@ -591,20 +643,23 @@ bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             for (int j = 0; j < DV; ++j) acc = fmaf(sS[tid * LDV + j], sD[tid * LDV + j], acc);
             rs[tid] = acc;
         }
-        {   // X1 = S dO, X2 = S dR, Y = dS' U, as [token][channel]
-            float x1[4][2], x2[4][2], y[4][2];
-            MX::zero(x1);
-            MX::zero(x2);
-            MX::zero(y);
-            MX::run(x1, sO, LDV, 1, sS, 1, LDV, DV);
-            MX::run(x2, sR, LDV, 1, sS, 1, LDV, DV);
-            MX::run(y, sU, LDV, 1, sD, 1, LDV, DV);
+        {   // X1 = S dO, X2 = S dR, Y = dS' U, as [token][channel]; 64 x 32, 16 x 16 per warp
+            const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;
+            Wt<1, 2> x1, x2, y;
+            x1.zero();
+            x2.zero();
+            y.zero();
+            x1.run(sO, LDV, 1, sS, 1, LDV, DV, m0, n0);
+            x2.run(sR, LDV, 1, sS, 1, LDV, DV, m0, n0);
+            y.run(sU, LDV, 1, sD, 1, LDV, DV, m0, n0);
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int t = MX::mg() + r * 16, i = MX::ng() + cc * 16;
-                    X1[t * LB + i] = x1[r][cc]; X2[t * LB + i] = x2[r][cc]; Y[t * LB + i] = y[r][cc];
+                for (int i = 0; i < 4; ++i) {
+                    const int t = x1.row(m0, 0, i), ic = x1.col(n0, b, i);
+                    X1[t * LB + ic] = x1.c[0][b][i];
+                    X2[t * LB + ic] = x2.c[0][b][i];
+                    Y[t * LB + ic] = y.c[0][b][i];
                 }
         }
         __syncthreads();
