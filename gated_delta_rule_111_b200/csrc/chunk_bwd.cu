@@ -52,11 +52,7 @@ constexpr int kC = 64;            // chunk length
 constexpr int kCS = 32;           // value columns per CTA of the state kernel
 constexpr int kThreads = 256;
 constexpr int LDT = kC + 1;       // row stride of 64 x 64 tiles in shared memory
-constexpr int LDZ = kCS + 1;      // row stride of column-slice tiles
-constexpr float kAlphaMin = 5.42101086e-20f;   // 2^-64
-
-// log2 of the clamped decay, to an ulp (the exponentials below are base 2)
-__device__ __forceinline__ float log2_alpha(const float *p) { return log2f(fmaxf(__ldg(p), kAlphaMin)); }
+constexpr float kAlphaMin = 5.42101086e-20f;   // 2^-64; log2f of the clamped decay is accurate to an ulp
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -252,17 +248,29 @@ bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const floa
     const int s = tid & 63, tb = tid >> 6;
     for (int ib = 0; ib < DK; ib += 32) {
         __syncthreads();
-        for (int idx = tid; idx < kC * 32; idx += kThreads) {
-            const int t = idx >> 5, i = idx & 31;
-            float g = 0.f, kk = 0.f, qq = 0.f, ee = 0.f;
-            if (t < n) {
-                const size_t off = ((tok0 + t) * H + h) * DK + ib + i;
-                g = log2_alpha(alpha + off);
-                kk = Elem<TIn>::load(k + off);
-                qq = Elem<TIn>::load(q + off);
-                ee = __ldg(bgate + off) * kk;
+        {   // all loads first, then the transforms
+            constexpr int E = kC * 32 / kThreads;
+            float ra[E], rk[E], rq[E], rb[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
+                ra[e] = 1.f; rk[e] = rq[e] = rb[e] = 0.f;
+                if (t < n) {
+                    const size_t off = ((tok0 + t) * H + h) * DK + ib + i;
+                    ra[e] = __ldg(alpha + off);
+                    rk[e] = Elem<TIn>::load(k + off);
+                    rq[e] = Elem<TIn>::load(q + off);
+                    rb[e] = __ldg(bgate + off);
+                }
             }
-            cg[t * LB + i] = g; ck[t * LB + i] = kk; cq[t * LB + i] = qq; ce[t * LB + i] = ee;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
+                cg[t * LB + i] = log2f(fmaxf(ra[e], kAlphaMin));
+                ck[t * LB + i] = rk[e];
+                cq[t * LB + i] = rq[e];
+                ce[t * LB + i] = rb[e] * rk[e];
+            }
         }
         __syncthreads();
         comp_cumsum<32>(cg, cl, LB);
@@ -351,21 +359,30 @@ bwd_prep2_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, con
     float *kb = KB + chunk * L::floats;
 
     const float *tp = TP + chunk * 2 * kC * kC;
-    for (int idx = tid; idx < kC * kC; idx += kThreads) {
-        Tm[(idx >> 6) * LT + (idx & 63)] = tp[idx];
-        Pm[(idx >> 6) * LT + (idx & 63)] = tp[kC * kC + idx];
-    }
-    for (int idx = tid; idx < kC * DV; idx += kThreads) {
-        const int t = idx / DV, j = idx % DV;
-        float o = 0.f, z = 0.f;
-        if (t < n) {
-            const size_t off = ((tok0 + t) * H + h) * DV + j;
-            o = Elem<TIn>::load(dO + off);
-            z = __ldg(wgate + off) * Elem<TIn>::load(v + off);
+    copy_tile_async(Tm, LT, tp, kC, kC, kC);
+    copy_tile_async(Pm, LT, tp + kC * kC, kC, kC, kC);
+    cp_async_commit();
+    for (int base = 0; base < kC * DV; base += 8 * kThreads) {     // eight loads in flight per thread
+        float ro[8], rw[8], rv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int idx = base + tid + e * kThreads, t = idx / DV, j = idx % DV;
+            ro[e] = rw[e] = rv[e] = 0.f;
+            if (t < n) {
+                const size_t off = ((tok0 + t) * H + h) * DV + j;
+                ro[e] = Elem<TIn>::load(dO + off);
+                rw[e] = __ldg(wgate + off);
+                rv[e] = Elem<TIn>::load(v + off);
+            }
         }
-        sO[t * LDV + j] = o;
-        sZ[t * LDV + j] = z;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int idx = base + tid + e * kThreads, t = idx / DV, j = idx % DV;
+            sO[t * LDV + j] = ro[e];
+            sZ[t * LDV + j] = rw[e] * rv[e];
+        }
     }
+    cp_async_wait<0>();
     __syncthreads();
     const int vm0 = (warp >> 2) * 32, vn0 = (warp & 3) * (DV / 4);   // 64 x DV outputs: 32 x DV/4 per warp
     {   // W = P^T dO
@@ -399,12 +416,11 @@ bwd_prep2_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, con
     }
     for (int ib = 0; ib < DK; ib += 32) {
         __syncthreads();
-        for (int idx = tid; idx < kC * 32; idx += kThreads) {
-            const int t = idx >> 5, i = idx & 31;
-            b1[t * LB + i] = kb[L::ET + t * L::LK + ib + i];
-            b2[t * LB + i] = kb[L::KH + t * L::LK + ib + i];
-            b3[t * LB + i] = kb[L::QT + t * L::LK + ib + i];
-        }
+        copy_tile_async(b1, LB, kb + L::ET + ib, L::LK, kC, 32);
+        copy_tile_async(b2, LB, kb + L::KH + ib, L::LK, kC, 32);
+        copy_tile_async(b3, LB, kb + L::QT + ib, L::LK, kC, 32);
+        cp_async_commit();
+        cp_async_wait<0>();
         __syncthreads();
         {   // TEt = T Et, TKh = T^T Kh on this channel block (64 x 32: 16 x 16 per warp)
             const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;
@@ -618,30 +634,43 @@ bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
     }
     for (int ib = 0; ib < DK; ib += 32) {
         __syncthreads();
-        const float *sc = ws.Sc + chunk * DK * DV + (size_t)ib * DV;
-        const float *dsc = ws.dSc + chunk * DK * DV + (size_t)ib * DV;
-        for (int idx = tid; idx < 32 * DV; idx += kThreads) {
-            const int i = idx / DV, j = idx % DV;
-            sS[i * LDV + j] = sc[idx];
-            sD[i * LDV + j] = dsc[idx];
-        }
-        for (int idx = tid; idx < kC * 32; idx += kThreads) {
-            const int t = idx >> 5, i = idx & 31;
-            float g = 0.f, kk = 0.f, qq = 0.f, ee = 0.f;
-            if (t < n) {
-                const size_t off = ((tok0 + t) * H + h) * DK + ib + i;
-                g = log2_alpha(alpha + off);
-                kk = Elem<TIn>::load(k + off);
-                qq = Elem<TIn>::load(q + off);
-                ee = __ldg(bgate + off) * kk;
+        copy_tile_async(sS, LDV, ws.Sc + chunk * DK * DV + (size_t)ib * DV, DV, 32, DV);
+        copy_tile_async(sD, LDV, ws.dSc + chunk * DK * DV + (size_t)ib * DV, DV, 32, DV);
+        cp_async_commit();
+        {   // this block's key side: all loads first, then the transforms
+            constexpr int E = kC * 32 / kThreads;
+            float ra[E], rk[E], rq[E], rb[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
+                ra[e] = 1.f; rk[e] = rq[e] = rb[e] = 0.f;
+                if (t < n) {
+                    const size_t off = ((tok0 + t) * H + h) * DK + ib + i;
+                    ra[e] = __ldg(alpha + off);
+                    rk[e] = Elem<TIn>::load(k + off);
+                    rq[e] = Elem<TIn>::load(q + off);
+                    rb[e] = __ldg(bgate + off);
+                }
             }
-            cg[t * LB + i] = g; ck[t * LB + i] = kk; cq[t * LB + i] = qq; ce[t * LB + i] = ee;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
+                cg[t * LB + i] = log2f(fmaxf(ra[e], kAlphaMin));
+                ck[t * LB + i] = rk[e];
+                cq[t * LB + i] = rq[e];
+                ce[t * LB + i] = rb[e] * rk[e];
+            }
         }
+        cp_async_wait<0>();
         __syncthreads();
-        if (tid < 32) {                 // row sums of S * dS'
+        {   // row sums of S * dS': eight lanes per row
+            const int i = tid >> 3, part = tid & 7;
             float acc = 0.f;
-            for (int j = 0; j < DV; ++j) acc = fmaf(sS[tid * LDV + j], sD[tid * LDV + j], acc);
-            rs[tid] = acc;
+            for (int j = part; j < DV; j += 8) acc = fmaf(sS[i * LDV + j], sD[i * LDV + j], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+            if (part == 0) rs[i] = acc;
         }
         {   // X1 = S dO, X2 = S dR, Y = dS' U, as [token][channel]; 64 x 32, 16 x 16 per warp
             const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;
@@ -707,12 +736,26 @@ bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             X2[(idx >> 5) * LB + (idx & 31)] = dlg[e];
         }
         __syncthreads();
-        if (tid < 32) {                     // dalpha = reverse cumulative sum / alpha
+        {   // dalpha = reverse cumulative sum of dlog gamma / alpha: (channel, 8-token segment) per thread
+            const int i = tid & 31, seg = tid >> 5;
+            float ra[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int t = seg * 8 + u;
+                ra[u] = t < n ? __ldg(alpha + ((tok0 + t) * H + h) * DK + ib + i) : 1.f;
+            }
+            float tot = 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) tot += X2[(seg * 8 + u) * LB + i];
+            X1[seg * LB + i] = tot;             // X1 is free: segment totals
+            __syncthreads();
             float run = 0.f;
-            for (int t = n - 1; t >= 0; --t) {
-                run += X2[t * LB + tid];
-                const size_t off = ((tok0 + t) * H + h) * DK + ib + tid;
-                dalpha[off] = run / fmaxf(__ldg(alpha + off), kAlphaMin);
+            for (int s2 = seg + 1; s2 < 8; ++s2) run += X1[s2 * LB + i];
+#pragma unroll
+            for (int u = 7; u >= 0; --u) {
+                const int t = seg * 8 + u;
+                run += X2[t * LB + i];
+                if (t < n) dalpha[((tok0 + t) * H + h) * DK + ib + i] = run / fmaxf(ra[u], kAlphaMin);
             }
         }
     }
