@@ -49,6 +49,7 @@ def _bind(path):
     lib.oracle_gdn.argtypes = [i] * 5 + [dp] * 8
     lib.oracle_b0_sum.argtypes = [i] * 5 + [dp] * 7
     lib.oracle_gdn2_bwd.argtypes = [i] * 5 + [dp] * 16
+    lib.oracle_gdn2_prep.argtypes = [ctypes.c_longlong, i, i] + [dp] * 12
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
 
@@ -172,3 +173,27 @@ def gdn2_bwd(q, k, v, alpha, b, w, S0=None, dO=None, dST=None, *, lib=None):
                                _ptr(S0), _ptr(dO), _ptr(dST), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
                                _ptr(out["dalpha"]), _ptr(out["db"]), _ptr(out["dw"]), _ptr(out["dS0"]))
     return out
+
+
+def gdn2_prep(xq, xk, xv, xa, xb, xw, *, lib=None):
+    """The recurrence's inputs from pre-activation logits (per token and head):
+    q, k = L2-normalised SiLU of xq, xk; v = SiLU(xv); alpha = exp(-softplus(xa));
+    b, w = sigmoid(xb), sigmoid(xw) -- the query/key/value paths of "Token processing
+    and parallel training" and the sigmoid gates of "Independent decisions on two axes"
+    (alpha's parameterisation is this package's reading: the pages leave it open).
+    Inputs [..., d] (any leading shape, channels last); returns a dict of float64 arrays
+    q, k, v, alpha, b, w of the same shapes."""
+    xq, xk, xv, xa, xb, xw = map(_f64, (xq, xk, xv, xa, xb, xw))
+    dk, dv = xq.shape[-1], xv.shape[-1]
+    rows = xq.size // dk
+    out = {n: np.empty_like(x) for n, x in (("q", xq), ("k", xk), ("v", xv), ("alpha", xa), ("b", xb), ("w", xw))}
+    _load(lib).oracle_gdn2_prep(rows, dk, dv, _ptr(xq), _ptr(xk), _ptr(xv), _ptr(xa), _ptr(xb), _ptr(xw),
+                                _ptr(out["q"]), _ptr(out["k"]), _ptr(out["v"]), _ptr(out["alpha"]), _ptr(out["b"]),
+                                _ptr(out["w"]))
+    return out
+
+
+def gdn2_from_logits(xq, xk, xv, xa, xb, xw, S0=None, *, lib=None):
+    """:func:`gdn2` applied to :func:`gdn2_prep` of the logits ([B,T,H,d] each)."""
+    x = gdn2_prep(xq, xk, xv, xa, xb, xw, lib=lib)
+    return gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], S0, lib=lib)

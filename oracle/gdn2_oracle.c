@@ -24,6 +24,8 @@
  *   oracle_gdn       Gated DeltaNet (scalar decay), written in transition-matrix form
  *   oracle_b0_sum    closed-form decayed causal linear attention (the b = 0 case)
  *   oracle_gdn2_bwd  gradient of oracle_gdn2 (reverse mode through its token loop)
+ *   oracle_gdn2_prep the activations that turn pre-activation logits into the
+ *                    recurrence's inputs (q, k, v, alpha, b, w)
  */
 #include <math.h>
 #include <stdlib.h>
@@ -353,4 +355,52 @@ void oracle_gdn2_bwd(int B, int T, int H, int dk, int dv,
             if (dS0) memcpy(STATE(dS0, b, h, H, dk, dv), G, sizeof(double) * D2);
             free(Sst); free(G); free(Sb); free(e); free(z); free(u); free(du); free(de);
         }
+}
+
+/*
+ * Input preparation from pre-activation logits ("Independent decisions on two
+ * axes": the erase gate b and the write gate w are sigmoids of their own linear
+ * projections; "Token processing and parallel training": the query and key paths
+ * end in SiLU then L2 normalisation, the value path in SiLU).  The pages give the
+ * channel-wise decay alpha without its parameterisation; it is taken here as
+ * alpha = exp(-softplus(xa)), the usual log-space gate, which is in (0, 1).
+ * Per token row and head:
+ *   q = silu(xq) / ||silu(xq)||_2   (a zero row stays zero)      [dk]
+ *   k = silu(xk) / ||silu(xk)||_2                                 [dk]
+ *   v = silu(xv)                                                  [dv]
+ *   alpha = exp(-softplus(xa)) = exp(-log(1 + exp(xa)))           [dk]
+ *   b = sigmoid(xb),  w = sigmoid(xw)                             [dk], [dv]
+ * with silu(x) = x sigmoid(x) and sigmoid(x) = 1 / (1 + exp(-x)).  rows = B*T*H.
+ */
+static double prep_sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+static double prep_softplus(double x) { return x > 0 ? x + log1p(exp(-x)) : log1p(exp(x)); }
+
+static void prep_silu_l2(const double *x, double *y, int d) {
+    double ss = 0.0;
+    for (int i = 0; i < d; ++i) {
+        y[i] = x[i] * prep_sigmoid(x[i]);
+        ss += y[i] * y[i];
+    }
+    const double inv = ss > 0.0 ? 1.0 / sqrt(ss) : 0.0;
+    for (int i = 0; i < d; ++i) y[i] *= inv;
+}
+
+void oracle_gdn2_prep(long long rows, int dk, int dv,
+                      const double *xq, const double *xk, const double *xv,
+                      const double *xa, const double *xb, const double *xw,
+                      double *q, double *k, double *v, double *alpha, double *b, double *w) {
+#pragma omp parallel for schedule(static)
+    for (long long r = 0; r < rows; ++r) {
+        const size_t ok = (size_t)r * dk, ov = (size_t)r * dv;
+        prep_silu_l2(xq + ok, q + ok, dk);
+        prep_silu_l2(xk + ok, k + ok, dk);
+        for (int i = 0; i < dk; ++i) {
+            alpha[ok + i] = exp(-prep_softplus(xa[ok + i]));
+            b[ok + i] = prep_sigmoid(xb[ok + i]);
+        }
+        for (int j = 0; j < dv; ++j) {
+            v[ov + j] = xv[ov + j] * prep_sigmoid(xv[ov + j]);
+            w[ov + j] = prep_sigmoid(xw[ov + j]);
+        }
+    }
 }
