@@ -50,6 +50,7 @@ def _bind(path):
     lib.oracle_b0_sum.argtypes = [i] * 5 + [dp] * 7
     lib.oracle_gdn2_bwd.argtypes = [i] * 5 + [dp] * 16
     lib.oracle_gdn2_prep.argtypes = [ctypes.c_longlong, i, i] + [dp] * 12
+    lib.oracle_output_gate.argtypes = [ctypes.c_longlong, i, dp, dp, dp, ctypes.c_double, dp]
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
 
@@ -197,3 +198,15 @@ def gdn2_from_logits(xq, xk, xv, xa, xb, xw, S0=None, *, lib=None):
     """:func:`gdn2` applied to :func:`gdn2_prep` of the logits ([B,T,H,d] each)."""
     x = gdn2_prep(xq, xk, xv, xa, xb, xw, lib=lib)
     return gdn2(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], S0, lib=lib)
+
+
+def output_gate(o, g, weight, eps=1e-6, *, lib=None):
+    """Output epilogue of "Token processing and parallel training" (RMS norm, then a
+    separate output gate): per row of the last axis, y = o / sqrt(mean(o^2) + eps) * weight
+    * sigmoid(g).  The norm's per-channel weight, the epsilon and the sigmoid form of the
+    gate are this package's readings.  o, g [..., dv]; weight [dv].  Returns float64."""
+    o, g, weight = map(_f64, (o, g, weight))
+    dv = o.shape[-1]
+    y = np.empty_like(o)
+    _load(lib).oracle_output_gate(o.size // dv, dv, _ptr(o), _ptr(g), _ptr(weight), float(eps), _ptr(y))
+    return y

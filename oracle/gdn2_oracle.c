@@ -26,6 +26,7 @@
  *   oracle_gdn2_bwd  gradient of oracle_gdn2 (reverse mode through its token loop)
  *   oracle_gdn2_prep the activations that turn pre-activation logits into the
  *                    recurrence's inputs (q, k, v, alpha, b, w)
+ *   oracle_output_gate  RMS norm and sigmoid output gate applied to the recurrence's output
  */
 #include <math.h>
 #include <stdlib.h>
@@ -402,5 +403,28 @@ void oracle_gdn2_prep(long long rows, int dk, int dv,
             v[ov + j] = xv[ov + j] * prep_sigmoid(xv[ov + j]);
             w[ov + j] = prep_sigmoid(xw[ov + j]);
         }
+    }
+}
+
+/*
+ * Output epilogue ("Token processing and parallel training": after the recurrent
+ * update, RMS normalisation and a separate output gate, distinct from the write
+ * gate, come before the output projection).  The pages name the two steps but
+ * not their exact form; the readings taken here: the RMS norm runs over each
+ * head's d_v channels with a learned per-channel scale and an epsilon, and the
+ * output gate is a sigmoid of its own logits, like the pages' other gates:
+ *   y = o / sqrt(mean_j(o_j^2) + eps) * weight * sigmoid(g)
+ * per row (one token and head) of rows = B*T*H rows of dv channels.
+ */
+void oracle_output_gate(long long rows, int dv, const double *o, const double *g, const double *weight,
+                        double eps, double *y) {
+#pragma omp parallel for schedule(static)
+    for (long long r = 0; r < rows; ++r) {
+        const double *orow = o + (size_t)r * dv, *grow = g + (size_t)r * dv;
+        double ms = 0.0;
+        for (int j = 0; j < dv; ++j) ms += orow[j] * orow[j];
+        ms /= dv;
+        const double inv = 1.0 / sqrt(ms + eps);
+        for (int j = 0; j < dv; ++j) y[(size_t)r * dv + j] = orow[j] * inv * weight[j] / (1.0 + exp(-grow[j]));
     }
 }
