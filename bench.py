@@ -8,7 +8,10 @@ state, S0 = 0).  One timed step = one gdn2_chunk_fwd call on that batch (one
 kernel launch).  The decode step (batch 256, H=16, d=128, FP32 state, 64
 consecutive in-place steps) is timed in the same run and reported under
 "decode" as state GB/s; the chunkwise backward (gdn2_chunk_bwd: gradients of
-every input of the prefill workload) under "backward" as tokens/s.
+every input of the prefill workload) under "backward" as tokens/s, and the
+prefill from BF16 pre-activation logits (gdn2_chunk_fwd_logits) under
+"prefill_logits", and the output epilogue (gdn2_output_gate) under
+"output_gate".
 
 * value      device time, inputs resident in HBM, CUDA events on the launching
              stream, max over ranks; inputs (675 MB) exceed the 126 MB L2.
@@ -98,6 +101,18 @@ def backward_bytes(B, T, H, dk, dv):
     written.  The workspace (chunk-boundary states, T, P, U, dR) is not counted."""
     per = 2 * (2 * dk + dv) + 4 * (2 * dk + dv) + 2 * dv + 2 * (2 * dk + dv) + 4 * (2 * dk + dv)
     return B * T * H * per + B * H * dk * dv * 4
+
+
+def logits_bytes(B, T, H, dk, dv):
+    """Algorithmic HBM bytes of one logits prefill: six BF16 logit tensors read and BF16 o
+    written (1,792 B per token-head at d = 128), plus the FP32 final state."""
+    return B * T * H * (2 * (4 * dk + 2 * dv) + 2 * dv) + B * H * dk * dv * 4
+
+
+def output_gate_bytes(B, T, H, dv, es=2):
+    """Algorithmic bytes of the output epilogue: o and g read, y written (768 B per
+    token-head in BF16 at d_v = 128) and the weight vector."""
+    return B * T * H * dv * es * 3 + dv * 4
 
 
 def decode_bytes(B, H, dk, dv):
@@ -326,7 +341,13 @@ def run_ours(args):
     bwd_ms = float("nan")
     if args.workload in ("all", "backward"):
         bwd_ms = run_backward(args, torch, dist, g, world, rank, dev, stream)
-    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms, bwd_ms)
+    lg_ms = float("nan")
+    if args.workload in ("all", "logits"):
+        lg_ms = run_prefill_logits(args, torch, dist, g, world, rank, dev, stream)
+    og_ms = float("nan")
+    if args.workload in ("all", "output_gate"):
+        og_ms = run_output_gate(args, torch, dist, g, world, rank, dev, stream)
+    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms, bwd_ms, lg_ms, og_ms)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -490,6 +511,66 @@ def run_backward(args, torch, dist, g, world, rank, dev, stream):
     return ms
 
 
+def run_prefill_logits(args, torch, dist, g, world, rank, dev, stream):
+    """gdn2_chunk_fwd_logits on the prefill workload (BF16 logits, activations and gates
+    inside the kernel); returns ms per call."""
+    B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
+    x = gi.logit_inputs(B, T, H, dk, dv, seed=rank)
+    d = {n: torch.from_numpy(x[n]).to(dev).to(torch.bfloat16) for n in ("xq", "xk", "xv", "xa", "xb", "xw")}
+    del x
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    ST = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+
+    def call():
+        g.gdn2_chunk_fwd_logits(d["xq"], d["xk"], d["xv"], d["xa"], d["xb"], d["xw"], None, o=o, S_T=ST,
+                                stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    sync_ranks(torch, dist, world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(3, args.steps)
+    ev0.record(stream)
+    for _ in range(reps):
+        call()
+    ev1.record(stream)
+    sync_ranks(torch, dist, world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / reps, torch, dist, world, dev)
+    del d, o, ST
+    torch.cuda.empty_cache()
+    return ms
+
+
+def run_output_gate(args, torch, dist, g, world, rank, dev, stream):
+    """gdn2_output_gate on the prefill workload's output shape (BF16 o and gate logits);
+    returns ms per call."""
+    B, T, H, dv = (PREFILL[n] for n in ("B", "T", "H", "dv"))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(200 + rank)
+    o = torch.randn((B, T, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    gl = torch.randn((B, T, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    w = torch.rand((dv,), generator=gen, device=dev) + 0.5
+    y = torch.empty_like(o)
+
+    def call():
+        g.gdn2_output_gate(o, gl, w, 1e-6, y=y, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    sync_ranks(torch, dist, world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(10, args.steps)
+    ev0.record(stream)
+    for _ in range(reps):
+        call()
+    ev1.record(stream)
+    sync_ranks(torch, dist, world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / reps, torch, dist, world, dev)
+    del o, gl, w, y
+    torch.cuda.empty_cache()
+    return ms
+
+
 def bench_config(world):
     """The workload description both arms print (the reference arm times the same workload)."""
     B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
@@ -504,7 +585,8 @@ def _num(x):
     return None if x != x else x      # NaN (workload not run) -> null
 
 
-def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=float("nan"), bwd_ms=float("nan")):
+def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=float("nan"), bwd_ms=float("nan"),
+           lg_ms=float("nan"), og_ms=float("nan")):
     B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
     Bd, Hd = DECODE["B"], DECODE["H"]
     steps_d = DECODE["steps"]
@@ -523,6 +605,10 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=fl
     atflops = algo_flops / (ms_step / 1e3) / 1e12
     bpeak, bsrc = measured_bf16_peak()
 
+    og_bytes = output_gate_bytes(B, T, H, dv)
+    og_gbs = og_bytes / (og_ms / 1e3) / 1e9
+    lg_bytes = logits_bytes(B, T, H, dk, dv)
+    lg_gbs = lg_bytes / (lg_ms / 1e3) / 1e9
     bwd_bytes = backward_bytes(B, T, H, dk, dv)
     bwd_gbs = bwd_bytes / (bwd_ms / 1e3) / 1e9
     cpu = dec_cpu = long_cpu = bwd_cpu = None
@@ -579,6 +665,20 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=fl
                                       "note": "whole call (prep + state + grad launches) against the "
                                               "algorithmic bytes; workspace traffic not counted"},
                          "cpu_baseline": bwd_cpu},
+            "prefill_logits": {"metric": "GDN-2 chunk fwd from BF16 logits tokens/s @H16 d128 T4K",
+                               "unit": "tokens/s", "value": _num(job_tokens_per_s(B, T, world, lg_ms)),
+                               "ms_per_call": _num(lg_ms),
+                               "workload": "the prefill workload from BF16 pre-activation logits (SiLU, L2 norm, "
+                                           "sigmoid gates and the decay inside the kernel)",
+                               "roofline": {"bound": "hbm", "achieved": _num(lg_gbs), "peak": hbm, "unit": "GB/s",
+                                            "frac": _num(lg_gbs / hbm), "traffic": traffic.get("gdn2_chunk_logits"),
+                                            "algorithmic_bytes_per_launch": lg_bytes}},
+            "output_gate": {"metric": "GDN-2 output epilogue (RMS norm + sigmoid gate) tokens/s @H16 d128",
+                            "unit": "tokens/s", "value": _num(job_tokens_per_s(B, T, world, og_ms)),
+                            "us_per_call": _num(og_ms * 1e3),
+                            "roofline": {"bound": "hbm", "achieved": _num(og_gbs), "peak": hbm, "unit": "GB/s",
+                                         "frac": _num(og_gbs / hbm), "traffic": traffic.get("gdn2_output_gate"),
+                                         "algorithmic_bytes_per_launch": og_bytes}},
             "gpu_launches": args.steps,
             "clocks": clk.summary() if clk is not None else None,
             "cpu_baseline": cpu,
@@ -642,7 +742,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["all", "prefill", "decode", "long", "backward"], default="all",
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "long", "backward", "logits", "output_gate"], default="all",
                     help="run only one workload's measurement (for profiling one kernel)")
     args = ap.parse_args()
     if args.impl == "ours":

@@ -9,7 +9,9 @@ Functions (same names as the C ABI):
   gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, ...)  -> (o, S_T)   chunkwise prefill
   gdn2_chunk_fwd_varlen(q, k, v, alpha, b, w, cu_seqlens, S0=None, ...)
                                                       -> (o, S_T)   packed variable-length batch
+  gdn2_chunk_fwd_logits(xq, xk, xv, xa, xb, xw, S0=None, ...) -> (o, S_T)  prefill from BF16 logits
   gdn2_recurrent_step(q, k, v, alpha, b, w, S, ...)   -> o          in-place decode step
+  gdn2_output_gate(o, g, weight, eps, ...)            -> y          RMS norm + sigmoid output gate
   gdn2_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dST, ...) -> dict    gradients of every input
   gdn2_chunk_bwd_workspace_size(B, T, H, dk, dv)      -> bytes      workspace of gdn2_chunk_bwd
   gdn2_chunk_bwd_noalloc(..., out)                    -> dict       the same, workspace inside the library
@@ -24,7 +26,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_recurrent_step", "gdn2_chunk_bwd",
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_logits", "gdn2_output_gate", "gdn2_recurrent_step", "gdn2_chunk_bwd",
            "gdn2_chunk_bwd_workspace_size", "gdn2_chunk_bwd_noalloc", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
            "load_library", "exported_symbols",
            "GDN2_OK", "GDN2_ERR_INVALID_ARG", "GDN2_ERR_UNSUPPORTED", "GDN2_ERR_CUDA", "Gdn2Error"]
@@ -60,6 +62,10 @@ def load_library(rebuild_if_stale: bool = True) -> ctypes.CDLL:
     lib.gdn2_chunk_fwd.restype = i
     lib.gdn2_chunk_fwd_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, i, fp, vp, fp, i, i, i, i, i, vp]
     lib.gdn2_chunk_fwd_varlen.restype = i
+    lib.gdn2_chunk_fwd_logits.argtypes = [vp, vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
+    lib.gdn2_chunk_fwd_logits.restype = i
+    lib.gdn2_output_gate.argtypes = [vp, vp, fp, ctypes.c_float, vp, i, i, i, i, i, vp]
+    lib.gdn2_output_gate.restype = i
     lib.gdn2_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn2_recurrent_step.restype = i
     sz = ctypes.c_size_t
@@ -206,6 +212,56 @@ def gdn2_chunk_fwd_varlen(q, k, v, alpha, b, w, cu_seqlens, S0=None, *, o=None, 
         _check(lib.gdn2_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(cu_seqlens),
                                          N, _ptr(S0), _ptr(o), _ptr(S_T), T, H, dk, dv, code, _stream(stream, dev)))
     return o, S_T
+
+
+def gdn2_chunk_fwd_logits(xq, xk, xv, xa, xb, xw, S0=None, *, o=None, S_T=None, output_final_state=True,
+                          stream=None):
+    """Chunkwise prefill from BF16 pre-activation logits [B,T,H,128] each (activations and
+    gates computed inside the kernel); S0 [B,H,128,128] fp32 or None.  Returns (o, S_T)."""
+    lib = load_library()
+    if xq.device.type != "cuda":
+        raise ValueError("gdn2_chunk_fwd_logits needs CUDA tensors (there is no CPU implementation)")
+    B, T, H, dk = xq.shape
+    dv = xv.shape[-1]
+    dev = xq.device
+    for name, t, d in (("xq", xq, dk), ("xk", xk, dk), ("xv", xv, dv), ("xa", xa, dk), ("xb", xb, dk),
+                       ("xw", xw, dv)):
+        _need(t, name, torch.bfloat16, (B, T, H, d), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    else:
+        _need(o, "o", torch.bfloat16, (B, T, H, dv), dev)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    elif S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        _check(lib.gdn2_chunk_fwd_logits(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(xa), _ptr(xb), _ptr(xw), _ptr(S0),
+                                         _ptr(o), _ptr(S_T), B, T, H, dk, dv, _stream(stream, dev)))
+    return o, S_T
+
+
+def gdn2_output_gate(o, g, weight, eps=1e-6, *, y=None, stream=None):
+    """Output epilogue: y = o / sqrt(mean(o^2) + eps) * weight * sigmoid(g) per (token, head) row.
+    o, g [B,T,H,dv] (bf16 or fp32, same dtype), weight [dv] fp32; y may be o (in place)."""
+    lib = load_library()
+    if o.device.type != "cuda":
+        raise ValueError("gdn2_output_gate needs CUDA tensors (there is no CPU implementation)")
+    B, T, H, dv = o.shape
+    dev, dt = o.device, o.dtype
+    code = _dtype_code(o)
+    _need(g, "g", dt, (B, T, H, dv), dev)
+    _need(weight, "weight", torch.float32, (dv,), dev)
+    if y is None:
+        y = torch.empty_like(o)
+    else:
+        _need(y, "y", dt, (B, T, H, dv), dev)
+    with torch.cuda.device(dev):
+        _check(lib.gdn2_output_gate(_ptr(o), _ptr(g), _ptr(weight), float(eps), _ptr(y), B, T, H, dv, code,
+                                    _stream(stream, dev)))
+    return y
 
 
 def gdn2_recurrent_step(q, k, v, alpha, b, w, S, *, o=None, stream=None):

@@ -138,8 +138,11 @@ struct Kb {
 //   TP  [units][nch][2][64][64]  T = (I + A)^{-1}, then P
 //   U, dR [B][T][H][dv]        per token, laid out like o
 //   KB  [units][nch][Kb::floats]  the key block above
+//   DPA [units][nch][2][64][64]   dP, then dA (masked)
+//   XS  [units][nch][3][64][dk]   S dO, S dR, dS' U as [token][channel]
+//   RS  [units][nch][dk]          row sums of S * dS'
 struct Ws {
-    float *Sc, *dSc, *TP, *U, *dR, *KB;
+    float *Sc, *dSc, *TP, *U, *dR, *KB, *DPA, *XS, *RS;
 };
 
 // ---------------------------------------------------------------------------
@@ -219,33 +222,67 @@ struct Wt {
 };
 
 // ---------------------------------------------------------------------------
-// prep: A, P, T of one chunk.
+// prep: A, P, T of one chunk.  The chunk is cut into four 16-token blocks.  For a
+// key s in an earlier block than the row t, the decay 2^(G_t - G_s) is split at
+// the first token r of t's block into 2^(G_t - G_r) 2^(G_r - G_s), both at most 1
+// (s < r <= t), so those entries are products of scaled tiles on the tensor cores;
+// the four 16 x 16 diagonal blocks take each pair's decay directly.
 template <int DK>
 struct PrepSmem {
-    static constexpr int LB = 33;
-    static constexpr size_t floats = 5 * (size_t)kC * LB + 3 * (size_t)kC * LDT;
+    static constexpr int LB = 33, LE = 36;
+    // per channel block: cg, cl, ck, ce, cq [64][LB]; Er, Qr [48][LE]; Kr [96][LE]
+    static constexpr size_t blk = 5 * (size_t)kC * LB + (48 + 48 + 96) * (size_t)LE;
+    // after the channel loop: A, P, T [64][LDT], over the same memory
+    static constexpr size_t fin = 3 * (size_t)kC * LDT;
+    static constexpr size_t floats = blk > fin ? blk : fin;
     static constexpr size_t bytes = floats * sizeof(float);
 };
+
+// Rows of Kr: block tau = 1, 2, 3 holds the keys s < 16 tau scaled to reference 16 tau.
+__device__ __forceinline__ int kr_offset(int tau) { return tau == 1 ? 0 : (tau == 2 ? 16 : 48); }
 
 template <typename TIn, int DK, int DV>
 __global__ void __launch_bounds__(kThreads)
 bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const float *__restrict__ alpha,
                 const float *__restrict__ bgate, float *TP, float *KB, int T, int H) {
     using L = Kb<DK, DV>;
-    constexpr int LB = PrepSmem<DK>::LB;
+    constexpr int LB = PrepSmem<DK>::LB, LE = PrepSmem<DK>::LE;
     extern __shared__ float smem[];
     float *cg = smem, *cl = cg + kC * LB, *ck = cl + kC * LB, *ce = ck + kC * LB, *cq = ce + kC * LB;
-    float *sA = cq + kC * LB, *sP = sA + kC * LDT, *sT = sP + kC * LDT;
+    float *Er = cq + kC * LB, *Qr = Er + 48 * LE, *Kr = Qr + 48 * LE;
+    float *sA = smem, *sP = sA + kC * LDT, *sT = sP + kC * LDT;     // after the channel loop
     const int c = blockIdx.x, unit = blockIdx.y, seq = unit / H, h = unit % H, tid = threadIdx.x;
+    const int warp = tid >> 5;
     const int nch = gridDim.x, c0 = c * kC, n = min(kC, T - c0);
     const size_t tok0 = (size_t)seq * T + c0;
     float *kb = KB + ((size_t)unit * nch + c) * L::floats;
 
-    // thread owns (t = tid/64 + 4r, s = tid%64), r = 0..15
-    float a[16], p[16];
+    // Off-diagonal blocks: 12 n8 column blocks per matrix (tau = 1: 2, tau = 2: 4, tau = 3: 6);
+    // warps 0-3 build A from Er, warps 4-7 build P from Qr, three column blocks each.
+    Wt<1, 1> off[3];
+    int off_tau[3], off_nb[3];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) a[r] = p[r] = 0.f;
-    const int s = tid & 63, tb = tid >> 6;
+    for (int j = 0; j < 3; ++j) {
+        const int b = (warp & 3) * 3 + j;
+        off_tau[j] = b < 2 ? 1 : (b < 6 ? 2 : 3);
+        off_nb[j] = b - (off_tau[j] == 1 ? 0 : (off_tau[j] == 2 ? 2 : 6));
+        off[j].zero();
+    }
+    // Diagonal blocks: pair p = tid + 256 j of 4 x 136 (s <= t inside one 16-token block).
+    int pt[3], ps[3];
+    float pa[3], pp[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const int p = tid + j * kThreads;
+        const int blk = p / 136, qd = p - blk * 136;
+        int tt = (int)((sqrtf(8.f * qd + 1.f) - 1.f) * 0.5f);
+        while ((tt + 1) * (tt + 2) / 2 <= qd) ++tt;
+        while (tt * (tt + 1) / 2 > qd) --tt;
+        pt[j] = p < 4 * 136 ? blk * 16 + tt : -1;
+        ps[j] = p < 4 * 136 ? blk * 16 + qd - tt * (tt + 1) / 2 : -1;
+        pa[j] = pp[j] = 0.f;
+    }
+
     for (int ib = 0; ib < DK; ib += 32) {
         __syncthreads();
         {   // all loads first, then the transforms
@@ -256,11 +293,11 @@ bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const floa
                 const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
                 ra[e] = 1.f; rk[e] = rq[e] = rb[e] = 0.f;
                 if (t < n) {
-                    const size_t off = ((tok0 + t) * H + h) * DK + ib + i;
-                    ra[e] = __ldg(alpha + off);
-                    rk[e] = Elem<TIn>::load(k + off);
-                    rq[e] = Elem<TIn>::load(q + off);
-                    rb[e] = __ldg(bgate + off);
+                    const size_t off2 = ((tok0 + t) * H + h) * DK + ib + i;
+                    ra[e] = __ldg(alpha + off2);
+                    rk[e] = Elem<TIn>::load(k + off2);
+                    rq[e] = Elem<TIn>::load(q + off2);
+                    rb[e] = __ldg(bgate + off2);
                 }
             }
 #pragma unroll
@@ -285,28 +322,62 @@ bwd_prep_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const floa
             kb[L::QT + t * L::LK + ib + i] = cq[t * LB + i] * f;
             if (t == kC - 1) kb[L::GNF + ib + i] = f;
         }
+        // scaled tiles: Er, Qr rows t = 16..63 to reference r = 16 (t / 16); Kr as above
+        for (int idx = tid; idx < 48 * 32; idx += kThreads) {
+            const int t = 16 + (idx >> 5), i = idx & 31, r = t & ~15;
+            const float f = ex2(gdiff(cg[t * LB + i], cl[t * LB + i], cg[r * LB + i], cl[r * LB + i]));
+            Er[(t - 16) * LE + i] = ce[t * LB + i] * f;
+            Qr[(t - 16) * LE + i] = cq[t * LB + i] * f;
+        }
+        for (int idx = tid; idx < 96 * 32; idx += kThreads) {
+            const int row = idx >> 5, i = idx & 31;
+            const int tau = row < 16 ? 1 : (row < 48 ? 2 : 3), s2 = row - kr_offset(tau), r = 16 * tau;
+            Kr[row * LE + i] = ck[s2 * LB + i] * ex2(gdiff(cg[r * LB + i], cl[r * LB + i], cg[s2 * LB + i], cl[s2 * LB + i]));
+        }
+        __syncthreads();
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int t = tb + 4 * r;
-            if (s <= t) {
-                const float *gt = cg + t * LB, *gs = cg + s * LB, *lt = cl + t * LB, *ls = cl + s * LB,
-                            *ks = ck + s * LB, *et = ce + t * LB, *qt = cq + t * LB;
-                float aa = a[r], pp = p[r];
+        for (int j = 0; j < 3; ++j) {       // off-diagonal blocks on the tensor cores
+            const float *Am = (warp < 4 ? Er : Qr) + (off_tau[j] - 1) * 16 * LE;
+            off[j].run(Am, LE, 1, Kr, 1, LE, 32, 0, kr_offset(off_tau[j]) + off_nb[j] * 8);
+        }
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {       // diagonal blocks, pair by pair
+            if (pt[j] < 0) continue;
+            const int t = pt[j], s2 = ps[j];
+            const float *gt = cg + t * LB, *gs = cg + s2 * LB, *lt = cl + t * LB, *ls = cl + s2 * LB,
+                        *ks = ck + s2 * LB, *et = ce + t * LB, *qt = cq + t * LB;
+            float aa = pa[j], qq = pp[j];
 #pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const float kd = ks[i] * ex2(gdiff(gt[i], lt[i], gs[i], ls[i]));
-                    aa = fmaf(et[i], kd, aa);
-                    pp = fmaf(qt[i], kd, pp);
-                }
-                a[r] = aa; p[r] = pp;
+            for (int i = 0; i < 32; ++i) {
+                const float kd = ks[i] * ex2(gdiff(gt[i], lt[i], gs[i], ls[i]));
+                aa = fmaf(et[i], kd, aa);
+                qq = fmaf(qt[i], kd, qq);
             }
+            pa[j] = aa; pp[j] = qq;
+        }
+    }
+    __syncthreads();                        // sA, sP, sT now take the channel tiles' memory
+    for (int idx = tid; idx < kC * kC; idx += kThreads) {
+        const int t = idx >> 6, s2 = idx & 63;
+        if (s2 >= t) {                      // above the diagonal (and A's diagonal): zero
+            sA[t * LDT + s2] = 0.f;
+            if (s2 > t) sP[t * LDT + s2] = 0.f;
         }
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        const int t = tb + 4 * r;
-        sA[t * LDT + s] = (s < t) ? a[r] : 0.f;
-        sP[t * LDT + s] = (s <= t) ? p[r] : 0.f;
+    for (int j = 0; j < 3; ++j) {
+        const int tau = off_tau[j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = 16 * tau + off[j].row(0, 0, i), s2 = off[j].col(off_nb[j] * 8, 0, i);
+            (warp < 4 ? sA : sP)[t * LDT + s2] = off[j].c[0][0][i];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        if (pt[j] < 0) continue;
+        if (ps[j] < pt[j]) sA[pt[j] * LDT + ps[j]] = pa[j];
+        sP[pt[j] * LDT + ps[j]] = pp[j];
     }
     __syncthreads();
     // T = (I + A)^{-1}: column j by four lanes, x_t = -sum_{j<=s<t} A[t,s] x_s
@@ -568,52 +639,79 @@ bwd_state_kernel(const float *S0, const float *dST, float *dS0, Ws ws, int T, in
 }
 
 // ---------------------------------------------------------------------------
-// grad: per-token gradients of one chunk.  Key channels in blocks of 32.
+// grad_a: the contractions over the value columns of one chunk.
 template <int DV>
-struct GradSmem {
-    static constexpr int LDV = DV + 4, LB = 33;
-    static constexpr size_t floats = 3 * (size_t)kC * LDV + 2 * (size_t)kC * LDT + 2 * 32 * (size_t)LDV +
-                                     7 * (size_t)kC * LB + 32;
-    static_assert(2 * 32 * LDV >= kC * LB, "the lo tile fits where S and dS' were");
+struct GradASmem {
+    static constexpr int LDV = DV + 4;
+    static constexpr size_t floats = 3 * (size_t)kC * LDV + 2 * 32 * (size_t)LDV;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
 template <typename TIn, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
-                const float *__restrict__ alpha, const float *__restrict__ bgate, const float *__restrict__ wgate,
-                const TIn *__restrict__ dO, Ws ws, TIn *dq, TIn *dk, TIn *dvv, float *dalpha, float *db,
-                float *dw, int T, int H) {
-    constexpr int LDV = GradSmem<DV>::LDV, LB = GradSmem<DV>::LB;
-    extern __shared__ float smem[];
+bwd_grada_kernel(const TIn *__restrict__ v, const float *__restrict__ wgate, const TIn *__restrict__ dO, Ws ws,
+                 TIn *dvv, float *dw, int T, int H) {
+    constexpr int LDV = GradASmem<DV>::LDV;
+    extern __shared__ __align__(16) float smem[];
     const int warp = threadIdx.x >> 5;
     float *sO = smem, *sU = sO + kC * LDV, *sR = sU + kC * LDV;
-    float *dP = sR + kC * LDV, *dA = dP + kC * LDT;
-    float *sS = dA + kC * LDT, *sD = sS + 32 * LDV;
-    float *cg = sD + 32 * LDV, *ck = cg + kC * LB, *cq = ck + kC * LB, *ce = cq + kC * LB;
-    float *X1 = ce + kC * LB, *X2 = X1 + kC * LB, *Y = X2 + kC * LB;
-    float *rs = Y + kC * LB;
-    float *cl = sS;                     // lo parts of the cumulative log decay, once sS, sD are consumed
-
+    float *sS = sR + kC * LDV, *sD = sS + 32 * LDV;
     const int c = blockIdx.x, unit = blockIdx.y, seq = unit / H, h = unit % H, tid = threadIdx.x;
     const int nch = gridDim.x, c0 = c * kC, n = min(kC, T - c0);
     const size_t tok0 = (size_t)seq * T + c0;
     const size_t chunk = (size_t)unit * nch + c;
 
-    for (int idx = tid; idx < kC * DV; idx += kThreads) {
-        const int t = idx / DV, j = idx % DV;
-        float o = 0.f, u = 0.f, r = 0.f;
+    // U, dR of the chunk's valid rows (asynchronously), dO through registers; padding rows zero
+    for (int idx = tid; idx < kC * (DV / 4); idx += kThreads) {
+        const int t = idx / (DV / 4), j4 = (idx % (DV / 4)) * 4;
         if (t < n) {
-            const size_t off = ((tok0 + t) * H + h) * DV + j;
-            o = Elem<TIn>::load(dO + off);
-            u = ws.U[off];
-            r = ws.dR[off];
-            dw[off] = r * Elem<TIn>::load(v + off);
-            Elem<TIn>::store(dvv + off, r * __ldg(wgate + off));
+            const size_t off = ((tok0 + t) * H + h) * DV + j4;
+            cp_async16(sU + t * LDV + j4, ws.U + off);
+            cp_async16(sR + t * LDV + j4, ws.dR + off);
+        } else {
+            *reinterpret_cast<float4 *>(sU + t * LDV + j4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(sR + t * LDV + j4) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        sO[t * LDV + j] = o; sU[t * LDV + j] = u; sR[t * LDV + j] = r;
     }
+    cp_async_commit();
+    for (int base = 0; base < kC * DV; base += 8 * kThreads) {
+        float ro[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int idx = base + tid + e * kThreads, t = idx / DV, j = idx % DV;
+            ro[e] = t < n ? Elem<TIn>::load(dO + ((tok0 + t) * H + h) * DV + j) : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int idx = base + tid + e * kThreads;
+            sO[(idx / DV) * LDV + idx % DV] = ro[e];
+        }
+    }
+    cp_async_wait<0>();
     __syncthreads();
+    for (int base = 0; base < kC * DV; base += 8 * kThreads) {   // dw = dR v, dv = dR w
+        float rv[8], rw[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int idx = base + tid + e * kThreads, t = idx / DV, j = idx % DV;
+            rv[e] = rw[e] = 0.f;
+            if (t < n) {
+                const size_t off = ((tok0 + t) * H + h) * DV + j;
+                rv[e] = Elem<TIn>::load(v + off);
+                rw[e] = __ldg(wgate + off);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int idx = base + tid + e * kThreads, t = idx / DV, j = idx % DV;
+            if (t < n) {
+                const size_t off = ((tok0 + t) * H + h) * DV + j;
+                const float r = sR[t * LDV + j];
+                dw[off] = r * rv[e];
+                Elem<TIn>::store(dvv + off, r * rw[e]);
+            }
+        }
+    }
     {   // dP = dO U^T (s <= t), dA = -dR U^T (s < t); 64 x 64, 32 x 16 per warp
         const int m0 = (warp >> 2) * 32, n0 = (warp & 3) * 16;
         Wt<2, 2> wp, wa;
@@ -621,21 +719,101 @@ bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
         wa.zero();
         wp.run(sO, LDV, 1, sU, 1, LDV, DV, m0, n0);
         wa.run(sR, LDV, 1, sU, 1, LDV, DV, m0, n0);
+        float *dpa = ws.DPA + chunk * 2 * kC * kC;
 #pragma unroll
         for (int a = 0; a < 2; ++a)
 #pragma unroll
             for (int b = 0; b < 2; ++b)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int t = wp.row(m0, a, i), s = wp.col(n0, b, i);
-                    dP[t * LDT + s] = (s <= t) ? wp.c[a][b][i] : 0.f;
-                    dA[t * LDT + s] = (s < t) ? -wa.c[a][b][i] : 0.f;
+                    const int t = wp.row(m0, a, i), s2 = wp.col(n0, b, i);
+                    dpa[t * kC + s2] = (s2 <= t) ? wp.c[a][b][i] : 0.f;
+                    dpa[kC * kC + t * kC + s2] = (s2 < t) ? -wa.c[a][b][i] : 0.f;
                 }
     }
+    float *xs = ws.XS + chunk * 3 * kC * DK;
     for (int ib = 0; ib < DK; ib += 32) {
-        __syncthreads();
         copy_tile_async(sS, LDV, ws.Sc + chunk * DK * DV + (size_t)ib * DV, DV, 32, DV);
         copy_tile_async(sD, LDV, ws.dSc + chunk * DK * DV + (size_t)ib * DV, DV, 32, DV);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        {   // row sums of S * dS': eight lanes per row
+            const int i = tid >> 3, part = tid & 7;
+            float acc = 0.f;
+            for (int j = part; j < DV; j += 8) acc = fmaf(sS[i * LDV + j], sD[i * LDV + j], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+            if (part == 0) ws.RS[chunk * DK + ib + i] = acc;
+        }
+        {   // X1 = S dO, X2 = S dR, Y = dS' U, as [token][channel]; 64 x 32, 16 x 16 per warp
+            const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;
+            Wt<1, 2> x1, x2, y;
+            x1.zero();
+            x2.zero();
+            y.zero();
+            x1.run(sO, LDV, 1, sS, 1, LDV, DV, m0, n0);
+            x2.run(sR, LDV, 1, sS, 1, LDV, DV, m0, n0);
+            y.run(sU, LDV, 1, sD, 1, LDV, DV, m0, n0);
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = x1.row(m0, 0, i), ic = ib + x1.col(n0, b, i);
+                    xs[t * DK + ic] = x1.c[0][b][i];
+                    xs[kC * DK + t * DK + ic] = x2.c[0][b][i];
+                    xs[2 * kC * DK + t * DK + ic] = y.c[0][b][i];
+                }
+        }
+        __syncthreads();                    // sS, sD are refilled by the next block
+    }
+}
+
+// ---------------------------------------------------------------------------
+// grad_b: the per-token gradients of one chunk, key channels in blocks of 32.
+// The decay-weighted sums over pairs of tokens use the 16-token block split of
+// the prep kernel: pairs in different blocks go through scaled tiles on the
+// tensor cores, pairs inside one block are summed directly.
+//   rows:    sum_{s < r} dP[t,s] k_s 2^(G_t - G_s) = 2^(G_t - G_r) (dP Kr)[t]      (r: first token of t's block)
+//   columns: sum_{t in tau} (dA[t,s] e_t + dP[t,s] q_t) 2^(G_t - G_s)
+//          = 2^(G_r - G_s) (dA^T Er + dP^T Qr)[s]                                  (r: first token of block tau > s's)
+struct GradBSmem {
+    static constexpr int LP = kC + 4, LB = 36, LE = 40;
+    // dP, dA [64][LP]; per block: cg, cl, ck, cq, ce, X1, X2, Y, OQ, OE, OK [64][LB];
+    // Er, Qr [48][LE]; Kr, F [96][LE]; rs [32]
+    static constexpr size_t floats = 2 * (size_t)kC * LP + 11 * (size_t)kC * LB + (48 * 2 + 96 * 2) * (size_t)LE + 32;
+    static constexpr size_t bytes = floats * sizeof(float);
+};
+
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_gradb_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const float *__restrict__ alpha,
+                 const float *__restrict__ bgate, Ws ws, TIn *dq, TIn *dk, float *dalpha, float *db, int T, int H) {
+    constexpr int LP = GradBSmem::LP, LB = GradBSmem::LB, LE = GradBSmem::LE;
+    extern __shared__ __align__(16) float smem[];
+    float *dP = smem, *dA = dP + kC * LP;
+    float *cg = dA + kC * LP, *cl = cg + kC * LB, *ck = cl + kC * LB, *cq = ck + kC * LB, *ce = cq + kC * LB;
+    float *X1 = ce + kC * LB, *X2 = X1 + kC * LB, *Y = X2 + kC * LB;
+    float *OQ = Y + kC * LB, *OE = OQ + kC * LB, *OK = OE + kC * LB;
+    float *Er = OK + kC * LB, *Qr = Er + 48 * LE, *Kr = Qr + 48 * LE, *F = Kr + 96 * LE;
+    float *rs = F + 96 * LE;
+    const int c = blockIdx.x, unit = blockIdx.y, seq = unit / H, h = unit % H, tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int nch = gridDim.x, c0 = c * kC, n = min(kC, T - c0);
+    const size_t tok0 = (size_t)seq * T + c0;
+    const size_t chunk = (size_t)unit * nch + c;
+
+    copy_tile_async(dP, LP, ws.DPA + chunk * 2 * kC * kC, kC, kC, kC);
+    copy_tile_async(dA, LP, ws.DPA + chunk * 2 * kC * kC + kC * kC, kC, kC, kC);
+    cp_async_commit();
+    const float *xs = ws.XS + chunk * 3 * kC * DK;
+    for (int ib = 0; ib < DK; ib += 32) {
+        __syncthreads();
+        copy_tile_async(X1, LB, xs + ib, DK, kC, 32);
+        copy_tile_async(X2, LB, xs + kC * DK + ib, DK, kC, 32);
+        copy_tile_async(Y, LB, xs + 2 * kC * DK + ib, DK, kC, 32);
+        copy_tile_async(rs, 32, ws.RS + chunk * DK + ib, 32, 1, 32);
         cp_async_commit();
         {   // this block's key side: all loads first, then the transforms
             constexpr int E = kC * 32 / kThreads;
@@ -661,53 +839,93 @@ bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
                 ce[t * LB + i] = rb[e] * rk[e];
             }
         }
+        __syncthreads();
+        comp_cumsum<32>(cg, cl, LB);
+        // scaled tiles (both factors of every split decay are at most 1)
+        for (int idx = tid; idx < 48 * 32; idx += kThreads) {
+            const int t = 16 + (idx >> 5), i = idx & 31, r = t & ~15;
+            const float f = ex2(gdiff(cg[t * LB + i], cl[t * LB + i], cg[r * LB + i], cl[r * LB + i]));
+            Er[(t - 16) * LE + i] = ce[t * LB + i] * f;
+            Qr[(t - 16) * LE + i] = cq[t * LB + i] * f;
+        }
+        for (int idx = tid; idx < 96 * 32; idx += kThreads) {
+            const int row = idx >> 5, i = idx & 31;
+            const int tau = row < 16 ? 1 : (row < 48 ? 2 : 3), s2 = row - kr_offset(tau), r = 16 * tau;
+            const float f = ex2(gdiff(cg[r * LB + i], cl[r * LB + i], cg[s2 * LB + i], cl[s2 * LB + i]));
+            F[row * LE + i] = f;
+            Kr[row * LE + i] = ck[s2 * LB + i] * f;
+        }
+        for (int idx = tid; idx < 16 * 32; idx += kThreads) {     // no earlier block for rows 0-15,
+            const int t = idx >> 5, i = idx & 31;                 // no later block for keys 48-63
+            OQ[t * LB + i] = 0.f;
+            OE[t * LB + i] = 0.f;
+            OK[(48 + t) * LB + i] = 0.f;
+        }
         cp_async_wait<0>();
         __syncthreads();
-        {   // row sums of S * dS': eight lanes per row
-            const int i = tid >> 3, part = tid & 7;
-            float acc = 0.f;
-            for (int j = part; j < DV; j += 8) acc = fmaf(sS[i * LDV + j], sD[i * LDV + j], acc);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-            if (part == 0) rs[i] = acc;
-        }
-        {   // X1 = S dO, X2 = S dR, Y = dS' U, as [token][channel]; 64 x 32, 16 x 16 per warp
-            const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;
-            Wt<1, 2> x1, x2, y;
-            x1.zero();
-            x2.zero();
-            y.zero();
-            x1.run(sO, LDV, 1, sS, 1, LDV, DV, m0, n0);
-            x2.run(sR, LDV, 1, sS, 1, LDV, DV, m0, n0);
-            y.run(sU, LDV, 1, sD, 1, LDV, DV, m0, n0);
+        if (warp < 6) {
+            {   // rows of block tau = 1 + warp / 2 against all earlier keys: warp & 1 ? dA : dP
+                const int tau = 1 + (warp >> 1);
+                Wt<1, 4> w;
+                w.zero();
+                w.run((warp & 1 ? dA : dP) + 16 * tau * LP, LP, 1, Kr + kr_offset(tau) * LE, LE, 1, 16 * tau, 0, 0);
+                float *out = warp & 1 ? OE : OQ;
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
+                for (int b = 0; b < 4; ++b)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = x1.row(m0, 0, i), ic = x1.col(n0, b, i);
-                    X1[t * LB + ic] = x1.c[0][b][i];
-                    X2[t * LB + ic] = x2.c[0][b][i];
-                    Y[t * LB + ic] = y.c[0][b][i];
+                    for (int i = 0; i < 4; ++i) {
+                        const int t = 16 * tau + w.row(0, 0, i), ic = w.col(0, b, i), r = 16 * tau;
+                        out[t * LB + ic] = w.c[0][b][i] *
+                            ex2(gdiff(cg[t * LB + ic], cl[t * LB + ic], cg[r * LB + ic], cl[r * LB + ic]));
+                    }
+            }
+            {   // keys of block sigma = warp / 2, channels 16 (warp & 1) ..: every later block tau
+                const int sigma = warp >> 1, n0 = 16 * (warp & 1);
+                float acc[2][4];
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[b][i] = 0.f;
+                for (int tau = sigma + 1; tau < 4; ++tau) {
+                    Wt<1, 2> w;
+                    w.zero();
+                    w.run(dA + 16 * tau * LP, 1, LP, Er + 16 * (tau - 1) * LE, LE, 1, 16, 16 * sigma, n0);
+                    w.run(dP + 16 * tau * LP, 1, LP, Qr + 16 * (tau - 1) * LE, LE, 1, 16, 16 * sigma, n0);
+#pragma unroll
+                    for (int b = 0; b < 2; ++b)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int s2 = w.row(16 * sigma, 0, i), ic = w.col(n0, b, i);
+                            acc[b][i] = fmaf(F[(kr_offset(tau) + s2) * LE + ic], w.c[0][b][i], acc[b][i]);
+                        }
                 }
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int s2 = 16 * sigma + ((threadIdx.x & 31) >> 2) + (i >> 1) * 8;
+                        const int ic = n0 + b * 8 + 2 * (threadIdx.x & 3) + (i & 1);
+                        OK[s2 * LB + ic] = acc[b][i];
+                    }
+            }
         }
         __syncthreads();
-        comp_cumsum<32>(cg, cl, LB);        // S and dS' are consumed: cl takes their place
         float dlg[kC * 32 / kThreads];
 #pragma unroll
         for (int e = 0; e < kC * 32 / kThreads; ++e) {
             const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
+            const int r = t & ~15;
             const float gt = cg[t * LB + i], lt = cl[t * LB + i];
             const float gnh = cg[(kC - 1) * LB + i], gnl = cl[(kC - 1) * LB + i];
-            float sq = 0.f, se = 0.f, sk = 0.f;
-            for (int s = 0; s <= t; ++s) {          // dq, de: earlier keys of the chunk
-                const float r = ck[s * LB + i] * ex2(gdiff(gt, lt, cg[s * LB + i], cl[s * LB + i]));
-                sq = fmaf(dP[t * LDT + s], r, sq);
-                se = fmaf(dA[t * LDT + s], r, se);
+            float sq = OQ[t * LB + i], se = OE[t * LB + i], sk = OK[t * LB + i];
+            for (int s2 = r; s2 <= t; ++s2) {       // dq, de: earlier keys of t's own block
+                const float f = ck[s2 * LB + i] * ex2(gdiff(gt, lt, cg[s2 * LB + i], cl[s2 * LB + i]));
+                sq = fmaf(dP[t * LP + s2], f, sq);
+                se = fmaf(dA[t * LP + s2], f, se);
             }
-            for (int u = t; u < kC; ++u) {          // dk: later tokens of the chunk
-                const float r = ex2(gdiff(cg[u * LB + i], cl[u * LB + i], gt, lt));
-                sk = fmaf(fmaf(dA[u * LDT + t], ce[u * LB + i], dP[u * LDT + t] * cq[u * LB + i]), r, sk);
+            for (int u = t; u < r + 16; ++u) {      // dk: later tokens of t's own block
+                const float f = ex2(gdiff(cg[u * LB + i], cl[u * LB + i], gt, lt));
+                sk = fmaf(fmaf(dA[u * LP + t], ce[u * LB + i], dP[u * LP + t] * cq[u * LB + i]), f, sk);
             }
             const float ft = ex2(gt + lt);
             const float dqv = fmaf(ft, X1[t * LB + i], sq);
@@ -715,10 +933,11 @@ bwd_grad_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             const float kkey = fmaf(ex2(gdiff(gnh, gnl, gt, lt)), Y[t * LB + i], sk);
             const float kk = ck[t * LB + i];
             float l = dev * ce[t * LB + i] + dqv * cq[t * LB + i] - kkey * kk;
-            if (t == n - 1) {               // through g_n: diag(exp g_n) S and every Khat_s
+            if (t == n - 1) {               // through g_n: diag(2^g_n) S and every Khat_s
                 float kh = 0.f;
                 for (int s2 = 0; s2 < n; ++s2)
-                    kh = fmaf(ck[s2 * LB + i] * ex2(gdiff(gnh, gnl, cg[s2 * LB + i], cl[s2 * LB + i])), Y[s2 * LB + i], kh);
+                    kh = fmaf(ck[s2 * LB + i] * ex2(gdiff(gnh, gnl, cg[s2 * LB + i], cl[s2 * LB + i])),
+                              Y[s2 * LB + i], kh);
                 l += fmaf(ex2(gnh + gnl), rs[i], kh);
             }
             dlg[e] = (t < n) ? l : 0.f;
@@ -777,12 +996,14 @@ cudaError_t launch_bwd_typed(const void *q_, const void *k_, const void *v_, con
     auto kp = bwd_prep_kernel<TIn, DK, DV>;
     auto kp2 = bwd_prep2_kernel<TIn, DK, DV>;
     auto ks = bwd_state_kernel<DK, DV>;
-    auto kg = bwd_grad_kernel<TIn, DK, DV>;
+    auto kga = bwd_grada_kernel<TIn, DK, DV>;
+    auto kgb = bwd_gradb_kernel<TIn, DK>;
     cudaError_t err;
     if ((err = set_smem(kp, PrepSmem<DK>::bytes)) != cudaSuccess) return err;
     if ((err = set_smem(kp2, Prep2Smem<DV>::bytes)) != cudaSuccess) return err;
     if ((err = set_smem(ks, StateSmem<DK>::bytes)) != cudaSuccess) return err;
-    if ((err = set_smem(kg, GradSmem<DV>::bytes)) != cudaSuccess) return err;
+    if ((err = set_smem(kga, GradASmem<DV>::bytes)) != cudaSuccess) return err;
+    if ((err = set_smem(kgb, GradBSmem::bytes)) != cudaSuccess) return err;
     const dim3 grid_c((unsigned)nch, (unsigned)units);
     kp<<<grid_c, kThreads, PrepSmem<DK>::bytes, stream>>>(q, k, alpha, b, ws.TP, ws.KB, T, H);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -791,9 +1012,10 @@ cudaError_t launch_bwd_typed(const void *q_, const void *k_, const void *v_, con
     ks<<<dim3((unsigned)units, (unsigned)(DV / kCS)), kThreads, StateSmem<DK>::bytes, stream>>>(S0, dST, dS0, ws, T,
                                                                                                  H);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    kg<<<dim3((unsigned)nch, (unsigned)units), kThreads, GradSmem<DV>::bytes, stream>>>(
-        q, k, v, alpha, b, w, dO, ws, static_cast<TIn *>(dq), static_cast<TIn *>(dk), static_cast<TIn *>(dv), dalpha,
-        db, dw, T, H);
+    kga<<<grid_c, kThreads, GradASmem<DV>::bytes, stream>>>(v, w, dO, ws, static_cast<TIn *>(dv), dw, T, H);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    kgb<<<grid_c, kThreads, GradBSmem::bytes, stream>>>(q, k, alpha, b, ws, static_cast<TIn *>(dq),
+                                                         static_cast<TIn *>(dk), dalpha, db, T, H);
     return cudaGetLastError();
 }
 
@@ -824,7 +1046,7 @@ static size_t kb_floats(int dk, int dv) {
 size_t chunk_bwd_workspace_floats(int B, int T, int H, int dk, int dv) {
     const size_t nch = (size_t)(T + kC - 1) / kC, units = (size_t)B * H;
     return 2 * units * nch * dk * dv + units * nch * 2 * kC * kC + 2 * (size_t)B * T * H * dv +
-           units * nch * kb_floats(dk, dv);
+           units * nch * kb_floats(dk, dv) + units * nch * (2 * kC * kC + 3 * kC * dk + dk);
 }
 
 cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const float *b,
@@ -839,6 +1061,9 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
     ws.U = ws.TP + units * nch * 2 * kC * kC;
     ws.dR = ws.U + (size_t)B * T * H * d_v;
     ws.KB = ws.dR + (size_t)B * T * H * d_v;
+    ws.DPA = ws.KB + units * nch * kb_floats(d_k, d_v);
+    ws.XS = ws.DPA + units * nch * 2 * kC * kC;
+    ws.RS = ws.XS + units * nch * 3 * kC * d_k;
     if (dt == GDN2_BF16)
         return launch_bwd_dt<__nv_bfloat16>(q, k, v, alpha, b, w, S0, dO, dST, dq, dk, dv, dalpha, db, dw, dS0, ws, B,
                                             T, H, d_k, d_v, stream);

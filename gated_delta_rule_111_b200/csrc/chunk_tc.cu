@@ -56,6 +56,14 @@
 // The FP32 state lives in Tensor Memory: the state-update MMA accumulates
 // Ktil^T U onto it, the epilogue scales it by the chunk decay and writes the
 // TF32 copy that the next chunk's X product reads.
+//
+// Logits variant (kLogits): every input arrives as BF16 pre-activation logits.
+// alpha and b land as BF16 tiles in the first half of AT and BT; before the
+// decay products, the key side turns them into the FP32 gates (alpha =
+// exp(-softplus(x)) = 1 / (1 + e^x), b = sigmoid(x)); pass A applies SiLU and the
+// L2 norm over each token's 128 channels (a warp holds whole token rows) in FP32
+// as it reads the raw q, k logits.  The state side forms
+// z = sigmoid(x_w) silu(x_v) from BF16 loads.  The rest of the kernel is unchanged.
 #include <cudaTypedefs.h>
 #include <stdio.h>
 
@@ -119,6 +127,7 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 static_assert(OFF_REC % 16 == 0 && sizeof(ChunkRec) % 16 == 0, "record alignment");
 constexpr uint32_t TX_AB = 8 * TILE;                   // alpha and b of one chunk
+constexpr uint32_t TX_AB_LOGITS = 4 * TILE;            // their BF16 logits
 constexpr uint32_t TX_QK = 4 * TILE;                   // q and k of one chunk
 
 // Tensor Memory columns (512 allocated).
@@ -144,7 +153,7 @@ struct Maps {
 };
 struct Params {
     const __nv_bfloat16 *q, *k, *v;
-    const float *alpha, *b, *w;
+    const void *alpha, *b, *w;    // float gates, or BF16 logits in the logits variant
     const float *S0;
     __nv_bfloat16 *o;
     float *S_T;
@@ -201,6 +210,7 @@ __device__ __forceinline__ bool solo_wait(const Ctx &c, int which, uint32_t pari
     return true;
 }
 
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
@@ -211,6 +221,7 @@ __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 
 // products from the alpha tile, the chunk length, then in place alpha -> Qtil
 // and b -> Etil, and Ktil into KG.  Tokens past the chunk become padding (no
 // decay, zero rows).  Returns the chunk length n (uniform across the group).
+template <bool kLogits>
 __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int navail, int te, ChunkRec &r, bool el) {
     const int cg = ktid & 31, tg = ktid >> 5, lane = ktid & 31;
     const int tl0 = 8 * tg;
@@ -273,8 +284,29 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
         const uint2 kr = valid ? *reinterpret_cast<const uint2 *>(c.sm + OFF_KT + o16) : make_uint2(0u, 0u);
         const uint2 qr = valid ? *reinterpret_cast<const uint2 *>(c.sm + OFF_QT + o16) : make_uint2(0u, 0u);
         const float4 b4 = *reinterpret_cast<const float4 *>(c.sm + OFF_BT + o32);
-        const float kk[4] = {bf_lo(kr.x), bf_hi(kr.x), bf_lo(kr.y), bf_hi(kr.y)};
-        const float qq[4] = {bf_lo(qr.x), bf_hi(qr.x), bf_lo(qr.y), bf_hi(qr.y)};
+        float kk[4] = {bf_lo(kr.x), bf_hi(kr.x), bf_lo(kr.y), bf_hi(kr.y)};
+        float qq[4] = {bf_lo(qr.x), bf_hi(qr.x), bf_lo(qr.y), bf_hi(qr.y)};
+        if constexpr (kLogits) {     // q, k = silu(x) / ||silu(x)||, in FP32 from the raw logits;
+            float sk = 0.f, sq = 0.f; // the warp holds token t's 128 channels
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                kk[e] *= sigmoid_fast(kk[e]);
+                qq[e] *= sigmoid_fast(qq[e]);
+                sk = fmaf(kk[e], kk[e], sk);
+                sq = fmaf(qq[e], qq[e], sq);
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) {
+                sk += __shfl_xor_sync(0xffffffffu, sk, m);
+                sq += __shfl_xor_sync(0xffffffffu, sq, m);
+            }
+            const float ik = sk > 0.f ? rsqrtf(sk) : 0.f, iq = sq > 0.f ? rsqrtf(sq) : 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                kk[e] *= ik;
+                qq[e] *= iq;
+            }
+        }
         const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
         float e4[4], q4[4], k4[4];
 #pragma unroll
@@ -297,6 +329,38 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
         r.last = (t0 + n >= te) ? 1 : 0;
     }
     return n;
+}
+
+
+// Logits variant, before pass A (same thread layout: channels 4 cg .. 4 cg + 3 of
+// tokens 8 tg .. 8 tg + 7, so a warp holds whole token rows).  The input
+// preparation of "Token processing and parallel training" and "Independent
+// decisions on two axes", in shared memory:
+//   alpha = exp(-softplus(x)) = 1 / (1 + e^x),  b = sigmoid(x)   BF16 -> the FP32 tiles
+// (pass A applies SiLU and the L2 norm to q and k as it reads them).  Every raw
+// alpha / b value is read before the group barrier, since the FP32 tiles overlay
+// the BF16 ones.
+__device__ __forceinline__ void key_logits(const Ctx &c, int ktid) {
+    const int cg = ktid & 31, tg = ktid >> 5;
+    const int tl0 = 8 * tg;
+    uint2 ra[8], rb[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const uint32_t o16 = (cg >> 4) * TILE + swz128(tl0 + u, (cg & 15) * 8);
+        ra[u] = *reinterpret_cast<const uint2 *>(c.sm + OFF_AT + o16);
+        rb[u] = *reinterpret_cast<const uint2 *>(c.sm + OFF_BT + o16);
+    }
+    named_bar(kBarK, kGroup);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const uint32_t o32 = (cg >> 3) * TILE + swz128(tl0 + u, (cg & 7) * 16);
+        const float a4[4] = {bf_lo(ra[u].x), bf_hi(ra[u].x), bf_lo(ra[u].y), bf_hi(ra[u].y)};
+        const float b4[4] = {bf_lo(rb[u].x), bf_hi(rb[u].x), bf_lo(rb[u].y), bf_hi(rb[u].y)};
+        *reinterpret_cast<float4 *>(c.sm + OFF_AT + o32) =
+            make_float4(sigmoid_fast(-a4[0]), sigmoid_fast(-a4[1]), sigmoid_fast(-a4[2]), sigmoid_fast(-a4[3]));
+        *reinterpret_cast<float4 *>(c.sm + OFF_BT + o32) =
+            make_float4(sigmoid_fast(b4[0]), sigmoid_fast(b4[1]), sigmoid_fast(b4[2]), sigmoid_fast(b4[3]));
+    }
 }
 
 // Key side, pass B (thread per token t, channel half ch): the rows of Etil
@@ -333,12 +397,16 @@ __device__ __forceinline__ void key_kt(const Ctx &c, uint32_t tmem, int warp, in
 }
 
 // The chunk's alpha and b tiles (or q and k) by TMA.
+// FP32 gates: four 32-channel blocks each.  Logits: two 64-channel BF16 blocks each,
+// at the start of the same regions (key_logits turns them into the FP32 tiles).
+template <bool kLogits>
 __device__ __forceinline__ void load_ab(const Ctx &c, const Maps &m, int h, int t0) {
     const uint32_t fb = c.bar(B_FULL_AB);
-    mbar_expect_tx(fb, TX_AB);
-    for (int a = 0; a < 4; ++a) {
-        tma_load_3d(c.sa + OFF_AT + a * TILE, &m.alpha, 32 * a, h, t0, fb);
-        tma_load_3d(c.sa + OFF_BT + a * TILE, &m.b, 32 * a, h, t0, fb);
+    mbar_expect_tx(fb, kLogits ? TX_AB_LOGITS : TX_AB);
+    for (int a = 0; a < (kLogits ? 2 : 4); ++a) {
+        const int x = kLogits ? 64 * a : 32 * a;
+        tma_load_3d(c.sa + OFF_AT + a * TILE, &m.alpha, x, h, t0, fb);
+        tma_load_3d(c.sa + OFF_BT + a * TILE, &m.b, x, h, t0, fb);
     }
 }
 __device__ __forceinline__ void load_qk(const Ctx &c, const Maps &m, int h, int t0) {
@@ -528,6 +596,7 @@ __device__ __noinline__ void issuer_role(const Ctx &c, uint32_t tmem) {
 }
 
 // ---------------------------------------------------------------------------
+template <bool kLogits>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -585,7 +654,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
         const uint32_t tlane = tmem + ((uint32_t)(32 * lq) << 16);
         int t0 = tb;
         if (el && !empty) {
-            load_ab(c, maps, h, t0);
+            load_ab<kLogits>(c, maps, h, t0);
             load_qk(c, maps, h, t0);
         }
         int pend_ab = empty ? -1 : 0, pend_qk = pend_ab;   // chunk whose loads are in flight, not yet awaited
@@ -601,11 +670,12 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                 *reinterpret_cast<volatile int *>(c.sm + OFF_MISC + 8) = kC;
                 const int tn = t0 + kC;
                 if (tn < te) {      // the next chunk's w, v into L2 for the state side
-                    for (int a = 0; a < 2; ++a) tma_prefetch_3d(&maps.w, col0 + 32 * a, h, tn);
+                    for (int a = 0; a < (kLogits ? 1 : 2); ++a) tma_prefetch_3d(&maps.w, col0 + 32 * a, h, tn);
                     tma_prefetch_3d(&maps.v, col0, h, tn);
                 }
             }
-            const int n = key_decay(c, ktid, t0, navail, te, r, el);
+            if constexpr (kLogits) key_logits(c, ktid);
+            const int n = key_decay<kLogits>(c, ktid, t0, navail, te, r, el);
             const bool last = t0 + n >= te;
             fence_proxy_async_smem();
             named_bar(kBarK, kGroup);
@@ -626,7 +696,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
             if (el) {
                 mbar_arrive(c.bar(B_KPREP));
                 if (!last) {
-                    load_ab(c, maps, h, t0 + n);       // alpha, b consumed: the next chunk's
+                    load_ab<kLogits>(c, maps, h, t0 + n);       // alpha, b consumed: the next chunk's
                     pend_ab = ck + 1;
                 }
             }
@@ -729,17 +799,34 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                 if (srow < 64) {
                     if (srow < n) {
                         const size_t row = ((size_t)(t0 + srow) * p.H + h) * kDV + col0 + 32 * sh;
-                        const float4 *wp = reinterpret_cast<const float4 *>(p.w + row);
                         const uint4 *vp = reinterpret_cast<const uint4 *>(p.v + row);
+                        if constexpr (kLogits) {      // z = sigmoid(xw) silu(xv)
+                            const uint4 *wp = reinterpret_cast<const uint4 *>(
+                                static_cast<const __nv_bfloat16 *>(p.w) + row);
 #pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            const uint4 vb = __ldg(vp + m);
-                            const float4 w0 = __ldg(wp + 2 * m), w1 = __ldg(wp + 2 * m + 1);
-                            float *zp = z + 8 * m;
-                            zp[0] = w0.x * bf_lo(vb.x); zp[1] = w0.y * bf_hi(vb.x);
-                            zp[2] = w0.z * bf_lo(vb.y); zp[3] = w0.w * bf_hi(vb.y);
-                            zp[4] = w1.x * bf_lo(vb.z); zp[5] = w1.y * bf_hi(vb.z);
-                            zp[6] = w1.z * bf_lo(vb.w); zp[7] = w1.w * bf_hi(vb.w);
+                            for (int m = 0; m < 4; ++m) {
+                                const uint4 vb = __ldg(vp + m), wb = __ldg(wp + m);
+                                const float vv[8] = {bf_lo(vb.x), bf_hi(vb.x), bf_lo(vb.y), bf_hi(vb.y),
+                                                     bf_lo(vb.z), bf_hi(vb.z), bf_lo(vb.w), bf_hi(vb.w)};
+                                const float ww[8] = {bf_lo(wb.x), bf_hi(wb.x), bf_lo(wb.y), bf_hi(wb.y),
+                                                     bf_lo(wb.z), bf_hi(wb.z), bf_lo(wb.w), bf_hi(wb.w)};
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    z[8 * m + e] = sigmoid_fast(ww[e]) * vv[e] * sigmoid_fast(vv[e]);
+                            }
+                        } else {
+                            const float4 *wp = reinterpret_cast<const float4 *>(
+                                static_cast<const float *>(p.w) + row);
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {
+                                const uint4 vb = __ldg(vp + m);
+                                const float4 w0 = __ldg(wp + 2 * m), w1 = __ldg(wp + 2 * m + 1);
+                                float *zp = z + 8 * m;
+                                zp[0] = w0.x * bf_lo(vb.x); zp[1] = w0.y * bf_hi(vb.x);
+                                zp[2] = w0.z * bf_lo(vb.y); zp[3] = w0.w * bf_hi(vb.y);
+                                zp[4] = w1.x * bf_lo(vb.z); zp[5] = w1.y * bf_hi(vb.z);
+                                zp[6] = w1.z * bf_lo(vb.w); zp[7] = w1.w * bf_hi(vb.w);
+                            }
                         }
                     } else {
 #pragma unroll
@@ -890,9 +977,9 @@ cudaError_t read_device_error(unsigned int *value, bool clear) {
 
 // nseq sequences: of T tokens each (cu_seqlens == nullptr), or packed with
 // device offsets cu_seqlens[0..nseq] into T_total = T tokens.
-cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const float *b,
-                            const float *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
-                            const int *cu_seqlens, cudaStream_t stream) {
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *alpha, const void *b,
+                            const void *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
+                            const int *cu_seqlens, bool logits, cudaStream_t stream) {
     using namespace tc;
     const long long NT = cu_seqlens ? (long long)T : (long long)nseq * T;
     if (NT <= 0 && !cu_seqlens) return cudaSuccess;
@@ -901,15 +988,18 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     const long long NTm = NT > 0 ? NT : 1;
     if (!make_map(&m.q, q, BF, 2, NTm, H, kDK, 64, true) || !make_map(&m.k, k, BF, 2, NTm, H, kDK, 64, true) ||
         !make_map(&m.v, v, BF, 2, NTm, H, kDV, 64, false) ||
-        !make_map(&m.alpha, alpha, F32, 4, NTm, H, kDK, 32, true) ||
-        !make_map(&m.b, b, F32, 4, NTm, H, kDK, 32, true) || !make_map(&m.w, w, F32, 4, NTm, H, kDV, 32, false))
+        !make_map(&m.alpha, alpha, logits ? BF : F32, logits ? 2 : 4, NTm, H, kDK, logits ? 64 : 32, true) ||
+        !make_map(&m.b, b, logits ? BF : F32, logits ? 2 : 4, NTm, H, kDK, logits ? 64 : 32, true) ||
+        !make_map(&m.w, w, logits ? BF : F32, logits ? 2 : 4, NTm, H, kDV, logits ? 64 : 32, false))
         return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
     if (!bit || !(g_attr_set.load() & bit)) {
-        e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        e = cudaFuncSetAttribute(chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(chunk_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if (bit) g_attr_set.fetch_or(bit);
     }
@@ -928,7 +1018,10 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     prm.H = H;
     prm.wait_limit = g_wait_limit.load();
     const unsigned grid = 2u * (unsigned)nseq * (unsigned)H;
-    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(m, prm);
+    if (logits)
+        chunk_tc_kernel<true><<<grid, kThreads, SMEM_BYTES, stream>>>(m, prm);
+    else
+        chunk_tc_kernel<false><<<grid, kThreads, SMEM_BYTES, stream>>>(m, prm);
     return cudaGetLastError();
 }
 

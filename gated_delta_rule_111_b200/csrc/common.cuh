@@ -47,4 +47,8 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
                              void *dv, float *dalpha, float *db, float *dw, float *dS0, float *workspace, int B,
                              int T, int H, int d_k, int d_v, gdn2_dtype dt, cudaStream_t stream);
 
+// Output epilogue: rows = B*T*H rows of dv channels (dv 64 or 128).
+cudaError_t launch_output_gate(const void *o, const void *g, const float *weight, float eps, void *y,
+                               long long rows, int dv, gdn2_dtype dt, cudaStream_t stream);
+
 }  // namespace gdn2

@@ -6,9 +6,9 @@
 #include "common.cuh"
 
 namespace gdn2 {
-cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const float *b,
-                            const float *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
-                            const int *cu_seqlens, cudaStream_t stream);
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *alpha, const void *b,
+                            const void *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
+                            const int *cu_seqlens, bool logits, cudaStream_t stream);
 bool chunk_tc_supported(int dk, int dv, gdn2_dtype dt);
 void set_wait_limit(long long cycles);
 cudaError_t read_device_error(unsigned int *value, bool clear);
@@ -139,7 +139,7 @@ static gdn2_status chunk_fwd_common(const void *q, const void *k, const void *v,
 
     cudaError_t err;
     if (gdn2::chunk_tc_supported(d_k, d_v, dt))
-        err = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, nseq, T, H, cu, s);
+        err = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, nseq, T, H, cu, false, s);
     else
         err = gdn2::launch_chunk_simt(q, k, v, alpha, b, w, S0, o, S_T, nseq, T, H, d_k, d_v, dt, cu, s);
     return cuda_status(err, "gdn2_chunk_fwd launch");
@@ -215,6 +215,68 @@ gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v, const fl
     cudaError_t err = gdn2::launch_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dST, dq, dk, dv, dalpha, db, dw, dS0,
                                              static_cast<float *>(workspace), B, T, H, d_k, d_v, dt, s);
     return cuda_status(err, "gdn2_chunk_bwd launch");
+}
+
+gdn2_status gdn2_chunk_fwd_logits(const void *xq, const void *xk, const void *xv, const void *xa, const void *xb,
+                                  const void *xw, const float *S0, void *o, float *S_T, int B, int T, int H,
+                                  int d_k, int d_v, void *stream) {
+    g_last_error[0] = 0;
+    gdn2_status st = check_common(B, H, d_k, d_v, GDN2_BF16);
+    if (st != GDN2_OK) return st;
+    if (d_k != 128 || d_v != 128)
+        return fail(GDN2_ERR_UNSUPPORTED, "%s", "gdn2_chunk_fwd_logits: d_k = d_v = 128 only");
+    if (T < 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "negative T");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (B == 0 || H == 0) return GDN2_OK;
+    const size_t state_bytes = (size_t)B * H * d_k * d_v * sizeof(float);
+    if (S0 && (st = check_ptr(S0, "S0")) != GDN2_OK) return st;
+    if (S_T && (st = check_ptr(S_T, "S_T")) != GDN2_OK) return st;
+    if (S0 && S_T && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes))
+        return fail(GDN2_ERR_INVALID_ARG, "%s", "S_T partially overlaps S0 (only exact aliasing is allowed)");
+    if (T == 0) {
+        if (!S_T || S_T == S0) return GDN2_OK;
+        cudaError_t err = S0 ? cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, s)
+                             : cudaMemsetAsync(S_T, 0, state_bytes, s);
+        return cuda_status(err, "T = 0 state copy");
+    }
+    const void *ins[6] = {xq, xk, xv, xa, xb, xw};
+    const char *names[6] = {"xq", "xk", "xv", "xa", "xb", "xw"};
+    const size_t row_bytes = (size_t)B * T * H * 128 * 2;      // every logit tensor is [B][T][H][128] BF16
+    for (int i = 0; i < 6; ++i)
+        if ((st = check_ptr(ins[i], names[i])) != GDN2_OK) return st;
+    if ((st = check_ptr(o, "o")) != GDN2_OK) return st;
+    for (int i = 0; i < 6; ++i) {
+        if (overlaps(o, row_bytes, ins[i], row_bytes)) return fail(GDN2_ERR_INVALID_ARG, "o overlaps %s", names[i]);
+        if (S_T && overlaps(S_T, state_bytes, ins[i], row_bytes))
+            return fail(GDN2_ERR_INVALID_ARG, "S_T overlaps %s", names[i]);
+    }
+    if (overlaps(o, row_bytes, S0, state_bytes) || overlaps(o, row_bytes, S_T, state_bytes))
+        return fail(GDN2_ERR_INVALID_ARG, "%s", "o overlaps a state buffer");
+    cudaError_t err = gdn2::launch_chunk_tc(xq, xk, xv, xa, xb, xw, S0, o, S_T, B, T, H, nullptr, true, s);
+    return cuda_status(err, "gdn2_chunk_fwd_logits launch");
+}
+
+gdn2_status gdn2_output_gate(const void *o, const void *g, const float *weight, float eps, void *y, int B, int T,
+                             int H, int d_v, gdn2_dtype dt, void *stream) {
+    g_last_error[0] = 0;
+    if (B < 0 || T < 0 || H < 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "negative size");
+    if (dt != GDN2_BF16 && dt != GDN2_FP32) return fail(GDN2_ERR_UNSUPPORTED, "%s", "unknown dtype");
+    if (d_v != 64 && d_v != 128) return fail(GDN2_ERR_UNSUPPORTED, "%s", "d_v must be 64 or 128");
+    if (!(eps >= 0.f) || eps > 3.0e38f) return fail(GDN2_ERR_INVALID_ARG, "%s", "eps must be finite and >= 0");
+    const long long rows = (long long)B * T * H;
+    if (rows == 0) return GDN2_OK;
+    gdn2_status st;
+    if ((st = check_ptr(o, "o")) != GDN2_OK || (st = check_ptr(g, "g")) != GDN2_OK ||
+        (st = check_ptr(weight, "weight")) != GDN2_OK || (st = check_ptr(y, "y")) != GDN2_OK)
+        return st;
+    const size_t bytes = (size_t)rows * d_v * (dt == GDN2_BF16 ? 2 : 4);
+    if (y != o && overlaps(y, bytes, o, bytes))
+        return fail(GDN2_ERR_INVALID_ARG, "%s", "y partially overlaps o (only exact aliasing is allowed)");
+    if (overlaps(y, bytes, g, bytes)) return fail(GDN2_ERR_INVALID_ARG, "%s", "y overlaps g");
+    if (overlaps(y, bytes, weight, (size_t)d_v * sizeof(float)))
+        return fail(GDN2_ERR_INVALID_ARG, "%s", "y overlaps weight");
+    return cuda_status(gdn2::launch_output_gate(o, g, weight, eps, y, rows, d_v, dt, static_cast<cudaStream_t>(stream)),
+                       "gdn2_output_gate launch");
 }
 
 gdn2_status gdn2_recurrent_step(const void *q, const void *k, const void *v, const float *alpha,

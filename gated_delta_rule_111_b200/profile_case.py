@@ -1,8 +1,9 @@
-"""Run one prefill, decode or backward case a few times on seeded inputs, for profilers.
+"""Run one prefill, decode, backward or logits-prefill case a few times on seeded inputs, for profilers.
 
     python -m gated_delta_rule_111_b200.profile_case prefill --B 2 --T 4096 --H 16 --calls 3
     python -m gated_delta_rule_111_b200.profile_case decode --B 64 --H 16 --calls 3
     python -m gated_delta_rule_111_b200.profile_case backward --B 1 --T 4096 --H 16 --calls 2
+    python -m gated_delta_rule_111_b200.profile_case logits --B 2 --T 4096 --H 16 --calls 3
 
 Inputs come from ``gdn2_inputs`` (same recipe as the tests and ``bench.py``), are moved to the GPU
 once, and every call goes through the C ABI.  Nothing is checked or timed here: this exists so that
@@ -19,12 +20,13 @@ import torch
 sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 import gdn2_inputs as gi  # noqa: E402
 
-from . import gdn2_chunk_bwd, gdn2_chunk_bwd_workspace_size, gdn2_chunk_fwd, gdn2_recurrent_step  # noqa: E402
+from . import (gdn2_chunk_bwd, gdn2_chunk_bwd_workspace_size, gdn2_chunk_fwd, gdn2_chunk_fwd_logits,  # noqa: E402
+               gdn2_recurrent_step)
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("mode", choices=["prefill", "decode", "backward"])
+    ap.add_argument("mode", choices=["prefill", "decode", "backward", "logits"])
     ap.add_argument("--B", type=int, default=2)
     ap.add_argument("--T", type=int, default=4096)
     ap.add_argument("--H", type=int, default=16)
@@ -34,6 +36,16 @@ def main(argv=None):
     a = ap.parse_args(argv)
     tdt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
     dev = torch.device("cuda:0")
+    if a.mode == "logits":
+        x = gi.logit_inputs(a.B, a.T, a.H, a.d, a.d, seed=0)
+        lg = {n: torch.from_numpy(x[n]).to(dev).to(torch.bfloat16) for n in ("xq", "xk", "xv", "xa", "xb", "xw")}
+        o = torch.empty(a.B, a.T, a.H, a.d, dtype=torch.bfloat16, device=dev)
+        S_T = torch.empty(a.B, a.H, a.d, a.d, dtype=torch.float32, device=dev)
+        for _ in range(a.calls):
+            gdn2_chunk_fwd_logits(lg["xq"], lg["xk"], lg["xv"], lg["xa"], lg["xb"], lg["xw"], o=o, S_T=S_T)
+        torch.cuda.synchronize()
+        print(f"logits B={a.B} T={a.T} H={a.H} d={a.d}: {a.calls} calls done")
+        return
     if a.mode in ("prefill", "backward"):
         x = gi.chunk_inputs(a.B, a.T, a.H, a.d, a.d, dtype=a.dtype, seed=0)
     else:

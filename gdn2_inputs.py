@@ -99,6 +99,26 @@ def chunk_inputs(B, T, H, dk, dv, *, dtype="bf16", seed=0, s0_std=None, gates="g
     return out
 
 
+def logit_inputs(B, T, H, dk, dv, *, seed=0, s0_std=None, a_shift=-2.0):
+    """Pre-activation inputs for the logits prefill: xq, xk, xv, xb, xw ~ N(0, 1) and
+    xa ~ N(0, 1) + a_shift, each rounded to BF16 (the kernel reads BF16), [B,T,H,d];
+    S0 [B,H,dk,dv] or None.  With a_shift = -2 the decays have the distribution of
+    chunk_inputs' alpha."""
+    rng = np.random.default_rng(seed)
+    f32 = np.float32
+    out = {}
+    for n, d in (("xq", dk), ("xk", dk), ("xv", dv), ("xa", dk), ("xb", dk), ("xw", dv)):
+        x = rng.standard_normal((B, T, H, d), dtype=f32)
+        if n == "xa":
+            x = x + f32(a_shift)
+        out[n] = round_to_bf16(x)
+    out["S0"] = None
+    if s0_std is not None:
+        out["S0"] = (rng.standard_normal((B, H, dk, dv), dtype=f32) * f32(s0_std)).astype(f32)
+    out.update(B=B, T=T, H=H, dk=dk, dv=dv, dtype="bf16")
+    return out
+
+
 def decode_inputs(steps, B, H, dk, dv, *, dtype="bf16", seed=0, s0_std=0.02, gates="gdn2"):
     """Inputs for ``steps`` decode steps: tensors [steps,B,H,d] and S0 [B,H,dk,dv]."""
     rng = np.random.default_rng(seed)

@@ -121,6 +121,50 @@ gdn2_status gdn2_chunk_fwd_varlen(const void *q, const void *k, const void *v,
                                   gdn2_dtype dt, void *stream);
 
 /*
+ * Chunkwise prefill from pre-activation logits, with the input preparation fused
+ * into the tensor-core kernel ("Token processing and parallel training": the query
+ * and key paths end in SiLU and L2 normalisation, the value path in SiLU;
+ * "Independent decisions on two axes": the erase and write gates are sigmoids of
+ * their own projections).  Per token and head, inside the kernel:
+ *   q = silu(xq) / ||silu(xq)||_2,  k = silu(xk) / ||silu(xk)||_2  (a zero row stays zero)
+ *   v = silu(xv),  alpha = exp(-softplus(xa)) = 1 / (1 + e^xa),  b = sigmoid(xb),  w = sigmoid(xw)
+ * then the recurrence of gdn2_chunk_fwd (alpha's parameterisation is this
+ * library's reading: the paper does not give it).  Every input is BF16, which
+ * cuts the bytes read per token and head from 2,304 (BF16 q, k, v and FP32
+ * gates) to 1,536.  The activations and the norm are computed in FP32 from the
+ * BF16 logits; nothing is rounded back to BF16 on the way.
+ *
+ *   xq, xk, xa, xb  [B][T][H][128]  BF16   read
+ *   xv, xw          [B][T][H][128]  BF16   read
+ *   S0, o, S_T      as in gdn2_chunk_fwd (o BF16)
+ *
+ * d_k = d_v = 128 only (GDN2_ERR_UNSUPPORTED otherwise).  T = 0 writes S_T = S0;
+ * B = 0 or H = 0 is a no-op; o must not overlap any input.
+ */
+gdn2_status gdn2_chunk_fwd_logits(const void *xq, const void *xk, const void *xv,
+                                  const void *xa, const void *xb, const void *xw,
+                                  const float *S0, void *o, float *S_T,
+                                  int B, int T, int H, int d_k, int d_v, void *stream);
+
+/*
+ * Output epilogue ("Token processing and parallel training": after the recurrent
+ * update, RMS normalisation and a separate output gate, distinct from the write
+ * gate, come before the output projection).  Per (token, head) row of d_v
+ * channels, in one pass:
+ *   y = o / sqrt(mean_j(o_j^2) + eps) * weight * sigmoid(g)
+ * The paper names the two steps without their form; this library's readings are
+ * a norm over one head's channels with a per-channel weight, and a sigmoid gate.
+ *
+ *   o, g     [B][T][H][d_v]  dt      read (o: the recurrence's output; g: gate logits)
+ *   weight   [d_v]           float   read
+ *   y        [B][T][H][d_v]  dt      written; may alias o exactly (in place)
+ *
+ * d_v 64 or 128; eps finite and >= 0.  FP32 arithmetic, output rounded to dt.
+ */
+gdn2_status gdn2_output_gate(const void *o, const void *g, const float *weight, float eps, void *y,
+                             int B, int T, int H, int d_v, gdn2_dtype dt, void *stream);
+
+/*
  * Chunkwise backward ("Token processing and parallel training": training goes
  * through the chunkwise form, so its gradient carries the channel-wise decay and
  * the separate erase and write gates through every per-block factor).  Computes

@@ -168,7 +168,9 @@ def test_backward_host_checks(lib):
     # chunk states and gradients, T and P, U and dR per token, and the key block
     # (five [64][132] tiles, two [64][132], one [128][132], 128 decay factors)
     key_block = 5 * 64 * 132 + 2 * 64 * 132 + 128 * 132 + 128
-    assert need == 4 * (2 * 128 * 128 + 2 * 64 * 64 + 2 * 10 * 128 + key_block)
+    # and the gradient kernels' hand-over: dP and dA, S dO / S dR / dS' U, row sums
+    grad_block = 2 * 64 * 64 + 3 * 64 * 128 + 128
+    assert need == 4 * (2 * 128 * 128 + 2 * 64 * 64 + 2 * 10 * 128 + key_block + grad_block)
     assert _bwd(lib, ws_bytes=need - 4) == g.GDN2_ERR_INVALID_ARG
     assert b"workspace" in lib.gdn2_last_error()
     assert _bwd(lib, ws=None) == g.GDN2_ERR_INVALID_ARG
@@ -183,3 +185,26 @@ def test_backward_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         g.gdn2_chunk_bwd(x, x, x, x, x, x)
+
+
+def test_logits_host_checks(lib):
+    args = [A16 * (1 + i) for i in range(6)]
+    assert lib.gdn2_chunk_fwd_logits(*args, None, A16 * 64, None, 1, 10, 1, 64, 64, None) == g.GDN2_ERR_UNSUPPORTED
+    assert lib.gdn2_chunk_fwd_logits(*args, None, A16 * 64, None, 1, -1, 1, 128, 128, None) == g.GDN2_ERR_INVALID_ARG
+    assert lib.gdn2_chunk_fwd_logits(*args, None, A16 * 64, None, 0, 10, 1, 128, 128, None) == g.GDN2_OK
+    bad = list(args)
+    bad[3] = A16 + 4
+    assert lib.gdn2_chunk_fwd_logits(*bad, None, A16 * 64, None, 1, 10, 1, 128, 128, None) == g.GDN2_ERR_INVALID_ARG
+    assert lib.gdn2_chunk_fwd_logits(*args, None, A16 * 2, None, 1, 10, 1, 128, 128, None) == g.GDN2_ERR_INVALID_ARG
+    assert b"overlaps" in lib.gdn2_last_error()
+
+
+def test_output_gate_host_checks(lib):
+    c = ctypes.c_float
+    assert lib.gdn2_output_gate(A16, A16 * 2, A16 * 3, c(1e-6), A16 * 64, 1, 4, 2, 96, BF16, None) == g.GDN2_ERR_UNSUPPORTED
+    assert lib.gdn2_output_gate(A16, A16 * 2, A16 * 3, c(-1.0), A16 * 64, 1, 4, 2, 128, BF16, None) == g.GDN2_ERR_INVALID_ARG
+    assert lib.gdn2_output_gate(A16, A16 * 2, A16 * 3, c(1e-6), A16 * 64, 0, 4, 2, 128, BF16, None) == g.GDN2_OK
+    assert lib.gdn2_output_gate(A16 + 2, A16 * 2, A16 * 3, c(1e-6), A16 * 64, 1, 4, 2, 128, BF16, None) == g.GDN2_ERR_INVALID_ARG
+    # y partially overlapping o is refused; exact aliasing would be allowed
+    assert lib.gdn2_output_gate(A16, A16 * 2, A16 * 3, c(1e-6), A16 + 16, 1, 4, 2, 128, BF16, None) == g.GDN2_ERR_INVALID_ARG
+    assert b"overlaps" in lib.gdn2_last_error()

@@ -102,3 +102,24 @@ def test_backward_entry(capsys):
     # 4,864 B per token-head (q,k,v,dO bf16 + alpha,b,w fp32 in; dq,dk,dv bf16 + dalpha,db,dw fp32 out)
     assert bench.backward_bytes(1, 1, 1, 128, 128) == 4864 + 128 * 128 * 4
     assert bw["roofline"]["achieved"] == pytest.approx(bench.backward_bytes(4, 4096, 16, 128, 128) / 2.0e-3 / 1e9)
+
+
+def test_logits_entry(capsys):
+    args = argparse.Namespace(steps=20, warmup=5, no_cpu_baseline=True, cpu_budget=1.0)
+    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), float("nan"), float("nan"), 0.4)
+    d = json.loads(capsys.readouterr().out.strip())
+    lg = d["prefill_logits"]
+    # six BF16 logit tensors in, BF16 o out: 1,792 B per token-head at d = 128
+    assert bench.logits_bytes(1, 1, 1, 128, 128) == 1792 + 128 * 128 * 4
+    assert lg["roofline"]["achieved"] == pytest.approx(bench.logits_bytes(4, 4096, 16, 128, 128) / 0.4e-3 / 1e9)
+    assert d["backward"]["value"] is None
+
+
+def test_output_gate_entry(capsys):
+    args = argparse.Namespace(steps=20, warmup=5, no_cpu_baseline=True, cpu_budget=1.0)
+    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), float("nan"), float("nan"), float("nan"), 0.04)
+    d = json.loads(capsys.readouterr().out.strip())
+    og = d["output_gate"]
+    # o and g read, y written, BF16: 768 B per token-head at d_v = 128
+    assert bench.output_gate_bytes(1, 1, 1, 128) == 768 + 512
+    assert og["roofline"]["achieved"] == pytest.approx(bench.output_gate_bytes(4, 4096, 16, 128) / 0.04e-3 / 1e9)
