@@ -58,12 +58,13 @@
 // TF32 copy that the next chunk's X product reads.
 //
 // Logits variant (kLogits): every input arrives as BF16 pre-activation logits.
-// alpha and b land as BF16 tiles in the first half of AT and BT; before the
-// decay products, the key side turns them into the FP32 gates (alpha =
-// exp(-softplus(x)) = 1 / (1 + e^x), b = sigmoid(x)); pass A applies SiLU and the
-// L2 norm over each token's 128 channels (a warp holds whole token rows) in FP32
-// as it reads the raw q, k logits.  The state side forms
-// z = sigmoid(x_w) silu(x_v) from BF16 loads.  The rest of the kernel is unchanged.
+// alpha and b land as BF16 tiles in the first half of AT and BT; the decay pass
+// reads every raw alpha and b value before it writes any tile, forms the FP32
+// gates (alpha = exp(-softplus(x)) = 1 / (1 + e^x), b = sigmoid(x)) in
+// registers, and applies SiLU and the L2 norm over each token's 128 channels (a
+// warp holds whole token rows) to q and k in FP32 as it reads them.  The state
+// side forms z = sigmoid(x_w) silu(x_v) from BF16 loads.  The rest of the kernel
+// is unchanged.
 #include <cudaTypedefs.h>
 #include <stdio.h>
 
@@ -226,9 +227,19 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
     const int cg = ktid & 31, tg = ktid >> 5, lane = ktid & 31;
     const int tl0 = 8 * tg;
     float p[8][4];
+    uint2 braw[kLogits ? 8 : 1];     // logits: b's raw BF16 values, read before any tile is rewritten
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-        const float4 a = *reinterpret_cast<const float4 *>(c.sm + OFF_AT + (cg >> 3) * TILE + swz128(tl0 + u, (cg & 7) * 16));
+        float4 a;
+        if constexpr (kLogits) {     // alpha = exp(-softplus(x)) = 1 / (1 + e^x) from the BF16 logit
+            const uint32_t o16 = (cg >> 4) * TILE + swz128(tl0 + u, (cg & 15) * 8);
+            const uint2 ar = *reinterpret_cast<const uint2 *>(c.sm + OFF_AT + o16);
+            braw[u] = *reinterpret_cast<const uint2 *>(c.sm + OFF_BT + o16);
+            a = make_float4(sigmoid_fast(-bf_lo(ar.x)), sigmoid_fast(-bf_hi(ar.x)), sigmoid_fast(-bf_lo(ar.y)),
+                            sigmoid_fast(-bf_hi(ar.y)));
+        } else {
+            a = *reinterpret_cast<const float4 *>(c.sm + OFF_AT + (cg >> 3) * TILE + swz128(tl0 + u, (cg & 7) * 16));
+        }
         const bool v = tl0 + u < navail;
         p[u][0] = v ? fmaxf(a.x, kGammaMin) : 1.f;
         p[u][1] = v ? fmaxf(a.y, kGammaMin) : 1.f;
@@ -283,7 +294,12 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
         const bool valid = t < n;
         const uint2 kr = valid ? *reinterpret_cast<const uint2 *>(c.sm + OFF_KT + o16) : make_uint2(0u, 0u);
         const uint2 qr = valid ? *reinterpret_cast<const uint2 *>(c.sm + OFF_QT + o16) : make_uint2(0u, 0u);
-        const float4 b4 = *reinterpret_cast<const float4 *>(c.sm + OFF_BT + o32);
+        float4 b4;
+        if constexpr (kLogits)
+            b4 = make_float4(sigmoid_fast(bf_lo(braw[u].x)), sigmoid_fast(bf_hi(braw[u].x)),
+                             sigmoid_fast(bf_lo(braw[u].y)), sigmoid_fast(bf_hi(braw[u].y)));
+        else
+            b4 = *reinterpret_cast<const float4 *>(c.sm + OFF_BT + o32);
         float kk[4] = {bf_lo(kr.x), bf_hi(kr.x), bf_lo(kr.y), bf_hi(kr.y)};
         float qq[4] = {bf_lo(qr.x), bf_hi(qr.x), bf_lo(qr.y), bf_hi(qr.y)};
         if constexpr (kLogits) {     // q, k = silu(x) / ||silu(x)||, in FP32 from the raw logits;
@@ -332,36 +348,6 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
 }
 
 
-// Logits variant, before pass A (same thread layout: channels 4 cg .. 4 cg + 3 of
-// tokens 8 tg .. 8 tg + 7, so a warp holds whole token rows).  The input
-// preparation of "Token processing and parallel training" and "Independent
-// decisions on two axes", in shared memory:
-//   alpha = exp(-softplus(x)) = 1 / (1 + e^x),  b = sigmoid(x)   BF16 -> the FP32 tiles
-// (pass A applies SiLU and the L2 norm to q and k as it reads them).  Every raw
-// alpha / b value is read before the group barrier, since the FP32 tiles overlay
-// the BF16 ones.
-__device__ __forceinline__ void key_logits(const Ctx &c, int ktid) {
-    const int cg = ktid & 31, tg = ktid >> 5;
-    const int tl0 = 8 * tg;
-    uint2 ra[8], rb[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        const uint32_t o16 = (cg >> 4) * TILE + swz128(tl0 + u, (cg & 15) * 8);
-        ra[u] = *reinterpret_cast<const uint2 *>(c.sm + OFF_AT + o16);
-        rb[u] = *reinterpret_cast<const uint2 *>(c.sm + OFF_BT + o16);
-    }
-    named_bar(kBarK, kGroup);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        const uint32_t o32 = (cg >> 3) * TILE + swz128(tl0 + u, (cg & 7) * 16);
-        const float a4[4] = {bf_lo(ra[u].x), bf_hi(ra[u].x), bf_lo(ra[u].y), bf_hi(ra[u].y)};
-        const float b4[4] = {bf_lo(rb[u].x), bf_hi(rb[u].x), bf_lo(rb[u].y), bf_hi(rb[u].y)};
-        *reinterpret_cast<float4 *>(c.sm + OFF_AT + o32) =
-            make_float4(sigmoid_fast(-a4[0]), sigmoid_fast(-a4[1]), sigmoid_fast(-a4[2]), sigmoid_fast(-a4[3]));
-        *reinterpret_cast<float4 *>(c.sm + OFF_BT + o32) =
-            make_float4(sigmoid_fast(b4[0]), sigmoid_fast(b4[1]), sigmoid_fast(b4[2]), sigmoid_fast(b4[3]));
-    }
-}
 
 // Key side, pass B (thread per token t, channel half ch): the rows of Etil
 // (lanes 0-63) or Qtil (lanes 64-127) of 64 channels into the TMEM operand.
@@ -398,7 +384,7 @@ __device__ __forceinline__ void key_kt(const Ctx &c, uint32_t tmem, int warp, in
 
 // The chunk's alpha and b tiles (or q and k) by TMA.
 // FP32 gates: four 32-channel blocks each.  Logits: two 64-channel BF16 blocks each,
-// at the start of the same regions (key_logits turns them into the FP32 tiles).
+// at the start of the same regions (the decay pass reads them as logits).
 template <bool kLogits>
 __device__ __forceinline__ void load_ab(const Ctx &c, const Maps &m, int h, int t0) {
     const uint32_t fb = c.bar(B_FULL_AB);
@@ -674,7 +660,6 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                     tma_prefetch_3d(&maps.v, col0, h, tn);
                 }
             }
-            if constexpr (kLogits) key_logits(c, ktid);
             const int n = key_decay<kLogits>(c, ktid, t0, navail, te, r, el);
             const bool last = t0 + n >= te;
             fence_proxy_async_smem();
