@@ -179,6 +179,8 @@ gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v, const fl
     if (dS0 && (st = check_ptr(dS0, "dS0")) != GDN2_OK) return st;
     if (dST && (st = check_ptr(dST, "dST")) != GDN2_OK) return st;
     if (B == 0 || H == 0) return GDN2_OK;
+    if ((long long)B * H > 65535)       // (sequence, head) pairs index the grid's second dimension
+        return fail(GDN2_ERR_UNSUPPORTED, "%s", "gdn2_chunk_bwd: B * H above 65535");
     if (dS0 && overlaps(dS0, state_bytes, dST, state_bytes))
         return fail(GDN2_ERR_INVALID_ARG, "%s", "dS0 overlaps dST");
     if (T == 0) {          // no tokens: dS0 = dST

@@ -188,7 +188,8 @@ gdn2_status gdn2_output_gate(const void *o, const void *g, const float *weight, 
  * The forward pass is recomputed inside (the states at chunk boundaries go to
  * the workspace), so nothing from gdn2_chunk_fwd needs to be kept.  alpha is
  * differentiated at max(alpha, 2^-64), the value the prefill computes with;
- * dalpha divides by that value.  Supported: d_k, d_v in {64, 128}, BF16 or FP32.
+ * dalpha divides by that value.  Supported: d_k, d_v in {64, 128}, BF16 or FP32,
+ * B * H <= 65535 (GDN2_ERR_UNSUPPORTED beyond).
  * T = 0, B = 0 or H = 0: nothing is read; dS0 = dST (zero if dST is NULL).
  * No output may overlap an input, another output or the workspace.
  */

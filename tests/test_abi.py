@@ -164,6 +164,7 @@ def test_backward_host_checks(lib):
     assert _bwd(lib, dt=7) == g.GDN2_ERR_UNSUPPORTED
     assert _bwd(lib, T=-1) == g.GDN2_ERR_INVALID_ARG
     assert _bwd(lib, B=0) == g.GDN2_OK and _bwd(lib, H=0) == g.GDN2_OK
+    assert _bwd(lib, B=4096, H=16) == g.GDN2_ERR_UNSUPPORTED        # B * H beyond the grid's 65535
     need = lib.gdn2_chunk_bwd_workspace_size(1, 10, 1, 128, 128)
     # chunk states and gradients, T and P, U and dR per token, and the key block
     # (five [64][132] tiles, two [64][132], one [128][132], 128 decay factors)
