@@ -51,6 +51,7 @@ namespace {
 constexpr int kC = 64;            // chunk length
 constexpr int kCS = 32;           // value columns per CTA of the state kernel
 constexpr int kThreads = 256;
+constexpr int kThreadsB = 512;   // the gradient gathers (grad_b): 16 warps, to hide their load latency
 constexpr int LDT = kC + 1;       // row stride of 64 x 64 tiles in shared memory
 constexpr float kAlphaMin = 5.42101086e-20f;   // 2^-64; log2f of the clamped decay is accurate to an ulp
 
@@ -75,9 +76,9 @@ __device__ __forceinline__ float gdiff(float ht, float lt, float hs, float ls) {
 // entry (0 on padding rows); on exit hi + lo is the compensated prefix sum from the
 // chunk start.  Each (channel, half of the chunk) runs over 32 tokens, then the
 // second half adds the first half's total.  Ends with __syncthreads().
-template <int NCH>
+template <int NCH, int NT = kThreads>
 __device__ void comp_cumsum(float *hi, float *lo, int ld) {
-    for (int idx = threadIdx.x; idx < 2 * NCH; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < 2 * NCH; idx += NT) {
         const int i = idx % NCH, half = idx / NCH;
         float run = 0.f, comp = 0.f, err;
         for (int t = half * 32; t < half * 32 + 32; ++t) {
@@ -88,7 +89,7 @@ __device__ void comp_cumsum(float *hi, float *lo, int ld) {
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < 32 * NCH; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < 32 * NCH; idx += NT) {
         const int t = 32 + idx / NCH, i = idx % NCH;
         float err;
         const float h = two_sum(hi[31 * ld + i], hi[t * ld + i], err);
@@ -108,11 +109,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// rows x cols floats (cols a multiple of 4; both row strides multiples of 4 floats).
+// rows x cols floats (cols a multiple of 4; both row strides multiples of 4 floats), by NT threads.
+template <int NT = kThreads>
 __device__ __forceinline__ void copy_tile_async(float *dst, int dst_ld, const float *src, size_t src_ld, int rows,
                                                 int cols) {
     const int per = cols >> 2;
-    for (int idx = threadIdx.x; idx < rows * per; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < rows * per; idx += NT) {
         const int r = idx / per, c4 = (idx - r * per) << 2;
         cp_async16(dst + r * dst_ld + c4, src + r * src_ld + c4);
     }
@@ -787,7 +789,7 @@ struct GradBSmem {
 };
 
 template <typename TIn, int DK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsB, 1)
 bwd_gradb_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const float *__restrict__ alpha,
                  const float *__restrict__ bgate, Ws ws, TIn *dq, TIn *dk, float *dalpha, float *db, int T, int H) {
     constexpr int LP = GradBSmem::LP, LB = GradBSmem::LB, LE = GradBSmem::LE;
@@ -804,23 +806,23 @@ bwd_gradb_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const flo
     const size_t tok0 = (size_t)seq * T + c0;
     const size_t chunk = (size_t)unit * nch + c;
 
-    copy_tile_async(dP, LP, ws.DPA + chunk * 2 * kC * kC, kC, kC, kC);
-    copy_tile_async(dA, LP, ws.DPA + chunk * 2 * kC * kC + kC * kC, kC, kC, kC);
+    copy_tile_async<kThreadsB>(dP, LP, ws.DPA + chunk * 2 * kC * kC, kC, kC, kC);
+    copy_tile_async<kThreadsB>(dA, LP, ws.DPA + chunk * 2 * kC * kC + kC * kC, kC, kC, kC);
     cp_async_commit();
     const float *xs = ws.XS + chunk * 3 * kC * DK;
     for (int ib = 0; ib < DK; ib += 32) {
         __syncthreads();
-        copy_tile_async(X1, LB, xs + ib, DK, kC, 32);
-        copy_tile_async(X2, LB, xs + kC * DK + ib, DK, kC, 32);
-        copy_tile_async(Y, LB, xs + 2 * kC * DK + ib, DK, kC, 32);
-        copy_tile_async(rs, 32, ws.RS + chunk * DK + ib, 32, 1, 32);
+        copy_tile_async<kThreadsB>(X1, LB, xs + ib, DK, kC, 32);
+        copy_tile_async<kThreadsB>(X2, LB, xs + kC * DK + ib, DK, kC, 32);
+        copy_tile_async<kThreadsB>(Y, LB, xs + 2 * kC * DK + ib, DK, kC, 32);
+        copy_tile_async<kThreadsB>(rs, 32, ws.RS + chunk * DK + ib, 32, 1, 32);
         cp_async_commit();
         {   // this block's key side: all loads first, then the transforms
-            constexpr int E = kC * 32 / kThreads;
+            constexpr int E = kC * 32 / kThreadsB;
             float ra[E], rk[E], rq[E], rb[E];
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
+                const int idx = tid + e * kThreadsB, t = idx >> 5, i = idx & 31;
                 ra[e] = 1.f; rk[e] = rq[e] = rb[e] = 0.f;
                 if (t < n) {
                     const size_t off = ((tok0 + t) * H + h) * DK + ib + i;
@@ -832,7 +834,7 @@ bwd_gradb_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const flo
             }
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
+                const int idx = tid + e * kThreadsB, t = idx >> 5, i = idx & 31;
                 cg[t * LB + i] = log2f(fmaxf(ra[e], kAlphaMin));
                 ck[t * LB + i] = rk[e];
                 cq[t * LB + i] = rq[e];
@@ -840,22 +842,22 @@ bwd_gradb_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const flo
             }
         }
         __syncthreads();
-        comp_cumsum<32>(cg, cl, LB);
+        comp_cumsum<32, kThreadsB>(cg, cl, LB);
         // scaled tiles (both factors of every split decay are at most 1)
-        for (int idx = tid; idx < 48 * 32; idx += kThreads) {
+        for (int idx = tid; idx < 48 * 32; idx += kThreadsB) {
             const int t = 16 + (idx >> 5), i = idx & 31, r = t & ~15;
             const float f = ex2(gdiff(cg[t * LB + i], cl[t * LB + i], cg[r * LB + i], cl[r * LB + i]));
             Er[(t - 16) * LE + i] = ce[t * LB + i] * f;
             Qr[(t - 16) * LE + i] = cq[t * LB + i] * f;
         }
-        for (int idx = tid; idx < 96 * 32; idx += kThreads) {
+        for (int idx = tid; idx < 96 * 32; idx += kThreadsB) {
             const int row = idx >> 5, i = idx & 31;
             const int tau = row < 16 ? 1 : (row < 48 ? 2 : 3), s2 = row - kr_offset(tau), r = 16 * tau;
             const float f = ex2(gdiff(cg[r * LB + i], cl[r * LB + i], cg[s2 * LB + i], cl[s2 * LB + i]));
             F[row * LE + i] = f;
             Kr[row * LE + i] = ck[s2 * LB + i] * f;
         }
-        for (int idx = tid; idx < 16 * 32; idx += kThreads) {     // no earlier block for rows 0-15,
+        for (int idx = tid; idx < 16 * 32; idx += kThreadsB) {     // no earlier block for rows 0-15,
             const int t = idx >> 5, i = idx & 31;                 // no later block for keys 48-63
             OQ[t * LB + i] = 0.f;
             OE[t * LB + i] = 0.f;
@@ -879,8 +881,11 @@ bwd_gradb_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const flo
                             ex2(gdiff(cg[t * LB + ic], cl[t * LB + ic], cg[r * LB + ic], cl[r * LB + ic]));
                     }
             }
-            {   // keys of block sigma = warp / 2, channels 16 (warp & 1) ..: every later block tau
-                const int sigma = warp >> 1, n0 = 16 * (warp & 1);
+        }
+        if (warp >= 6 && warp < 12) {
+            const int cw = warp - 6;
+            {   // keys of block sigma = cw / 2, channels 16 (cw & 1) ..: every later block tau
+                const int sigma = cw >> 1, n0 = 16 * (cw & 1);
                 float acc[2][4];
 #pragma unroll
                 for (int b = 0; b < 2; ++b)
@@ -910,10 +915,10 @@ bwd_gradb_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const flo
             }
         }
         __syncthreads();
-        float dlg[kC * 32 / kThreads];
+        float dlg[kC * 32 / kThreadsB];
 #pragma unroll
-        for (int e = 0; e < kC * 32 / kThreads; ++e) {
-            const int idx = tid + e * kThreads, t = idx >> 5, i = idx & 31;
+        for (int e = 0; e < kC * 32 / kThreadsB; ++e) {
+            const int idx = tid + e * kThreadsB, t = idx >> 5, i = idx & 31;
             const int r = t & ~15;
             const float gt = cg[t * LB + i], lt = cl[t * LB + i];
             const float gnh = cg[(kC - 1) * LB + i], gnl = cl[(kC - 1) * LB + i];
@@ -950,29 +955,30 @@ bwd_gradb_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const flo
         }
         __syncthreads();                    // X2 is free now: it takes dlog gamma
 #pragma unroll
-        for (int e = 0; e < kC * 32 / kThreads; ++e) {
-            const int idx = tid + e * kThreads;
+        for (int e = 0; e < kC * 32 / kThreadsB; ++e) {
+            const int idx = tid + e * kThreadsB;
             X2[(idx >> 5) * LB + (idx & 31)] = dlg[e];
         }
         __syncthreads();
-        {   // dalpha = reverse cumulative sum of dlog gamma / alpha: (channel, 8-token segment) per thread
+        {   // dalpha = reverse cumulative sum of dlog gamma / alpha: (channel, 4-token segment) per thread
+            constexpr int SEG = kC * 32 / kThreadsB, NSEG = kC / SEG;
             const int i = tid & 31, seg = tid >> 5;
-            float ra[8];
+            float ra[SEG];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int t = seg * 8 + u;
+            for (int u = 0; u < SEG; ++u) {
+                const int t = seg * SEG + u;
                 ra[u] = t < n ? __ldg(alpha + ((tok0 + t) * H + h) * DK + ib + i) : 1.f;
             }
             float tot = 0.f;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) tot += X2[(seg * 8 + u) * LB + i];
+            for (int u = 0; u < SEG; ++u) tot += X2[(seg * SEG + u) * LB + i];
             X1[seg * LB + i] = tot;             // X1 is free: segment totals
             __syncthreads();
             float run = 0.f;
-            for (int s2 = seg + 1; s2 < 8; ++s2) run += X1[s2 * LB + i];
+            for (int s2 = seg + 1; s2 < NSEG; ++s2) run += X1[s2 * LB + i];
 #pragma unroll
-            for (int u = 7; u >= 0; --u) {
-                const int t = seg * 8 + u;
+            for (int u = SEG - 1; u >= 0; --u) {
+                const int t = seg * SEG + u;
                 run += X2[t * LB + i];
                 if (t < n) dalpha[((tok0 + t) * H + h) * DK + ib + i] = run / fmaxf(ra[u], kAlphaMin);
             }
@@ -1014,7 +1020,7 @@ cudaError_t launch_bwd_typed(const void *q_, const void *k_, const void *v_, con
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     kga<<<grid_c, kThreads, GradASmem<DV>::bytes, stream>>>(v, w, dO, ws, static_cast<TIn *>(dv), dw, T, H);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    kgb<<<grid_c, kThreads, GradBSmem::bytes, stream>>>(q, k, alpha, b, ws, static_cast<TIn *>(dq),
+    kgb<<<grid_c, kThreadsB, GradBSmem::bytes, stream>>>(q, k, alpha, b, ws, static_cast<TIn *>(dq),
                                                          static_cast<TIn *>(dk), dalpha, db, T, H);
     return cudaGetLastError();
 }
