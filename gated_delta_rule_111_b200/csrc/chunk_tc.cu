@@ -102,9 +102,10 @@ constexpr long long kDrainLimit = 4000000000ll; // ~2 s: end-of-kernel waits for
 //   UH  R_hi, later U_hi, as [j][t] (2 token blocks);  UL  R_lo, later U_lo
 //   AS  A, then T in place (FP32 [64][68]);  XS block products (FP32 [32][36])
 constexpr uint32_t TILE = 8192;
-constexpr uint32_t OFF_AT = 0;
-constexpr uint32_t OFF_BT = OFF_AT + 4 * TILE;
-constexpr uint32_t OFF_QT = OFF_BT + 4 * TILE;
+constexpr uint32_t OFF_EQS = 0;     // Etil / b and Qtil / alpha blocks interleaved: E0 Q0 E1 Q1 E2 Q2 E3 Q3
+__host__ __device__ constexpr uint32_t OFF_E(int blk) { return OFF_EQS + 2u * blk * TILE; }
+__host__ __device__ constexpr uint32_t OFF_Q(int blk) { return OFF_EQS + (2u * blk + 1u) * TILE; }
+constexpr uint32_t OFF_QT = OFF_EQS + 8 * TILE;
 constexpr uint32_t OFF_KT = OFF_QT + 2 * TILE;
 constexpr uint32_t OFF_KG = OFF_KT + 2 * TILE;
 constexpr uint32_t OFF_SC = OFF_KG + 4 * TILE;
@@ -143,7 +144,7 @@ constexpr uint32_t TM_COLS = 512;
 enum {
     B_KPREP = 0, B_G_FULL, B_S_READY, B_X_FULL, B_R_READY, B_TP_READY0, B_TP_READY1, B_U_FULL, B_U_READY,
     B_D_FULL, B_O_FULL, B_KH_READY, B_KH_FREE, B_TP_FREE0, B_TP_FREE1, B_RR0, B_RR1, B_RR2, B_RR3,
-    B_FULL_AB, B_FULL_QK, B_DRAIN, NBARS
+    B_FULL_AB, B_FULL_QK, B_DRAIN, B_GRAM_GO, NBARS
 };
 static_assert(NBARS * 8 <= 256, "barrier area");
 
@@ -232,13 +233,13 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
     for (int u = 0; u < 8; ++u) {
         float4 a;
         if constexpr (kLogits) {     // alpha = exp(-softplus(x)) = 1 / (1 + e^x) from the BF16 logit
-            const uint32_t o16 = (cg >> 4) * TILE + swz128(tl0 + u, (cg & 15) * 8);
-            const uint2 ar = *reinterpret_cast<const uint2 *>(c.sm + OFF_AT + o16);
-            braw[u] = *reinterpret_cast<const uint2 *>(c.sm + OFF_BT + o16);
+            const uint32_t s16 = swz128(tl0 + u, (cg & 15) * 8);
+            const uint2 ar = *reinterpret_cast<const uint2 *>(c.sm + OFF_Q(cg >> 4) + s16);
+            braw[u] = *reinterpret_cast<const uint2 *>(c.sm + OFF_E(cg >> 4) + s16);
             a = make_float4(sigmoid_fast(-bf_lo(ar.x)), sigmoid_fast(-bf_hi(ar.x)), sigmoid_fast(-bf_lo(ar.y)),
                             sigmoid_fast(-bf_hi(ar.y)));
         } else {
-            a = *reinterpret_cast<const float4 *>(c.sm + OFF_AT + (cg >> 3) * TILE + swz128(tl0 + u, (cg & 7) * 16));
+            a = *reinterpret_cast<const float4 *>(c.sm + OFF_Q(cg >> 3) + swz128(tl0 + u, (cg & 7) * 16));
         }
         const bool v = tl0 + u < navail;
         p[u][0] = v ? fmaxf(a.x, kGammaMin) : 1.f;
@@ -289,7 +290,7 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         const int t = tl0 + u;
-        const uint32_t o32 = (cg >> 3) * TILE + swz128(t, (cg & 7) * 16);
+        const uint32_t s32 = swz128(t, (cg & 7) * 16);
         const uint32_t o16 = (cg >> 4) * TILE + swz128(t, (cg & 15) * 8);
         const bool valid = t < n;
         const uint2 kr = valid ? *reinterpret_cast<const uint2 *>(c.sm + OFF_KT + o16) : make_uint2(0u, 0u);
@@ -299,7 +300,7 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
             b4 = make_float4(sigmoid_fast(bf_lo(braw[u].x)), sigmoid_fast(bf_hi(braw[u].x)),
                              sigmoid_fast(bf_lo(braw[u].y)), sigmoid_fast(bf_hi(braw[u].y)));
         else
-            b4 = *reinterpret_cast<const float4 *>(c.sm + OFF_BT + o32);
+            b4 = *reinterpret_cast<const float4 *>(c.sm + OFF_E(cg >> 3) + s32);
         float kk[4] = {bf_lo(kr.x), bf_hi(kr.x), bf_lo(kr.y), bf_hi(kr.y)};
         float qq[4] = {bf_lo(qr.x), bf_hi(qr.x), bf_lo(qr.y), bf_hi(qr.y)};
         if constexpr (kLogits) {     // q, k = silu(x) / ||silu(x)||, in FP32 from the raw logits;
@@ -332,9 +333,9 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
             q4[e] = to_tf32(qq[e] * g);
             k4[e] = to_tf32(__fdividef(kk[e], g));
         }
-        *reinterpret_cast<float4 *>(c.sm + OFF_BT + o32) = make_float4(e4[0], e4[1], e4[2], e4[3]);
-        *reinterpret_cast<float4 *>(c.sm + OFF_AT + o32) = make_float4(q4[0], q4[1], q4[2], q4[3]);
-        *reinterpret_cast<float4 *>(c.sm + OFF_KG + o32) = make_float4(k4[0], k4[1], k4[2], k4[3]);
+        *reinterpret_cast<float4 *>(c.sm + OFF_E(cg >> 3) + s32) = make_float4(e4[0], e4[1], e4[2], e4[3]);
+        *reinterpret_cast<float4 *>(c.sm + OFF_Q(cg >> 3) + s32) = make_float4(q4[0], q4[1], q4[2], q4[3]);
+        *reinterpret_cast<float4 *>(c.sm + OFF_KG + (cg >> 3) * TILE + s32) = make_float4(k4[0], k4[1], k4[2], k4[3]);
     }
     if (tg == 7)
         *reinterpret_cast<float4 *>(r.gn + 4 * cg) =
@@ -354,15 +355,15 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
 __device__ __forceinline__ void key_rows(const Ctx &c, uint32_t tmem, int warp, int lane) {
     const int lq = warp & 3, ch = (warp - 1) >> 2;
     const int t = 32 * (lq & 1) + lane;
-    const uint32_t src = lq < 2 ? OFF_BT : OFF_AT;
     const uint32_t tl = tmem + TM_EQ + ((uint32_t)(32 * lq) << 16);
 #pragma unroll
     for (int blk = 0; blk < 2; ++blk) {
         const int a = 2 * ch + blk;
+        const uint32_t src = lq < 2 ? OFF_E(a) : OFF_Q(a);
         float x[32];
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
-            const float4 g4 = *reinterpret_cast<const float4 *>(c.sm + src + a * TILE + swz128(t, 16 * m));
+            const float4 g4 = *reinterpret_cast<const float4 *>(c.sm + src + swz128(t, 16 * m));
             x[4 * m] = g4.x; x[4 * m + 1] = g4.y; x[4 * m + 2] = g4.z; x[4 * m + 3] = g4.w;
         }
         tmem_st32_nowait(tl + 32 * a, x);
@@ -391,8 +392,8 @@ __device__ __forceinline__ void load_ab(const Ctx &c, const Maps &m, int h, int 
     mbar_expect_tx(fb, kLogits ? TX_AB_LOGITS : TX_AB);
     for (int a = 0; a < (kLogits ? 2 : 4); ++a) {
         const int x = kLogits ? 64 * a : 32 * a;
-        tma_load_3d(c.sa + OFF_AT + a * TILE, &m.alpha, x, h, t0, fb);
-        tma_load_3d(c.sa + OFF_BT + a * TILE, &m.b, x, h, t0, fb);
+        tma_load_3d(c.sa + OFF_Q(a), &m.alpha, x, h, t0, fb);
+        tma_load_3d(c.sa + OFF_E(a), &m.b, x, h, t0, fb);
     }
 }
 __device__ __forceinline__ void load_qk(const Ctx &c, const Maps &m, int h, int t0) {
@@ -514,6 +515,8 @@ __device__ __forceinline__ uint32_t kstep(int kk) { return ((kk >> 2) * TILE + (
 __device__ __noinline__ void issuer_role(const Ctx &c, uint32_t tmem) {
     // B descriptors as (low, high) halves; the K-step offset is added inside each MMA's asm.
     const uint64_t dSC = sdesc_sw128(c.sa + OFF_SC, 16, 1024), dKG = sdesc_sw128(c.sa + OFF_KG, 16, 1024);
+    // [Etil; Qtil] in shared memory: rows 0-63 from an E block, rows 64-127 from the Q block after it
+    const uint32_t eq = (uint32_t)sdesc_sw128(c.sa + OFF_EQS, 16, 1024);
     const uint64_t dUH = sdesc_sw128(c.sa + OFF_UH, 16, 1024), dUL = sdesc_sw128(c.sa + OFF_UL, 16, 1024);
     const uint32_t hi = (uint32_t)(dSC >> 32);      // identical for every tile (layout, SBO, version)
     const uint32_t sc = (uint32_t)dSC, kg = (uint32_t)dKG, uh = (uint32_t)dUH, ul = (uint32_t)dUL;
@@ -549,21 +552,23 @@ __device__ __noinline__ void issuer_role(const Ctx &c, uint32_t tmem) {
             }
             mma_commit(c.bar(B_U_FULL));
             ++cu;
-        } else if (cx < cg && mbar_test(c.bar(B_S_READY), cx & 1)) {
+        } else if (cx < cg && mbar_test(c.bar(B_KPREP), cx & 1) && mbar_test(c.bar(B_S_READY), cx & 1)) {
             // [Etil; Qtil] S
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 16; ++kk) mma_tf32_ts_off(tmem + TM_X, tmem + TM_EQ + 8 * kk, sc, hi, kstep(kk), id, kk > 0);
             mma_commit(c.bar(B_X_FULL));
             ++cx;
-        } else if (cg <= lastc && mbar_test(c.bar(B_KPREP), cg & 1) &&
+        } else if (cg <= lastc && mbar_test(c.bar(B_GRAM_GO), cg & 1) &&
                    (cg < 2 || mbar_test(c.bar((cg & 1) ? B_TP_FREE1 : B_TP_FREE0), ((cg - 2) >> 1) & 1))) {
             // Gram [Etil; Qtil] Ktil^T into the chunk's [T; P] buffer
             tc_fence_after();
             if (rec(c, cg).last) lastc = cg;
             const uint32_t tp = tmem + TM_TP + 64 * (cg & 1);
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk) mma_tf32_ts_off(tp, tmem + TM_EQ + 8 * kk, kg, hi, kstep(kk), id, kk > 0);
+            for (int kk = 0; kk < 16; ++kk)    // A from the shared-memory tiles, before they reach TMEM
+                mma_tf32_ss_off(tp, eq, (uint32_t)(((kk >> 2) * 2 * TILE + (kk & 3) * 32) >> 4), kg, kstep(kk), hi,
+                                id, kk > 0);
             mma_commit(c.bar(B_G_FULL));
             ++cg;
         } else {
@@ -666,6 +671,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
             named_bar(kBarK, kGroup);
             if (el) {
                 mbar_arrive(c.bar(B_RR0 + (ck & 3)));
+                mbar_arrive(c.bar(B_GRAM_GO));         // the Gram reads [Etil; Qtil] from shared memory
                 if (!last) {
                     load_qk(c, maps, h, t0 + n);       // q, k consumed: the next chunk's
                     pend_qk = ck + 1;
@@ -678,15 +684,13 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarK, kGroup);
-            if (el) {
-                mbar_arrive(c.bar(B_KPREP));
-                if (!last) {
-                    load_ab<kLogits>(c, maps, h, t0 + n);       // alpha, b consumed: the next chunk's
-                    pend_ab = ck + 1;
-                }
-            }
+            if (el) mbar_arrive(c.bar(B_KPREP));
             // Gram epilogue: A (rows 0-63, strictly lower) -> AS; P (rows 64-127) masked in place.
             if (!group_wait(c, B_G_FULL, ph, el, kBarK)) break;
+            if (el && !last) {                 // the Gram and the row pass have read alpha -> Qtil, b -> Etil
+                load_ab<kLogits>(c, maps, h, t0 + n);
+                pend_ab = ck + 1;
+            }
             tc_fence_after();
             {
                 const uint32_t tp = tlane + TM_TP + 64 * ph + 32 * ch;

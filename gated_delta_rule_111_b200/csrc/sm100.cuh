@@ -282,6 +282,22 @@ __device__ __forceinline__ void mma_tf32_ts_off(uint32_t d_tmem, uint32_t a_tmem
         "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(b_off), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A * B with both operands in shared memory, each descriptor given as
+// its two 32-bit halves plus a start-address offset (16-byte units) added inside
+// the asm statement.
+__device__ __forceinline__ void mma_tf32_ss_off(uint32_t d_tmem, uint32_t a_lo, uint32_t a_off, uint32_t b_lo,
+                                                uint32_t b_off, uint32_t hi, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b32 alo, blo;\n\t.reg .b64 ad, bd;\n\t"
+        "add.u32 alo, %1, %2;\n\t"
+        "add.u32 blo, %3, %4;\n\t"
+        "mov.b64 ad, {alo, %5};\n\t"
+        "mov.b64 bd, {blo, %5};\n\t"
+        "setp.ne.b32 p, %7, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], ad, bd, %6, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_lo), "r"(a_off), "r"(b_lo), "r"(b_off), "r"(hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
