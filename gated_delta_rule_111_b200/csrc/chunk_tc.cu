@@ -38,19 +38,20 @@
 //
 // Organisation: one CTA per (sequence, head, 64-column half of d_v), 17 warps
 // in three roles that run concurrently and hand work over through mbarriers:
-//   warp 0      MMA issuer: one thread issues every tcgen05 instruction, in
-//               whichever order their inputs become ready
+//   warp 0      MMA issuer: the warp decides, one elected lane issues every
+//               tcgen05 instruction, in whichever order their inputs become ready
 //   warps 1-8   key side, one chunk ahead of the state side.  alpha, b, q, k
 //               arrive by TMA in 128-byte-swizzled tiles; a thread per key
 //               channel forms the decay products and the chunk length and
-//               turns the tiles in place into Qtil and Etil, writes Ktil (the
-//               Gram's B operand) and Ktil^T into Tensor Memory (the state
-//               update's A operand); a thread per token then moves the rows
-//               of [Etil; Qtil] into Tensor Memory (the A operand of the Gram
-//               and X products); Gram epilogue; the whole inversion
+//               turns the tiles in place into Qtil and Etil (the A operand
+//               [Etil; Qtil] of the Gram and X products, read from shared
+//               memory) and writes Ktil (the Gram's B operand); while the Gram
+//               runs, Ktil^T goes into Tensor Memory (the state update's A
+//               operand, two buffers); Gram epilogue; the whole inversion
 //               T = (I + A)^{-1}
 //   warps 9-16  state side: R epilogue (w, v straight from global memory into
-//               registers), U, state and output epilogues
+//               registers), U, state and output epilogues; once X has read the
+//               chunk's [Etil; Qtil] it issues the next chunk's alpha, b load
 // The state chain of a chunk is X -> R -> U -> state update; everything that
 // does not depend on the state (gate prep, Gram, T) is done one chunk ahead.
 // The FP32 state lives in Tensor Memory: the state-update MMA accumulates
@@ -133,17 +134,17 @@ constexpr uint32_t TX_AB_LOGITS = 4 * TILE;            // their BF16 logits
 constexpr uint32_t TX_QK = 4 * TILE;                   // q and k of one chunk
 
 // Tensor Memory columns (512 allocated).
-constexpr uint32_t TM_EQ = 0;       // A operand [Etil; Qtil]: lane t (0-63 Etil, 64-127 Qtil), column i  (128 cols)
-constexpr uint32_t TM_X = 128;      // [Etil;Qtil] S, then + P U: lanes 64-127 -> O                     (64 cols)
-constexpr uint32_t TM_U = 192;      // U = T R (lanes 0-63)                                             (64 cols)
-constexpr uint32_t TM_S = 256;      // FP32 state S[i][j], lane i, column j                             (64 cols)
-constexpr uint32_t TM_TP = 320;     // 2 buffers: the Gram [A; P], then the A operand [T; P]            (2 x 64 cols)
-constexpr uint32_t TM_KH = 448;     // A operand Ktil^T, lane i, column s                               (64 cols)
+constexpr uint32_t TM_X = 0;        // [Etil;Qtil] S, then + P U: lanes 64-127 -> O                     (64 cols)
+constexpr uint32_t TM_U = 64;       // U = T R (lanes 0-63)                                             (64 cols)
+constexpr uint32_t TM_S = 128;      // FP32 state S[i][j], lane i, column j                             (64 cols)
+constexpr uint32_t TM_TP = 192;     // 2 buffers: the Gram [A; P], then the A operand [T; P]            (2 x 64 cols)
+constexpr uint32_t TM_KH = 320;     // 2 buffers: A operand Ktil^T, lane i, column s                    (2 x 64 cols)
 constexpr uint32_t TM_COLS = 512;
 
 enum {
-    B_KPREP = 0, B_G_FULL, B_S_READY, B_X_FULL, B_R_READY, B_TP_READY0, B_TP_READY1, B_U_FULL, B_U_READY,
-    B_D_FULL, B_O_FULL, B_KH_READY, B_KH_FREE, B_TP_FREE0, B_TP_FREE1, B_RR0, B_RR1, B_RR2, B_RR3,
+    B_G_FULL = 0, B_S_READY, B_X_FULL, B_R_READY, B_TP_READY0, B_TP_READY1, B_U_FULL, B_U_READY,
+    B_D_FULL, B_O_FULL, B_KH_READY0, B_KH_READY1, B_KH_FREE0, B_KH_FREE1, B_TP_FREE0, B_TP_FREE1, B_RR0, B_RR1,
+    B_RR2, B_RR3,
     B_FULL_AB, B_FULL_QK, B_DRAIN, B_GRAM_GO, NBARS
 };
 static_assert(NBARS * 8 <= 256, "barrier area");
@@ -350,29 +351,9 @@ __device__ __forceinline__ int key_decay(const Ctx &c, int ktid, int t0, int nav
 
 
 
-// Key side, pass B (thread per token t, channel half ch): the rows of Etil
-// (lanes 0-63) or Qtil (lanes 64-127) of 64 channels into the TMEM operand.
-__device__ __forceinline__ void key_rows(const Ctx &c, uint32_t tmem, int warp, int lane) {
-    const int lq = warp & 3, ch = (warp - 1) >> 2;
-    const int t = 32 * (lq & 1) + lane;
-    const uint32_t tl = tmem + TM_EQ + ((uint32_t)(32 * lq) << 16);
-#pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-        const int a = 2 * ch + blk;
-        const uint32_t src = lq < 2 ? OFF_E(a) : OFF_Q(a);
-        float x[32];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const float4 g4 = *reinterpret_cast<const float4 *>(c.sm + src + swz128(t, 16 * m));
-            x[4 * m] = g4.x; x[4 * m + 1] = g4.y; x[4 * m + 2] = g4.z; x[4 * m + 3] = g4.w;
-        }
-        tmem_st32_nowait(tl + 32 * a, x);
-    }
-}
-
 // Key side: Ktil^T of the chunk from KG into Tensor Memory (thread per key
 // channel i and token half, lane i), the A operand of the state update.
-__device__ __forceinline__ void key_kt(const Ctx &c, uint32_t tmem, int warp, int lane) {
+__device__ __forceinline__ void key_kt(const Ctx &c, uint32_t tmem, int warp, int lane, int buf) {
     const int cb = warp & 3, hh = (warp - 1) >> 2;
     const int i = 32 * cb + lane;
     const Swz sw((i & 31) * 4u);
@@ -380,7 +361,7 @@ __device__ __forceinline__ void key_kt(const Ctx &c, uint32_t tmem, int warp, in
     float x[32];
 #pragma unroll
     for (int tt = 0; tt < 32; ++tt) x[tt] = at(c, fb + tt * 128 + sw.o[tt & 7]);
-    tmem_st32_nowait(tmem + TM_KH + ((uint32_t)(32 * cb) << 16) + 32 * hh, x);
+    tmem_st32_nowait(tmem + TM_KH + 64 * buf + ((uint32_t)(32 * cb) << 16) + 32 * hh, x);
 }
 
 // The chunk's alpha and b tiles (or q and k) by TMA.
@@ -506,12 +487,22 @@ __device__ __forceinline__ void store_split_jt(const Ctx &c, const float (&x)[32
 // Descriptor offset (16-byte units) of K-step kk (8 TF32 = 32 bytes) in a
 // K-major tile of 64-row blocks: 4 K-steps per 128-byte row, then the next block.
 __device__ __forceinline__ uint32_t kstep(int kk) { return ((kk >> 2) * TILE + (kk & 3) * 32) >> 4; }
+// The same for the 128-row A operand [Etil; Qtil]: its channel blocks are E/Q tile pairs (2 tiles apart).
+__device__ __forceinline__ uint32_t eq_step(int kk) { return ((kk >> 2) * 2 * TILE + (kk & 3) * 32) >> 4; }
 
-// The MMA issuer (one thread).  Four streams of work, each in chunk order:
-// the Gram of chunk cg, the X product of chunk cx, U of chunk cu, the state
-// update and output of chunk cs.  Whichever has its inputs ready is issued,
-// the state chain first.  A separate function keeps its few live values out of
-// the other roles' register allocation.
+// A bounded mbarrier test whose outcome is the same in every lane of the warp
+// (a phase, once complete, stays complete, so any lane's yes is everyone's).
+__device__ __forceinline__ bool warp_test(const Ctx &c, int which, uint32_t parity) {
+    return __any_sync(0xffffffffu, mbar_test(c.bar(which), parity));
+}
+
+// The MMA issuer (warp 0).  Four streams of work, each in chunk order: the Gram
+// of chunk cg, the X product of chunk cx, U of chunk cu, the state update and
+// output of chunk cs.  Whichever has its inputs ready is issued, the state
+// chain first.  The whole warp runs the loop and takes every decision by vote,
+// so that descriptors and counters stay warp-uniform; one elected lane (always
+// the same, the lowest) issues the tcgen05 instructions.  A separate function
+// keeps its few live values out of the other roles' register allocation.
 __device__ __noinline__ void issuer_role(const Ctx &c, uint32_t tmem) {
     // B descriptors as (low, high) halves; the K-step offset is added inside each MMA's asm.
     const uint64_t dSC = sdesc_sw128(c.sa + OFF_SC, 16, 1024), dKG = sdesc_sw128(c.sa + OFF_KG, 16, 1024);
@@ -521,60 +512,73 @@ __device__ __noinline__ void issuer_role(const Ctx &c, uint32_t tmem) {
     const uint32_t hi = (uint32_t)(dSC >> 32);      // identical for every tile (layout, SBO, version)
     const uint32_t sc = (uint32_t)dSC, kg = (uint32_t)dKG, uh = (uint32_t)dUH, ul = (uint32_t)dUL;
     const uint32_t id = idesc_tf32(128, 64, 0, 0);
+    const bool lane0 = (threadIdx.x & 31) == 0;
     int cg = 0, cx = 0, cu = 0, cs = 0, lastc = 0x7fffffff;
     long long t_prog = clock64();
     while (cs <= lastc) {
-        if (cs < cu && mbar_test(c.bar(B_U_READY), cs & 1) && mbar_test(c.bar(B_KH_READY), cs & 1)) {
+        if (cs < cu && warp_test(c, B_U_READY, cs & 1) &&
+            warp_test(c, (cs & 1) ? B_KH_READY1 : B_KH_READY0, (cs >> 1) & 1)) {
             // S + Ktil^T (U_hi + U_lo) onto the state;  P U_hi onto TM_X (-> O)
-            const uint32_t tp = tmem + TM_TP + 64 * (cs & 1);
-            tc_fence_after();
+            const uint32_t tp = tmem + TM_TP + 64 * (cs & 1), kh = tmem + TM_KH + 64 * (cs & 1);
+            if (elect_one_sync()) {
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_tf32_ts_off(tmem + TM_S, tmem + TM_KH + 8 * kk, uh, hi, kstep(kk), id, 1);
-                mma_tf32_ts_off(tmem + TM_S, tmem + TM_KH + 8 * kk, ul, hi, kstep(kk), id, 1);
+                for (int kk = 0; kk < 8; ++kk) {
+                    mma_tf32_ts_off(tmem + TM_S, kh + 8 * kk, uh, hi, kstep(kk), id, 1);
+                    mma_tf32_ts_off(tmem + TM_S, kh + 8 * kk, ul, hi, kstep(kk), id, 1);
+                }
+                mma_commit(c.bar(B_D_FULL));
+                mma_commit(c.bar((cs & 1) ? B_KH_FREE1 : B_KH_FREE0));
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) mma_tf32_ts_off(tmem + TM_X, tp + 8 * kk, uh, hi, kstep(kk), id, 1);
+                mma_commit(c.bar(B_O_FULL));
+                mma_commit(c.bar((cs & 1) ? B_TP_FREE1 : B_TP_FREE0));
             }
-            mma_commit(c.bar(B_D_FULL));
-            mma_commit(c.bar(B_KH_FREE));
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) mma_tf32_ts_off(tmem + TM_X, tp + 8 * kk, uh, hi, kstep(kk), id, 1);
-            mma_commit(c.bar(B_O_FULL));
-            mma_commit(c.bar((cs & 1) ? B_TP_FREE1 : B_TP_FREE0));
+            __syncwarp();
             ++cs;
-        } else if (cu < cx && mbar_test(c.bar(B_R_READY), cu & 1) &&
-                   mbar_test(c.bar((cu & 1) ? B_TP_READY1 : B_TP_READY0), (cu >> 1) & 1)) {
+        } else if (cu < cx && warp_test(c, B_R_READY, cu & 1) &&
+                   warp_test(c, (cu & 1) ? B_TP_READY1 : B_TP_READY0, (cu >> 1) & 1)) {
             // U = [T; P] (R_hi + R_lo)
             const uint32_t tp = tmem + TM_TP + 64 * (cu & 1);
-            tc_fence_after();
+            if (elect_one_sync()) {
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_tf32_ts_off(tmem + TM_U, tp + 8 * kk, uh, hi, kstep(kk), id, kk > 0);
-                mma_tf32_ts_off(tmem + TM_U, tp + 8 * kk, ul, hi, kstep(kk), id, 1);
+                for (int kk = 0; kk < 8; ++kk) {
+                    mma_tf32_ts_off(tmem + TM_U, tp + 8 * kk, uh, hi, kstep(kk), id, kk > 0);
+                    mma_tf32_ts_off(tmem + TM_U, tp + 8 * kk, ul, hi, kstep(kk), id, 1);
+                }
+                mma_commit(c.bar(B_U_FULL));
             }
-            mma_commit(c.bar(B_U_FULL));
+            __syncwarp();
             ++cu;
-        } else if (cx < cg && mbar_test(c.bar(B_KPREP), cx & 1) && mbar_test(c.bar(B_S_READY), cx & 1)) {
-            // [Etil; Qtil] S
-            tc_fence_after();
+        } else if (cx < cg && warp_test(c, B_S_READY, cx & 1)) {
+            // [Etil; Qtil] S, A from the shared-memory tiles (the Gram of the chunk found them ready)
+            if (elect_one_sync()) {
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk) mma_tf32_ts_off(tmem + TM_X, tmem + TM_EQ + 8 * kk, sc, hi, kstep(kk), id, kk > 0);
-            mma_commit(c.bar(B_X_FULL));
+                for (int kk = 0; kk < 16; ++kk)
+                    mma_tf32_ss_off(tmem + TM_X, eq, eq_step(kk), sc, kstep(kk), hi, id, kk > 0);
+                mma_commit(c.bar(B_X_FULL));
+            }
+            __syncwarp();
             ++cx;
-        } else if (cg <= lastc && mbar_test(c.bar(B_GRAM_GO), cg & 1) &&
-                   (cg < 2 || mbar_test(c.bar((cg & 1) ? B_TP_FREE1 : B_TP_FREE0), ((cg - 2) >> 1) & 1))) {
+        } else if (cg <= lastc && warp_test(c, B_GRAM_GO, cg & 1) &&
+                   (cg < 2 || warp_test(c, (cg & 1) ? B_TP_FREE1 : B_TP_FREE0, ((cg - 2) >> 1) & 1))) {
             // Gram [Etil; Qtil] Ktil^T into the chunk's [T; P] buffer
-            tc_fence_after();
-            if (rec(c, cg).last) lastc = cg;
+            if (__any_sync(0xffffffffu, rec(c, cg).last != 0)) lastc = cg;
             const uint32_t tp = tmem + TM_TP + 64 * (cg & 1);
+            if (elect_one_sync()) {
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk)    // A from the shared-memory tiles, before they reach TMEM
-                mma_tf32_ss_off(tp, eq, (uint32_t)(((kk >> 2) * 2 * TILE + (kk & 3) * 32) >> 4), kg, kstep(kk), hi,
-                                id, kk > 0);
-            mma_commit(c.bar(B_G_FULL));
+                for (int kk = 0; kk < 16; ++kk) mma_tf32_ss_off(tp, eq, eq_step(kk), kg, kstep(kk), hi, id, kk > 0);
+                mma_commit(c.bar(B_G_FULL));
+            }
+            __syncwarp();
             ++cg;
         } else {
-            if (*c.abort_flag) break;
-            if (clock64() - t_prog > c.limit) {
-                record_abort(c, B_DRAIN);
+            if (__any_sync(0xffffffffu, *c.abort_flag != 0)) break;
+            if (__any_sync(0xffffffffu, clock64() - t_prog > c.limit)) {
+                if (lane0) record_abort(c, B_DRAIN);
                 break;
             }
             continue;
@@ -582,7 +586,8 @@ __device__ __noinline__ void issuer_role(const Ctx &c, uint32_t tmem) {
         t_prog = clock64();
     }
     // Every MMA issued above has completed before Tensor Memory is released (bounded).
-    mma_commit(c.bar(B_DRAIN));
+    if (elect_one_sync()) mma_commit(c.bar(B_DRAIN));
+    __syncwarp();
     (void)mbar_wait(c.bar(B_DRAIN), 0, kDrainLimit);
 }
 
@@ -634,7 +639,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
 
     if (warp == 0) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0 && !empty) issuer_role(c, tmem);
+        if (!empty) issuer_role(c, tmem);
         __syncwarp();
     } else if (warp <= 8) {
         // ------------------------------------------------ key side
@@ -660,9 +665,13 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
             if (el) {
                 *reinterpret_cast<volatile int *>(c.sm + OFF_MISC + 8) = kC;
                 const int tn = t0 + kC;
-                if (tn < te) {      // the next chunk's w, v into L2 for the state side
+                if (tn < te) {      // the next chunk's w, v (state side) and alpha, b (its TMA load) into L2
                     for (int a = 0; a < (kLogits ? 1 : 2); ++a) tma_prefetch_3d(&maps.w, col0 + 32 * a, h, tn);
                     tma_prefetch_3d(&maps.v, col0, h, tn);
+                    for (int a = 0; a < (kLogits ? 2 : 4); ++a) {
+                        tma_prefetch_3d(&maps.alpha, kLogits ? 64 * a : 32 * a, h, tn);
+                        tma_prefetch_3d(&maps.b, kLogits ? 64 * a : 32 * a, h, tn);
+                    }
                 }
             }
             const int n = key_decay<kLogits>(c, ktid, t0, navail, te, r, el);
@@ -677,20 +686,17 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                     pend_qk = ck + 1;
                 }
             }
-            // [Etil; Qtil] into Tensor Memory once the previous X product has read it
-            if (ck >= 1 && !group_wait(c, B_X_FULL, (ck - 1) & 1, el, kBarK)) break;
-            key_rows(c, tmem, warp, lane);
+            // While the Gram runs: Ktil^T into Tensor Memory (buffer ck & 1) once the state
+            // update two chunks back has read that buffer
+            if (ck >= 2 && !group_wait(c, ph ? B_KH_FREE1 : B_KH_FREE0, ((ck - 2) >> 1) & 1, el, kBarK)) break;
+            tc_fence_after();
+            key_kt(c, tmem, warp, lane, ph);
             tmem_wait_st();
-            fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarK, kGroup);
-            if (el) mbar_arrive(c.bar(B_KPREP));
+            if (el) mbar_arrive(c.bar(ph ? B_KH_READY1 : B_KH_READY0));
             // Gram epilogue: A (rows 0-63, strictly lower) -> AS; P (rows 64-127) masked in place.
             if (!group_wait(c, B_G_FULL, ph, el, kBarK)) break;
-            if (el && !last) {                 // the Gram and the row pass have read alpha -> Qtil, b -> Etil
-                load_ab<kLogits>(c, maps, h, t0 + n);
-                pend_ab = ck + 1;
-            }
             tc_fence_after();
             {
                 const uint32_t tp = tlane + TM_TP + 64 * ph + 32 * ch;
@@ -724,14 +730,6 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
             tc_fence_before();
             named_bar(kBarK, kGroup);
             if (el) mbar_arrive(c.bar(ph ? B_TP_READY1 : B_TP_READY0));
-            // Ktil^T into Tensor Memory once the previous state update has read it
-            if (ck >= 1 && !group_wait(c, B_KH_FREE, (ck - 1) & 1, el, kBarK)) break;
-            tc_fence_after();
-            key_kt(c, tmem, warp, lane);
-            tmem_wait_st();
-            tc_fence_before();
-            named_bar(kBarK, kGroup);
-            if (el) mbar_arrive(c.bar(B_KH_READY));
             if (last) break;
             t0 += n;
         }
@@ -776,6 +774,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
             named_bar(kBarS, kGroup);
             if (el) mbar_arrive(c.bar(B_S_READY));
             bool done_ok = true;
+            int pend_ab = -1;      // chunk whose alpha, b load this side issued, not yet known to be complete
             for (int ck = 0;; ++ck) {
                 const uint32_t ph = ck & 1;
                 if (!group_wait(c, B_RR0 + (ck & 3), (ck >> 2) & 1, el, kBarS)) { done_ok = false; break; }
@@ -824,6 +823,10 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                 }
                 // R = w*v - Etil S (lanes 0-63) -> R_hi, R_lo
                 if (!group_wait(c, B_X_FULL, ph, el, kBarS)) { done_ok = false; break; }
+                if (el && !last) {     // the Gram and X have read Qtil and Etil: the next chunk's alpha, b over them
+                    load_ab<kLogits>(c, maps, h, t0 + n);
+                    pend_ab = ck + 1;
+                }
                 tc_fence_after();
                 if (srow < 64) {
                     float x[32];
@@ -893,6 +896,8 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                 if (el) mbar_arrive(c.bar(B_S_READY));
                 if (last) break;
             }
+            // No copy into shared memory may still be in flight when the CTA ends (bounded).
+            if (el && pend_ab >= 0) (void)mbar_wait(c.bar(B_FULL_AB), pend_ab & 1, kDrainLimit);
             if (done_ok && *c.abort_flag == 0 && p.S_T) {
                 float S[32];
                 tmem_ld32(ts, S);

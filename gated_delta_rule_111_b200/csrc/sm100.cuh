@@ -298,6 +298,15 @@ __device__ __forceinline__ void mma_tf32_ss_off(uint32_t d_tmem, uint32_t a_lo, 
         "r"(a_lo), "r"(a_off), "r"(b_lo), "r"(b_off), "r"(hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// One lane of a fully active warp (the lowest) gets 1, the others 0.  Code that
+// decides and computes as a whole warp and lets this lane issue the tcgen05
+// instructions keeps the operands warp-uniform; a lone lane issuing them from
+// divergent code takes about twice as long per MMA.
+__device__ __forceinline__ uint32_t elect_one_sync() {
+    uint32_t p;
+    asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}\n" : "=r"(p));
+    return p;
+}
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
