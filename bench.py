@@ -335,9 +335,10 @@ def run_ours(args):
         ms_step, e2e_ms, h2d, d2h, clk = run_prefill(args, torch, dist, g, world, rank, dev, stream)
     if args.workload in ("all", "decode"):
         dec_ms = run_decode(args, torch, dist, g, world, rank, dev, stream)
-    long_ms = float("nan")
+    long_ms = long_seg_ms = float("nan")
+    long_segments = 1
     if args.workload in ("all", "long"):
-        long_ms = run_long(args, torch, dist, g, world, rank, dev, stream)
+        long_ms, long_seg_ms, long_segments = run_long(args, torch, dist, g, world, rank, dev, stream)
     bwd_ms = float("nan")
     if args.workload in ("all", "backward"):
         bwd_ms = run_backward(args, torch, dist, g, world, rank, dev, stream)
@@ -347,7 +348,8 @@ def run_ours(args):
     og_ms = float("nan")
     if args.workload in ("all", "output_gate"):
         og_ms = run_output_gate(args, torch, dist, g, world, rank, dev, stream)
-    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms, bwd_ms, lg_ms, og_ms)
+    report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, (long_ms, long_seg_ms, long_segments), bwd_ms,
+           lg_ms, og_ms)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -448,8 +450,9 @@ def run_decode(args, torch, dist, g, world, rank, dev, stream):
 
 
 def run_long(args, torch, dist, g, world, rank, dev, stream):
-    """One prefill call on the long ragged workload (B=1, T=65,573, H=16, S0 != 0): latency
-    bound (32 CTAs, 1,025 chunks each), reported for the record; returns ms per call."""
+    """The long ragged workload (B=1, T=65,573, H=16, S0 != 0): one sequential prefill call
+    (32 CTAs walk 1,025 chunks each) and one segment-parallel call with the automatic segment
+    count.  Returns (ms per sequential call, ms per segmented call, segments)."""
     x = gi.chunk_inputs(**LONG, seed=rank)
     d = device_inputs(torch, x, dev)
     S0 = torch.from_numpy(x["S0"]).to(dev)
@@ -458,22 +461,32 @@ def run_long(args, torch, dist, g, world, rank, dev, stream):
     o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
     ST = torch.empty_like(S0)
 
+    segments = g.gdn2_chunk_fwd_segments(B, T, H, LONG["dk"], dv, 0)
+    ws = torch.empty((max(g.gdn2_chunk_fwd_segmented_workspace_size(B, T, H, LONG["dk"], dv, 0), 1),),
+                     dtype=torch.uint8, device=dev)
+
     def call():
         g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], S0, o=o, S_T=ST, stream=stream)
 
-    call()
-    sync_ranks(torch, dist, world)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 3
-    ev0.record(stream)
-    for _ in range(reps):
-        call()
-    ev1.record(stream)
-    sync_ranks(torch, dist, world)
-    ms = max_over_ranks(ev0.elapsed_time(ev1) / reps, torch, dist, world, dev)
-    del d, S0, o, ST
+    def call_seg():
+        g.gdn2_chunk_fwd_segmented(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], S0, segments=0,
+                                   workspace=ws, o=o, S_T=ST, stream=stream)
+
+    out = []
+    for fn in (call, call_seg):
+        fn()
+        sync_ranks(torch, dist, world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        ev0.record(stream)
+        for _ in range(reps):
+            fn()
+        ev1.record(stream)
+        sync_ranks(torch, dist, world)
+        out.append(max_over_ranks(ev0.elapsed_time(ev1) / reps, torch, dist, world, dev))
+    del d, S0, o, ST, ws
     torch.cuda.empty_cache()
-    return ms
+    return out[0], out[1], segments
 
 
 def run_backward(args, torch, dist, g, world, rank, dev, stream):
@@ -585,8 +598,10 @@ def _num(x):
     return None if x != x else x      # NaN (workload not run) -> null
 
 
-def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=float("nan"), bwd_ms=float("nan"),
-           lg_ms=float("nan"), og_ms=float("nan")):
+def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long=(float("nan"), float("nan"), 1),
+           bwd_ms=float("nan"), lg_ms=float("nan"), og_ms=float("nan")):
+    """long: (ms per sequential call, ms per segmented call, segments) of the long ragged workload."""
+    long_ms, long_seg_ms, long_segments = long
     B, T, H, dk, dv = (PREFILL[n] for n in ("B", "T", "H", "dk", "dv"))
     Bd, Hd = DECODE["B"], DECODE["H"]
     steps_d = DECODE["steps"]
@@ -651,14 +666,18 @@ def report(args, world, rank, ms_step, e2e_ms, h2d, d2h, dec_ms, clk, long_ms=fl
                                     "frac_of_8TBps": _num(dec_gbs / 8000.0)},
                        "cpu_baseline": dec_cpu},
             "long_ragged": {"workload": "B=1 T=65573 H=16 d_k=d_v=128, S0 != 0 (ragged last chunk)",
-                            "ms_per_call": _num(long_ms),
-                            "tokens_per_s": _num(LONG["B"] * LONG["T"] * world / (long_ms / 1e3)),
-                            "note": "latency bound: 32 CTAs walk 1,025 chunks each; reported, no target",
+                            "ms_per_call": _num(long_seg_ms),
+                            "tokens_per_s": _num(LONG["B"] * LONG["T"] * world / (long_seg_ms / 1e3)),
+                            "segments": long_segments,
+                            "ms_per_call_sequential": _num(long_ms),
+                            "note": "gdn2_chunk_fwd_segmented with the automatic segment count (three passes "
+                                    "over 4 (P-1) + 2 P CTAs per head); the sequential call has 32 CTAs walk "
+                                    "1,025 chunks each; reported, no target",
                             "cpu_baseline": long_cpu},
             "backward": {"metric": "GDN-2 chunk bwd tokens/s @H16 d128 T4K", "unit": "tokens/s",
                          "value": _num(job_tokens_per_s(B, T, world, bwd_ms)), "ms_per_call": _num(bwd_ms),
                          "workload": "gradients of every input of the prefill workload (BF16 dO, dST = 0)",
-                         "launches_per_call": 3,
+                         "launches_per_call": 5,
                          "roofline": {"bound": "hbm", "achieved": _num(bwd_gbs), "peak": hbm, "unit": "GB/s",
                                       "frac": _num(bwd_gbs / hbm), "traffic": traffic.get("gdn2_chunk_bwd"),
                                       "algorithmic_bytes_per_launch": bwd_bytes,

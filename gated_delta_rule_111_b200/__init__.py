@@ -9,6 +9,10 @@ Functions (same names as the C ABI):
   gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, ...)  -> (o, S_T)   chunkwise prefill
   gdn2_chunk_fwd_varlen(q, k, v, alpha, b, w, cu_seqlens, S0=None, ...)
                                                       -> (o, S_T)   packed variable-length batch
+  gdn2_chunk_fwd_segmented(q, k, v, alpha, b, w, S0=None, segments=0, ...)
+                                                      -> (o, S_T)   segment-parallel prefill (long sequences)
+  gdn2_chunk_fwd_segmented_workspace_size(B, T, H, dk, dv, segments) -> bytes
+  gdn2_chunk_fwd_segments(B, T, H, dk, dv, segments)  -> int        segments that call would use
   gdn2_chunk_fwd_logits(xq, xk, xv, xa, xb, xw, S0=None, ...) -> (o, S_T)  prefill from BF16 logits
   gdn2_recurrent_step(q, k, v, alpha, b, w, S, ...)   -> o          in-place decode step
   gdn2_output_gate(o, g, weight, eps, ...)            -> y          RMS norm + sigmoid output gate
@@ -26,7 +30,8 @@ import torch
 
 from . import build as _build
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_logits", "gdn2_output_gate", "gdn2_recurrent_step", "gdn2_chunk_bwd",
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_segmented", "gdn2_chunk_fwd_segmented_workspace_size",
+           "gdn2_chunk_fwd_segments", "gdn2_chunk_fwd_logits", "gdn2_output_gate", "gdn2_recurrent_step", "gdn2_chunk_bwd",
            "gdn2_chunk_bwd_workspace_size", "gdn2_chunk_bwd_noalloc", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
            "load_library", "exported_symbols",
            "GDN2_OK", "GDN2_ERR_INVALID_ARG", "GDN2_ERR_UNSUPPORTED", "GDN2_ERR_CUDA", "Gdn2Error"]
@@ -57,18 +62,23 @@ def load_library(rebuild_if_stale: bool = True) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(f"libgdn2.so not found at {path}; run python -m gated_delta_rule_111_b200.build")
     lib = ctypes.CDLL(path)
-    vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+    vp, fp, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.gdn2_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp]
     lib.gdn2_chunk_fwd.restype = i
     lib.gdn2_chunk_fwd_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, i, fp, vp, fp, i, i, i, i, i, vp]
     lib.gdn2_chunk_fwd_varlen.restype = i
+    lib.gdn2_chunk_fwd_segmented.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.gdn2_chunk_fwd_segmented.restype = i
+    lib.gdn2_chunk_fwd_segmented_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.gdn2_chunk_fwd_segmented_workspace_size.restype = sz
+    lib.gdn2_chunk_fwd_segments.argtypes = [i, i, i, i, i, i]
+    lib.gdn2_chunk_fwd_segments.restype = i
     lib.gdn2_chunk_fwd_logits.argtypes = [vp, vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
     lib.gdn2_chunk_fwd_logits.restype = i
     lib.gdn2_output_gate.argtypes = [vp, vp, fp, ctypes.c_float, vp, i, i, i, i, i, vp]
     lib.gdn2_output_gate.restype = i
     lib.gdn2_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn2_recurrent_step.restype = i
-    sz = ctypes.c_size_t
     lib.gdn2_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, fp, vp, sz,
                                    i, i, i, i, i, i, vp]
     lib.gdn2_chunk_bwd.restype = i
@@ -174,6 +184,56 @@ def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, *, o=None, S_T=None, output_fi
     with torch.cuda.device(dev):
         _check(lib.gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
                                   _ptr(S_T), B, T, H, dk, dv, code, _stream(stream, dev)))
+    return o, S_T
+
+
+def gdn2_chunk_fwd_segmented_workspace_size(B, T, H, dk, dv, segments=0) -> int:
+    """Workspace bytes of gdn2_chunk_fwd_segmented (segments = 0 resolves against the current device)."""
+    return int(load_library().gdn2_chunk_fwd_segmented_workspace_size(B, T, H, dk, dv, segments))
+
+
+def gdn2_chunk_fwd_segments(B, T, H, dk, dv, segments=0) -> int:
+    """The number of segments gdn2_chunk_fwd_segmented uses for this shape (1: the plain call)."""
+    return int(load_library().gdn2_chunk_fwd_segments(B, T, H, dk, dv, segments))
+
+
+def gdn2_chunk_fwd_segmented(q, k, v, alpha, b, w, S0=None, *, segments=0, workspace=None, o=None, S_T=None,
+                             output_final_state=True, stream=None):
+    """Segment-parallel chunkwise prefill: arguments and result as gdn2_chunk_fwd; each sequence is cut
+    into ``segments`` pieces (0: chosen from the shape and the device) processed in parallel.
+    ``workspace``: a uint8 CUDA tensor of at least gdn2_chunk_fwd_segmented_workspace_size(...)
+    bytes, allocated here when None."""
+    lib = load_library()
+    if q.device.type != "cuda":
+        raise ValueError("gdn2_chunk_fwd_segmented needs CUDA tensors (there is no CPU implementation)")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("q", q, dk), ("k", k, dk), ("v", v, dv)):
+        _need(t, name, dt, (B, T, H, d), dev)
+    for name, t, d in (("alpha", alpha, dk), ("b", b, dk), ("w", w, dv)):
+        _need(t, name, torch.float32, (B, T, H, d), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _need(o, "o", dt, (B, T, H, dv), dev)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    elif S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        need = int(lib.gdn2_chunk_fwd_segmented_workspace_size(B, T, H, dk, dv, int(segments)))
+        if workspace is None:
+            workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=dev)
+        elif workspace.dtype != torch.uint8 or workspace.device != dev or not workspace.is_contiguous():
+            raise ValueError("workspace: expected a contiguous uint8 tensor on the inputs' device")
+        _check(lib.gdn2_chunk_fwd_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0),
+                                            _ptr(o), _ptr(S_T), B, T, H, dk, dv, code, int(segments),
+                                            _ptr(workspace) if need > 0 else None, workspace.numel(),
+                                            _stream(stream, dev)))
     return o, S_T
 
 

@@ -161,6 +161,9 @@ struct Params {
     __nv_bfloat16 *o;
     float *S_T;
     const int *cu_seqlens;    // nullptr: nseq sequences of T tokens; else packed offsets [nseq + 1]
+    const int4 *ranges;       // else (non-null): sequence i is tokens [x, y) of the flat axis, and z != 0 makes
+                              // its written values zero (the state's transition over the range alone)
+    int nst;                  // sequences with an index below this write S_T
     int T, H;
     long long wait_limit;     // SM cycles before a pipeline wait gives up
 };
@@ -609,7 +612,13 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
     const int unit = blockIdx.x >> 1, half = blockIdx.x & 1;   // unit = sequence * H + head
     const int seq = unit / p.H, h = unit % p.H;
     int tb, te;
-    if (p.cu_seqlens) {         // packed offsets, clamped to the T tokens there are
+    bool zero_z = false;
+    if (p.ranges) {             // explicit token ranges, clamped to the T tokens there are
+        const int4 rg = p.ranges[seq];
+        tb = min(max(rg.x, 0), p.T);
+        te = min(max(rg.y, tb), p.T);
+        zero_z = rg.z != 0;
+    } else if (p.cu_seqlens) {  // packed offsets, clamped to the T tokens there are
         tb = min(max(p.cu_seqlens[seq], 0), p.T);
         te = min(max(p.cu_seqlens[seq + 1], tb), p.T);
     } else {
@@ -746,8 +755,9 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
         const Swz ssw((srow & 31) * 4u);
         const uint32_t sbase = OFF_SC + (srow >> 5) * TILE + 32 * sh * 128;   // S[i][j] at [j][i]
         const size_t srow_off = soff + (size_t)srow * kDV + col0 + 32 * sh;
+        const bool write_st = p.S_T != nullptr && seq < p.nst;
         if (empty) {
-            if (p.S_T) {
+            if (write_st) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
                     const float4 x = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + srow_off + j)
@@ -785,7 +795,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                 // the loads complete while the MMA below runs.  Tokens past the chunk read as zero.
                 float z[32];
                 if (srow < 64) {
-                    if (srow < n) {
+                    if (srow < n && !zero_z) {
                         const size_t row = ((size_t)(t0 + srow) * p.H + h) * kDV + col0 + 32 * sh;
                         const uint4 *vp = reinterpret_cast<const uint4 *>(p.v + row);
                         if constexpr (kLogits) {      // z = sigmoid(xw) silu(xv)
@@ -872,7 +882,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
                     float v[32];
                     tmem_ld32(tlane + TM_X + 32 * sh, v);
                     const int t = srow - 64;
-                    if (t < n) {
+                    if (t < n && p.o) {
                         __nv_bfloat16 *dst = p.o + ((size_t)(t0 + t) * p.H + h) * kDV + col0 + 32 * sh;
 #pragma unroll
                         for (int j = 0; j < 32; j += 8) {
@@ -898,7 +908,7 @@ chunk_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Param
             }
             // No copy into shared memory may still be in flight when the CTA ends (bounded).
             if (el && pend_ab >= 0) (void)mbar_wait(c.bar(B_FULL_AB), pend_ab & 1, kDrainLimit);
-            if (done_ok && *c.abort_flag == 0 && p.S_T) {
+            if (done_ok && *c.abort_flag == 0 && write_st) {
                 float S[32];
                 tmem_ld32(ts, S);
 #pragma unroll
@@ -969,14 +979,19 @@ cudaError_t read_device_error(unsigned int *value, bool clear) {
     return e;
 }
 
-// nseq sequences: of T tokens each (cu_seqlens == nullptr), or packed with
-// device offsets cu_seqlens[0..nseq] into T_total = T tokens.
+// nseq sequences: of T tokens each (cu_seqlens and ranges null), packed with
+// device offsets cu_seqlens[0..nseq] into T_total = T tokens, or given as device
+// token ranges ranges[0..nseq) of T_total = T tokens (z != 0: written values
+// taken as zero).  o may be null (no output written); only sequences below nst
+// (all, when nst < 0) write S_T.
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *alpha, const void *b,
                             const void *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
-                            const int *cu_seqlens, bool logits, cudaStream_t stream) {
+                            const int *cu_seqlens, bool logits, cudaStream_t stream, const int4 *ranges,
+                            int nst) {
     using namespace tc;
-    const long long NT = cu_seqlens ? (long long)T : (long long)nseq * T;
-    if (NT <= 0 && !cu_seqlens) return cudaSuccess;
+    const bool packed = cu_seqlens != nullptr || ranges != nullptr;
+    const long long NT = packed ? (long long)T : (long long)nseq * T;
+    if (NT <= 0 && !packed) return cudaSuccess;
     Maps m;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const long long NTm = NT > 0 ? NT : 1;
@@ -1008,6 +1023,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const v
     prm.o = static_cast<__nv_bfloat16 *>(o);
     prm.S_T = S_T;
     prm.cu_seqlens = cu_seqlens;
+    prm.ranges = ranges;
+    prm.nst = nst < 0 ? nseq : nst;
     prm.T = T;
     prm.H = H;
     prm.wait_limit = g_wait_limit.load();

@@ -39,6 +39,24 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
                               int B, int T, int H, int dk, int dv, gdn2_dtype dt, const int *cu_seqlens,
                               cudaStream_t stream);
 
+// Chunkwise prefill on the tensor cores (BF16 q/k/v, d_k = d_v = 128): nseq
+// sequences of T tokens each; or packed, with device offsets cu_seqlens[0..nseq]
+// or device token ranges ranges[0..nseq) (x, y: tokens [x, y) of the flat axis;
+// z != 0: written values taken as zero) into T tokens in all.  o may be null;
+// only sequences below nst (all when nst < 0) write S_T.
+bool chunk_tc_supported(int dk, int dv, gdn2_dtype dt);
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *alpha, const void *b,
+                            const void *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
+                            const int *cu_seqlens, bool logits, cudaStream_t stream, const int4 *ranges = nullptr,
+                            int nst = -1);
+
+// Segment-parallel prefill of B sequences of T tokens cut into P segments of L
+// tokens (the last shorter): workspace of segmented_workspace_bytes(B, H, P).
+size_t segmented_workspace_bytes(int B, int H, int P);
+cudaError_t launch_chunk_segmented(const void *q, const void *k, const void *v, const float *alpha, const float *b,
+                                   const float *w, const float *S0, void *o, float *S_T, int B, int T, int H,
+                                   int P, int L, void *workspace, cudaStream_t stream);
+
 // Chunkwise backward: prep, state and gradient launches.  workspace holds
 // chunk_bwd_workspace_floats(B, T, H, dk, dv) floats.
 size_t chunk_bwd_workspace_floats(int B, int T, int H, int dk, int dv);

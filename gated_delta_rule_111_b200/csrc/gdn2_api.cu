@@ -6,10 +6,6 @@
 #include "common.cuh"
 
 namespace gdn2 {
-cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *alpha, const void *b,
-                            const void *w, const float *S0, void *o, float *S_T, int nseq, int T, int H,
-                            const int *cu_seqlens, bool logits, cudaStream_t stream);
-bool chunk_tc_supported(int dk, int dv, gdn2_dtype dt);
 void set_wait_limit(long long cycles);
 cudaError_t read_device_error(unsigned int *value, bool clear);
 }  // namespace gdn2
@@ -92,7 +88,7 @@ gdn2_status gdn2_device_error(unsigned int *code, int clear) {
 static gdn2_status chunk_fwd_common(const void *q, const void *k, const void *v, const float *alpha,
                                     const float *b, const float *w, const int *cu, const float *S0, void *o,
                                     float *S_T, int nseq, int T, int H, int d_k, int d_v, gdn2_dtype dt,
-                                    void *stream) {
+                                    void *stream, bool launch = true) {
     g_last_error[0] = 0;
     gdn2_status st = check_common(nseq, H, d_k, d_v, dt);
     if (st != GDN2_OK) return st;
@@ -137,6 +133,7 @@ static gdn2_status chunk_fwd_common(const void *q, const void *k, const void *v,
             return fail(GDN2_ERR_INVALID_ARG, "%s", "an output overlaps cu_seqlens");
     }
 
+    if (!launch) return GDN2_OK;
     cudaError_t err;
     if (gdn2::chunk_tc_supported(d_k, d_v, dt))
         err = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, nseq, T, H, cu, false, s);
@@ -158,6 +155,124 @@ gdn2_status gdn2_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
     if (!cu_seqlens && N > 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "null pointer: cu_seqlens");
     return chunk_fwd_common(q, k, v, alpha, b, w, reinterpret_cast<const int *>(cu_seqlens), S0, o, S_T, N, T_total,
                             H, d_k, d_v, dt, stream);
+}
+
+}  // extern "C"
+
+namespace {
+// Segments for gdn2_chunk_fwd_segmented: requested > 1 is capped at the number
+// of 64-token chunks; 0 picks the count with the least estimated time, in
+// chunk steps of one CTA per SM: 2 B H CTAs walk every chunk in one pass, or
+// 4 B H (P - 1) and then 2 B H P CTAs walk ceil(chunks / P) chunks each, in
+// waves of `sms` CTAs; each wave costs about 2 chunk steps more (start-up and
+// drain) and each of the P - 1 combine steps about 1.3 (both measured on a
+// B200 with the long workload, T = 65,573 and 16 heads, for P from 1 to 54).
+// Segments are L = ceil(chunks / P) chunks long; P is then ceil(T / L).
+void resolve_segments(int B, int T, int H, int d_k, int d_v, gdn2_dtype dt, int requested, int sms, int *P,
+                      int *L) {
+    *P = 1;
+    *L = T;
+    const long long nch = ((long long)T + 63) / 64;
+    if (!gdn2::chunk_tc_supported(d_k, d_v, dt) || nch <= 1 || requested == 1 || B <= 0 || H <= 0) return;
+    auto waves = [&](long long ctas) { return (ctas + sms - 1) / sms; };
+    long long best_p = 1;
+    if (requested > 1) {
+        best_p = requested < nch ? requested : nch;
+    } else {
+        // tenths of a chunk step
+        const long long bh = (long long)B * H, one = waves(2 * bh) * (nch + 2) * 10;
+        long long best = one;
+        for (long long p = 2; p <= 64 && p <= nch; ++p) {
+            const long long cost =
+                (waves(4 * bh * (p - 1)) + waves(2 * bh * p)) * ((nch + p - 1) / p + 2) * 10 + 13 * (p - 1);
+            if (cost < best) {
+                best = cost;
+                best_p = p;
+            }
+        }
+        if (best * 10 > one * 9) best_p = 1;     // not worth the three passes
+    }
+    if (best_p <= 1) return;
+    const long long lc = (nch + best_p - 1) / best_p;
+    *L = (int)(lc * 64);
+    *P = (int)((T + *L - 1) / *L);
+    if (*P <= 1) {
+        *P = 1;
+        *L = T;
+    }
+}
+
+int current_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        return 0;
+    }
+    return sms;
+}
+}  // namespace
+
+extern "C" {
+
+size_t gdn2_chunk_fwd_segmented_workspace_size(int B, int T, int H, int d_k, int d_v, int segments) {
+    if (B <= 0 || T <= 0 || H <= 0 || segments < 0) return 0;
+    const int sms = segments == 0 ? current_sms() : 1;
+    if (sms <= 0) return 0;
+    int P = 1, L = T;
+    resolve_segments(B, T, H, d_k, d_v, GDN2_BF16, segments, sms, &P, &L);
+    return gdn2::segmented_workspace_bytes(B, H, P);
+}
+
+int gdn2_chunk_fwd_segments(int B, int T, int H, int d_k, int d_v, int segments) {
+    if (B <= 0 || T <= 0 || H <= 0 || segments < 0) return 1;
+    const int sms = segments == 0 ? current_sms() : 1;
+    if (sms <= 0) return 1;
+    int P = 1, L = T;
+    resolve_segments(B, T, H, d_k, d_v, GDN2_BF16, segments, sms, &P, &L);
+    return P;
+}
+
+gdn2_status gdn2_chunk_fwd_segmented(const void *q, const void *k, const void *v, const float *alpha, const float *b,
+                                     const float *w, const float *S0, void *o, float *S_T, int B, int T, int H,
+                                     int d_k, int d_v, gdn2_dtype dt, int segments, void *workspace,
+                                     size_t workspace_bytes, void *stream) {
+    g_last_error[0] = 0;
+    if (segments < 0) return fail(GDN2_ERR_INVALID_ARG, "%s", "negative segments");
+    if (segments > 1 && !gdn2::chunk_tc_supported(d_k, d_v, dt))
+        return fail(GDN2_ERR_UNSUPPORTED, "%s", "segments > 1 need BF16 q/k/v with d_k = d_v = 128");
+    int P = 1, L = T;
+    if (B > 0 && T > 0 && H > 0) {
+        const int sms = segments == 0 ? current_sms() : 1;
+        if (sms <= 0) return fail(GDN2_ERR_CUDA, "%s", "gdn2_chunk_fwd_segmented: no current CUDA device");
+        resolve_segments(B, T, H, d_k, d_v, dt, segments, sms, &P, &L);
+    }
+    if (P <= 1) return gdn2_chunk_fwd(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, dt, stream);
+    gdn2_status st = chunk_fwd_common(q, k, v, alpha, b, w, nullptr, S0, o, S_T, B, T, H, d_k, d_v, dt, stream,
+                                      false);
+    if (st != GDN2_OK) return st;
+    if ((long long)B * P > (1 << 20)) return fail(GDN2_ERR_UNSUPPORTED, "%s", "too many segments in all");
+    if ((long long)B * T >= (1ll << 31)) return fail(GDN2_ERR_UNSUPPORTED, "%s", "B * T must be below 2^31");
+    const size_t need = gdn2::segmented_workspace_bytes(B, H, P);
+    if (!workspace) return fail(GDN2_ERR_INVALID_ARG, "%s", "null pointer: workspace");
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(GDN2_ERR_INVALID_ARG, "%s", "workspace not 256-byte aligned");
+    if (workspace_bytes < need) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "gdn2_chunk_fwd_segmented: workspace of %zu bytes, %zu needed for %d segments", workspace_bytes, need,
+                 P);
+        return GDN2_ERR_INVALID_ARG;
+    }
+    const size_t tok = (size_t)B * T * H, state_bytes = (size_t)B * H * d_k * d_v * sizeof(float);
+    const void *bufs[9] = {q, k, v, alpha, b, w, o, S0, S_T};
+    const char *names[9] = {"q", "k", "v", "alpha", "b", "w", "o", "S0", "S_T"};
+    const size_t bytes[9] = {tok * d_k * 2, tok * d_k * 2, tok * d_v * 2, tok * d_k * 4, tok * d_k * 4,
+                             tok * d_v * 4, tok * d_v * 2, state_bytes,   state_bytes};
+    for (int i = 0; i < 9; ++i)
+        if (overlaps(workspace, need, bufs[i], bytes[i])) return fail(GDN2_ERR_INVALID_ARG, "workspace overlaps %s", names[i]);
+    cudaError_t err = gdn2::launch_chunk_segmented(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, P, L, workspace,
+                                                   static_cast<cudaStream_t>(stream));
+    return cuda_status(err, "gdn2_chunk_fwd_segmented launch");
 }
 
 size_t gdn2_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v) {

@@ -121,6 +121,55 @@ gdn2_status gdn2_chunk_fwd_varlen(const void *q, const void *k, const void *v,
                                   gdn2_dtype dt, void *stream);
 
 /*
+ * Chunkwise prefill of B sequences of T tokens, with each sequence cut into P
+ * segments processed in parallel — for few long sequences, where the plain call
+ * runs one serial chain per (sequence, head).  Same arguments and result as
+ * gdn2_chunk_fwd (up to rounding: the state crosses segment boundaries through
+ * an FP32 matrix product instead of the chunk loop).
+ *
+ * The recurrence is affine in the state ("Independent decisions on two axes":
+ * S_t = (I - k_t e_t^T) diag(alpha_t) S_{t-1} + k_t z_t^T), so over a segment
+ * S_end = M S_start + C, with C the end state from a zero start and M the end
+ * state from the identity with z = 0.  The call runs the chunk kernel over
+ * segments 0 .. P-2 twice (C and M), chains S_start(s+1) = M_s S_start(s) + C_s,
+ * then runs every segment from its start state: about three times the
+ * sequential work on up to 3 P times as many SMs.
+ *
+ *   segments   0: chosen from the shape and the current device's SM count (1 —
+ *              the plain call — unless fewer chunk steps per SM result);
+ *              n >= 1: n segments (capped at the number of 64-token chunks).
+ *              Segments are whole chunks long, the last one shorter.
+ *   workspace  DEVICE, caller-owned, 256-byte aligned, at least
+ *              gdn2_chunk_fwd_segmented_workspace_size(B, T, H, d_k, d_v,
+ *              segments) bytes (0 when the call resolves to one segment, in
+ *              which case workspace may be NULL); contents on entry do not
+ *              matter; must not overlap any argument.
+ *
+ * More than one segment needs BF16 with d_k = d_v = 128 (the tensor-core path):
+ * GDN2_ERR_UNSUPPORTED otherwise (segments = 0 or 1 run the plain call for any
+ * supported shape).  A workspace that is NULL, misaligned or too small is
+ * GDN2_ERR_INVALID_ARG.  Five launches on the stream; nothing is allocated.
+ * The workspace must stay untouched until the stream reaches the end of the call.
+ */
+gdn2_status gdn2_chunk_fwd_segmented(const void *q, const void *k, const void *v,
+                                     const float *alpha, const float *b, const float *w,
+                                     const float *S0, void *o, float *S_T,
+                                     int B, int T, int H, int d_k, int d_v,
+                                     gdn2_dtype dt, int segments,
+                                     void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
+/* Workspace bytes of gdn2_chunk_fwd_segmented for these arguments (segments = 0
+ * resolves against the current device; 0 if there is none or the call needs no
+ * workspace).  Host-only, no device memory touched. */
+size_t gdn2_chunk_fwd_segmented_workspace_size(int B, int T, int H, int d_k, int d_v,
+                                               int segments);
+
+/* The number of segments gdn2_chunk_fwd_segmented would use (BF16 assumed;
+ * 1 means the plain call).  Host-only. */
+int gdn2_chunk_fwd_segments(int B, int T, int H, int d_k, int d_v, int segments);
+
+/*
  * Chunkwise prefill from pre-activation logits, with the input preparation fused
  * into the tensor-core kernel ("Token processing and parallel training": the query
  * and key paths end in SiLU and L2 normalisation, the value path in SiLU;

@@ -209,3 +209,47 @@ def test_output_gate_host_checks(lib):
     # y partially overlapping o is refused; exact aliasing would be allowed
     assert lib.gdn2_output_gate(A16, A16 * 2, A16 * 3, c(1e-6), A16 + 16, 1, 4, 2, 128, BF16, None) == g.GDN2_ERR_INVALID_ARG
     assert b"overlaps" in lib.gdn2_last_error()
+
+
+WS = 0x10000000        # a fake, 256-byte aligned workspace address, clear of the fake inputs
+
+
+def _seg(lib, segments=3, ws=WS, ws_bytes=None, dt=BF16, B=1, T=300, H=1, o=A16 * 64):
+    P = ctypes.c_void_p
+    if ws_bytes is None:
+        ws_bytes = lib.gdn2_chunk_fwd_segmented_workspace_size(B, T, H, 128, 128, max(segments, 0))
+    return lib.gdn2_chunk_fwd_segmented(P(A16), P(A16), P(A16), P(A16), P(A16), P(A16), None, P(o), None, B, T, H,
+                                        128, 128, dt, segments, P(ws), ws_bytes, None)
+
+
+def test_segmented_host_checks(lib):
+    """Segment counts, the workspace size formula and every host-side refusal (each call below
+    fails validation; none reaches a launch)."""
+    assert lib.gdn2_chunk_fwd_segments(1, 65573, 16, 128, 128, 3) == 3   # 1,025 chunks: 342 per segment
+    assert lib.gdn2_chunk_fwd_segments(3, 130, 2, 128, 128, 8) == 3      # capped at the 3 chunks
+    assert lib.gdn2_chunk_fwd_segments(1, 64, 2, 128, 128, 8) == 1       # one chunk: the plain call
+    assert lib.gdn2_chunk_fwd_segments(1, 1000, 1, 128, 128, 1) == 1
+    assert lib.gdn2_chunk_fwd_segments(1, 1000, 1, 64, 64, 4) == 1       # not the tensor-core shape
+    state = 128 * 128 * 4
+    # token ranges of both launches (256-byte aligned), then C and M of segments 0 .. P-2 and every
+    # segment's start state
+    assert lib.gdn2_chunk_fwd_segmented_workspace_size(1, 65573, 16, 128, 128, 3) == \
+        256 + 256 + 2 * 2 * 16 * state + 3 * 16 * state
+    assert lib.gdn2_chunk_fwd_segmented_workspace_size(1, 1000, 1, 128, 128, 1) == 0
+    need = lib.gdn2_chunk_fwd_segmented_workspace_size(1, 300, 1, 128, 128, 3)
+    assert need == 256 + 256 + 4 * state + 3 * state
+    assert _seg(lib, segments=-1) == g.GDN2_ERR_INVALID_ARG
+    assert _seg(lib, dt=FP32) == g.GDN2_ERR_UNSUPPORTED
+    assert _seg(lib, ws_bytes=need - 256) == g.GDN2_ERR_INVALID_ARG
+    assert b"workspace" in lib.gdn2_last_error()
+    assert _seg(lib, ws=None) == g.GDN2_ERR_INVALID_ARG
+    assert _seg(lib, ws=WS + 16) == g.GDN2_ERR_INVALID_ARG                 # not 256-byte aligned
+    assert _seg(lib, ws=A16 * 2) == g.GDN2_ERR_INVALID_ARG                 # overlaps the inputs
+    assert b"overlaps" in lib.gdn2_last_error()
+    assert _seg(lib, o=A16) == g.GDN2_ERR_INVALID_ARG                      # o overlaps the inputs
+
+
+def test_segmented_binding_refuses_cpu_tensors():
+    x = torch.zeros(1, 4, 1, 128)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdn2_chunk_fwd_segmented(x, x, x, x, x, x)

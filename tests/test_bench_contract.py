@@ -94,7 +94,7 @@ def test_reference_arm_prints_the_same_config():
 
 def test_backward_entry(capsys):
     args = argparse.Namespace(steps=20, warmup=5, no_cpu_baseline=True, cpu_budget=1.0)
-    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), float("nan"), 2.0)
+    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), (float("nan"), float("nan"), 1), 2.0)
     d = json.loads(capsys.readouterr().out.strip())
     bw = d["backward"]
     P = bench.PREFILL
@@ -102,11 +102,22 @@ def test_backward_entry(capsys):
     # 4,864 B per token-head (q,k,v,dO bf16 + alpha,b,w fp32 in; dq,dk,dv bf16 + dalpha,db,dw fp32 out)
     assert bench.backward_bytes(1, 1, 1, 128, 128) == 4864 + 128 * 128 * 4
     assert bw["roofline"]["achieved"] == pytest.approx(bench.backward_bytes(4, 4096, 16, 128, 128) / 2.0e-3 / 1e9)
+    assert bw["launches_per_call"] == 5
+
+
+def test_long_ragged_entry(capsys):
+    """The long workload reports the segmented call (with its segment count) and the sequential one."""
+    args = argparse.Namespace(steps=20, warmup=5, no_cpu_baseline=True, cpu_budget=1.0)
+    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), (7.3, 4.9, 3))
+    lr = json.loads(capsys.readouterr().out.strip())["long_ragged"]
+    assert lr["ms_per_call"] == pytest.approx(4.9) and lr["ms_per_call_sequential"] == pytest.approx(7.3)
+    assert lr["segments"] == 3
+    assert lr["tokens_per_s"] == pytest.approx(bench.LONG["T"] / 4.9e-3)
 
 
 def test_logits_entry(capsys):
     args = argparse.Namespace(steps=20, warmup=5, no_cpu_baseline=True, cpu_budget=1.0)
-    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), float("nan"), float("nan"), 0.4)
+    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), (float("nan"), float("nan"), 1), float("nan"), 0.4)
     d = json.loads(capsys.readouterr().out.strip())
     lg = d["prefill_logits"]
     # six BF16 logit tensors in, BF16 o out: 1,792 B per token-head at d = 128
@@ -117,7 +128,7 @@ def test_logits_entry(capsys):
 
 def test_output_gate_entry(capsys):
     args = argparse.Namespace(steps=20, warmup=5, no_cpu_baseline=True, cpu_budget=1.0)
-    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), float("nan"), float("nan"), float("nan"), 0.04)
+    bench.report(args, 1, 0, 0.5, 12.0, 1, 1, 0.085, _Clocks(), (float("nan"), float("nan"), 1), float("nan"), float("nan"), 0.04)
     d = json.loads(capsys.readouterr().out.strip())
     og = d["output_gate"]
     # o and g read, y written, BF16: 768 B per token-head at d_v = 128
