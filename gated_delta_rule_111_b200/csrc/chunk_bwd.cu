@@ -27,7 +27,7 @@
 // log-decays are kept base 2 and as compensated (hi, lo) pairs, so a difference
 // g_t - g_s keeps its own precision however large |g| has grown in the chunk.
 //
-// Four launches on the caller's stream.  Everything that does not depend on the
+// Five launches on the caller's stream.  Everything that does not depend on the
 // carried state is computed for all chunks in parallel first, so the serial part
 // is two matrix products per chunk and direction:
 //   prep   grid (chunk, sequence x head): A and P from differences of logs, T by
