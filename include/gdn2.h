@@ -12,10 +12,12 @@
  *     S_t  = Sbar + k_t (z - r)^T         delta write
  *     o_t  = S_t^T q_t                    output from the state after this token's update
  *
- * Two entry points compute exactly this, in the two execution modes the pages
- * describe ("Token processing and parallel training": chunkwise WY with 64-token
- * chunks for training/prefill; the mindpattern.ai DeltaNet trail: a fused
- * recurrent mode for decode, with identical mathematics).
+ * The prefill entry points (gdn2_chunk_fwd and its packed, segmented and
+ * from-logits forms) and the decode step compute exactly this, in the two
+ * execution modes the pages describe ("Token processing and parallel training":
+ * chunkwise WY with 64-token chunks for training/prefill; the mindpattern.ai
+ * DeltaNet trail: a fused recurrent mode for decode, with identical
+ * mathematics).  gdn2_chunk_bwd gives the gradients of the prefill.
  *
  * Conventions shared by every call
  *   - All pointers are DEVICE pointers, 16-byte aligned, to dense row-major
