@@ -7,6 +7,8 @@ device these functions raise.
 
 Functions (same names as the C ABI):
   gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, ...)  -> (o, S_T)   chunkwise prefill
+  gdn2_chunk_fwd_from_host(q, k, v, alpha, b, w, S0=None, ...)
+                                                      -> (o, S_T)   the same from pinned host tensors, streamed
   gdn2_chunk_fwd_varlen(q, k, v, alpha, b, w, cu_seqlens, S0=None, ...)
                                                       -> (o, S_T)   packed variable-length batch
   gdn2_chunk_fwd_segmented(q, k, v, alpha, b, w, S0=None, segments=0, ...)
@@ -30,7 +32,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_segmented", "gdn2_chunk_fwd_segmented_workspace_size",
+__all__ = ["gdn2_chunk_fwd", "gdn2_chunk_fwd_from_host", "gdn2_chunk_fwd_varlen", "gdn2_chunk_fwd_segmented", "gdn2_chunk_fwd_segmented_workspace_size",
            "gdn2_chunk_fwd_segments", "gdn2_chunk_fwd_logits", "gdn2_output_gate", "gdn2_recurrent_step", "gdn2_chunk_bwd",
            "gdn2_chunk_bwd_workspace_size", "gdn2_chunk_bwd_noalloc", "gdn2_device_error", "gdn2_set_wait_limit", "library_path",
            "load_library", "exported_symbols",
@@ -184,6 +186,82 @@ def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0=None, *, o=None, S_T=None, output_fi
     with torch.cuda.device(dev):
         _check(lib.gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
                                   _ptr(S_T), B, T, H, dk, dv, code, _stream(stream, dev)))
+    return o, S_T
+
+
+_copy_streams = {}
+
+
+def _streams(device):
+    """Two side streams per device (host-to-device and device-to-host copies), created once."""
+    key = device.index
+    if key not in _copy_streams:
+        _copy_streams[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
+    return _copy_streams[key]
+
+
+def gdn2_chunk_fwd_from_host(q, k, v, alpha, b, w, S0=None, *, device=None, work=None, o=None, S_T=None,
+                             piece_tokens=None, stream=None):
+    """Chunkwise prefill from host tensors, arguments as gdn2_chunk_fwd but in (pinned) CPU memory;
+    returns host (o, S_T).  The batch is streamed in pieces of ``piece_tokens`` tokens of one
+    sequence (rounded down to a multiple of the 64-token chunk; None: whole sequences, the
+    fastest on the 4 x 4096 x 16 workload, where smaller pieces add more enqueue overhead than
+    they save at the tail): a piece's inputs go to the device on one copy
+    stream, its prefill (a gdn2_chunk_fwd call on ``stream``, started from the state the previous
+    piece of the sequence left) runs as soon as they have arrived, and its outputs come back on a
+    second copy stream while the next piece is copied in.  Pieces are whole chunks, so the result
+    equals one call over the batch bit for bit (unless a very strong decay makes the kernel cut a
+    chunk short, which moves later chunk boundaries; the result is then equally exact, to
+    rounding).
+
+    ``work``: dict of device tensors q, k, v, alpha, b, w (and S0 when given), o, S_T with the
+    inputs' shapes, reused across calls (allocated here when None).  ``o`` / ``S_T``: host output
+    tensors (pinned; allocated here when None).  On return every copy and launch is enqueued and
+    ``stream`` waits for the last of them; host outputs are valid after it synchronises."""
+    if q.device.type != "cpu":
+        raise ValueError("gdn2_chunk_fwd_from_host takes host tensors")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    names = ("q", "k", "v", "alpha", "b", "w")
+    src = dict(zip(names, (q, k, v, alpha, b, w)))
+    if work is None:
+        work = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in src.items()}
+        if S0 is not None:
+            work["S0"] = torch.empty(S0.shape, dtype=S0.dtype, device=dev)
+        work["o"] = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+        work["S_T"] = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype).pin_memory()
+    if S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32).pin_memory()
+    tp = max(T, 1) if piece_tokens is None else max(64, (int(piece_tokens) // 64) * 64)
+    with torch.cuda.device(dev):
+        main = torch.cuda.current_stream(dev) if stream is None else stream
+        s_in, s_out = _streams(dev)
+        s_in.wait_stream(main)
+        s_out.wait_stream(main)
+        for i in range(B):
+            if S0 is not None:
+                with torch.cuda.stream(s_in):
+                    work["S0"][i].copy_(S0[i], non_blocking=True)
+            state = work["S0"][i:i + 1] if S0 is not None else None
+            for t0 in range(0, max(T, 1), tp):
+                t1 = min(T, t0 + tp)
+                with torch.cuda.stream(s_in):
+                    for n in names:
+                        work[n][i, t0:t1].copy_(src[n][i, t0:t1], non_blocking=True)
+                main.wait_stream(s_in)
+                piece = {n: work[n][i:i + 1, t0:t1] for n in names}
+                gdn2_chunk_fwd(*(piece[n] for n in names), state, o=work["o"][i:i + 1, t0:t1],
+                               S_T=work["S_T"][i:i + 1], stream=main)
+                state = work["S_T"][i:i + 1]       # the next piece starts where this one ended
+                s_out.wait_stream(main)
+                with torch.cuda.stream(s_out):
+                    o[i, t0:t1].copy_(work["o"][i, t0:t1], non_blocking=True)
+            with torch.cuda.stream(s_out):
+                S_T[i].copy_(work["S_T"][i], non_blocking=True)
+        main.wait_stream(s_out)
     return o, S_T
 
 
