@@ -231,6 +231,9 @@ def gdn2_chunk_fwd_from_host(q, k, v, alpha, b, w, S0=None, *, device=None, work
             work["S0"] = torch.empty(S0.shape, dtype=S0.dtype, device=dev)
         work["o"] = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
         work["S_T"] = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    missing = [n for n in list(src) + (["S0"] if S0 is not None else []) + ["o", "S_T"] if n not in work]
+    if missing:
+        raise ValueError(f"work: missing device buffers {missing}")
     if o is None:
         o = torch.empty((B, T, H, dv), dtype=q.dtype).pin_memory()
     if S_T is None:
